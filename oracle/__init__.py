@@ -1,0 +1,185 @@
+"""Oracle for the DLRMv1 sparse/interaction stage (numpy front end).
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only callers. The product path never
+imports this package, and this package imports nothing from the product.
+
+The arithmetic lives in ``dlrm_oracle.c`` (plain C loops, built with gcc -O2,
+no fast-math, no FMA contraction); this module only compiles it, loads it with
+ctypes and marshals numpy arrays. What each function follows on the pages
+(luminal compare main...vanilla-pytorch):
+
+* :meth:`Oracle.embbag_sum_multi` -- embedding_bag.rs, module doc comment and
+  the multi-table section doc comment (pooled sum over K tables).
+* :meth:`Oracle.interact_lower_tri` -- dlrm_interact.rs, module doc comment
+  (the strict-lower-triangle dot products) and the stacked-kernel doc comment
+  (feature 0 = dense vector, features 1..N = pooled embeddings).
+* :meth:`Oracle.pair_list` -- dlrm_interact.rs, pair-table comment: row-major
+  over i then j, the torch.tril_indices(F, F, -1) order.
+
+Every function is pinned by ``tests/test_oracle_pins.py`` to facts fixed by
+the pages and by mathematics, not by this code.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "dlrm_oracle.c")
+LIBRARY = os.path.join(_HERE, "liboracle.so")
+
+OK = 0
+BAD_ARG = 1
+BAD_OFFSETS = 2
+INDEX_OOB = 3
+
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math"]
+
+
+class OracleError(RuntimeError):
+    """The oracle rejected its input; ``code`` is one of the codes above."""
+
+    def __init__(self, code: int, what: str):
+        super().__init__(f"oracle {what} rejected its input (code {code})")
+        self.code = code
+
+
+def compile_source(src: str, lib: str) -> str:
+    """Compile one C source file into a shared library with the oracle's flags."""
+    tmp = lib + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, src])
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False) -> str:
+    """Compile ``dlrm_oracle.c`` into ``liboracle.so`` (if stale) and return its path."""
+    if (not force and os.path.exists(LIBRARY)
+            and os.path.getmtime(LIBRARY) >= os.path.getmtime(SOURCE)):
+        return LIBRARY
+    return compile_source(SOURCE, LIBRARY)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+class Oracle:
+    """The oracle's functions, bound to one compiled copy of ``dlrm_oracle.c``."""
+
+    def __init__(self, libpath: str):
+        lib = ctypes.CDLL(libpath)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        lib.oracle_embbag_sum_multi.argtypes = [P, P, P, P, I, I, I, I, P, P, P]
+        lib.oracle_embbag_sum_multi.restype = I
+        lib.oracle_interact_lower_tri.argtypes = [P, P, I, I, I, P, I, P, P]
+        lib.oracle_interact_lower_tri.restype = I
+        lib.oracle_pair_list.argtypes = [I, P, P]
+        lib.oracle_pair_list.restype = ctypes.c_int64
+        self.lib = lib
+        self.path = libpath
+
+    def embbag_sum_multi(self, weights: Sequence[np.ndarray], indices: np.ndarray,
+                         offsets: np.ndarray, B: int, L: int, *, with_f64: bool = False):
+        """Pooled sums ``(B, F, D)`` f32 of F EmbeddingBag(sum) tables.
+
+        ``weights[k]`` is ``(rows_k, D)`` f32; ``indices`` is ``(F, B*L)``
+        int32 (table-major); ``offsets`` is ``(F, B)`` int32. With
+        ``with_f64`` it also returns the fp64 sums and the per-output sum of
+        ``|w|`` over the bag.
+        """
+        F = len(weights)
+        ws = [_f32(w) for w in weights]
+        D = int(ws[0].shape[1])
+        ptrs = (ctypes.c_void_p * F)(*[w.ctypes.data for w in ws])
+        rows = np.array([w.shape[0] for w in ws], dtype=np.int64)
+        idx = np.ascontiguousarray(indices, dtype=np.int32).reshape(F, -1)
+        off = np.ascontiguousarray(offsets, dtype=np.int32).reshape(F, B)
+        out = np.empty((B, F, D), dtype=np.float32)
+        o64 = np.empty((B, F, D), dtype=np.float64) if with_f64 else None
+        oab = np.empty((B, F, D), dtype=np.float64) if with_f64 else None
+        rc = self.lib.oracle_embbag_sum_multi(ctypes.cast(ptrs, ctypes.c_void_p), _ptr(rows),
+                                              _ptr(idx), _ptr(off), B, F, L, D, _ptr(out),
+                                              _ptr(o64), _ptr(oab))
+        if rc != OK:
+            raise OracleError(rc, "embbag_sum_multi")
+        return (out, o64, oab) if with_f64 else out
+
+    def interact_lower_tri(self, dense: np.ndarray, emb: np.ndarray, *,
+                           concat_dense: bool = False, with_f64: bool = False):
+        """Strict-lower-triangle dots over ``[dense, emb_0 .. emb_{F-1}]``.
+
+        ``dense`` is ``(B, D)``, ``emb`` is ``(B, F, D)``. Returns ``(B, P)``
+        f32 (``(B, D+P)`` with ``concat_dense``), ``P = (F+1)F/2``. With
+        ``with_f64`` it also returns the unrounded fp64 dots and the error
+        scale ``S_ij = sum_d |v_i v_j|``.
+        """
+        dn = _f32(dense)
+        em = _f32(emb)
+        B, F, D = em.shape
+        P = (F + 1) * F // 2
+        out = np.empty((B, D + P if concat_dense else P), dtype=np.float32)
+        o64 = np.empty((B, P), dtype=np.float64) if with_f64 else None
+        bnd = np.empty((B, P), dtype=np.float64) if with_f64 else None
+        rc = self.lib.oracle_interact_lower_tri(_ptr(dn), _ptr(em), B, F, D, _ptr(out),
+                                                1 if concat_dense else 0, _ptr(o64), _ptr(bnd))
+        if rc != OK:
+            raise OracleError(rc, "interact_lower_tri")
+        return (out, o64, bnd) if with_f64 else out
+
+    def sparse_interact(self, weights, indices, offsets, dense, B: int, L: int, *,
+                        concat_dense: bool = False, with_bound: bool = False):
+        """The whole stage: pooled ``(B,F,D)`` and the interaction row per sample."""
+        pooled = self.embbag_sum_multi(weights, indices, offsets, B, L)
+        if with_bound:
+            inter, _, bound = self.interact_lower_tri(dense, pooled, concat_dense=concat_dense,
+                                                      with_f64=True)
+            return pooled, inter, bound
+        return pooled, self.interact_lower_tri(dense, pooled, concat_dense=concat_dense)
+
+    def pair_list(self, nf: int):
+        """``(i, j)`` of the strict lower triangle of ``nf x nf``, nested-loop order."""
+        n = nf * (nf - 1) // 2
+        pi = np.empty(n, dtype=np.int32)
+        pj = np.empty(n, dtype=np.int32)
+        got = self.lib.oracle_pair_list(nf, _ptr(pi), _ptr(pj))
+        if got != n:
+            raise OracleError(-1, "pair_list")
+        return pi, pj
+
+
+_default = None
+
+
+def default() -> Oracle:
+    """The oracle built from ``dlrm_oracle.c`` as committed."""
+    global _default
+    if _default is None:
+        _default = Oracle(build())
+    return _default
+
+
+def embbag_sum_multi(*a, **k):
+    return default().embbag_sum_multi(*a, **k)
+
+
+def interact_lower_tri(*a, **k):
+    return default().interact_lower_tri(*a, **k)
+
+
+def sparse_interact(*a, **k):
+    return default().sparse_interact(*a, **k)
+
+
+def pair_list(*a, **k):
+    return default().pair_list(*a, **k)

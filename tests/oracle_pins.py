@@ -1,0 +1,356 @@
+"""Pins of the oracle: facts fixed by the pages and by mathematics.
+
+Each ``pin_*`` function takes an :class:`oracle.Oracle` and raises on the first
+violated fact. They are collected by ``test_oracle_pins.py`` (against the
+committed oracle) and by ``test_oracle_mutants.py`` (against copies of the
+oracle with a planted mistake, each of which must fail at least one pin).
+
+No expected value here is produced by the oracle itself: each comes from the
+pages (``tests/golden``), a closed form, a library routine (numpy, torch CPU in
+fp64), exact rational arithmetic, or an invariant that holds exactly.
+"""
+from __future__ import annotations
+
+import os
+import sys
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+U32 = 2.0 ** -24  # unit roundoff of f32
+
+
+def _golden_rows(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+def _fixed_offsets(F, B, L):
+    return np.broadcast_to((np.arange(B) * L).astype(np.int32), (F, B)).copy()
+
+
+def _rand_case(seed, B, F, N, D, L):
+    rng = np.random.default_rng(seed)
+    ws = [rng.normal(0.0, 0.1, size=(N, D)).astype(np.float32) for _ in range(F)]
+    idx = rng.integers(0, N, size=(F, B * L)).astype(np.int32)
+    dense = rng.normal(0.0, 1.0, size=(B, D)).astype(np.float32)
+    return ws, idx, _fixed_offsets(F, B, L), dense
+
+
+def _dyadic_table(rng, N, D):
+    # k/256 with |k| < 128: every sum of up to 2^16 such values is exact in f32
+    return (rng.integers(-127, 128, size=(N, D)) / 256.0).astype(np.float32)
+
+
+def _expect_code(fn, code):
+    from oracle import OracleError
+
+    try:
+        fn()
+    except OracleError as e:  # noqa: PERF203
+        assert e.code == code, f"expected oracle code {code}, got {e.code}"
+        return
+    raise AssertionError(f"oracle accepted an input it must reject (code {code})")
+
+
+# --------------------------------------------------------------------------- pairs
+
+def pin_pair_order_golden(orc):
+    """The first pairs the pages print, (1,0), (2,0), (2,1)."""
+    rows = _golden_rows("pair_order_head.txt")
+    for nf in (3, 4, 9, 33):
+        pi, pj = orc.pair_list(nf)
+        for p, i, j in rows:
+            assert (pi[int(p)], pj[int(p)]) == (int(i), int(j)), (nf, p)
+
+
+def pin_pair_count_golden(orc):
+    """528 dots at num_cat = 32 (F = 33 features), in both output layouts."""
+    kv = {k: int(v) for k, v in _golden_rows("pairs_at_num_cat_32.txt")}
+    F = kv["num_cat"]
+    assert F + 1 == kv["features"]
+    assert (kv["features"] - 1) // 2 == kv["reread_factor"]
+    dense = np.ones((2, 3), np.float32)
+    emb = np.ones((2, F, 3), np.float32)
+    assert orc.interact_lower_tri(dense, emb).shape == (2, kv["pairs"])
+    assert orc.interact_lower_tri(dense, emb, concat_dense=True).shape == (2, 3 + kv["pairs"])
+    pi, _ = orc.pair_list(kv["features"])
+    assert len(pi) == kv["pairs"]
+
+
+def pin_pair_list_is_tril_indices(orc):
+    """The pair table equals numpy's tril_indices(nf, -1) for every nf up to 129."""
+    for nf in range(1, 130):
+        pi, pj = orc.pair_list(nf)
+        ri, rj = np.tril_indices(nf, -1)
+        assert np.array_equal(pi, ri) and np.array_equal(pj, rj), nf
+
+
+def pin_interaction_identifies_pairs(orc):
+    """With D=1 and feature m equal to the m-th prime, dot p is prime_i * prime_j.
+
+    The factorisation is unique, so this fixes which two features (dense first,
+    then tables in order) every output column multiplies.
+    """
+    primes = [2, 3, 5, 7, 11, 13, 17, 19, 23, 29, 31, 37, 41, 43, 47, 53, 59, 61, 67, 71,
+              73, 79, 83, 89, 97, 101, 103, 107, 109, 113, 127, 131, 137]
+    for F in (1, 2, 5, 32):
+        B = 3
+        c = np.array(primes[: F + 1], dtype=np.float32)
+        dense = np.tile(c[0], (B, 1)).astype(np.float32) * np.arange(1, B + 1)[:, None]
+        emb = np.tile(c[1:], (B, 1))[:, :, None].astype(np.float32)
+        z = orc.interact_lower_tri(dense, emb)
+        ri, rj = np.tril_indices(F + 1, -1)
+        for b in range(B):
+            feat = np.concatenate([[c[0] * (b + 1)], c[1:]])
+            want = (feat[ri] * feat[rj]).astype(np.float32)
+            assert np.array_equal(z[b], want), (F, b)
+
+
+def pin_interaction_vs_torch_bmm(orc):
+    """Dots equal torch's cat -> bmm(T, T^T) -> tril gather, taken in fp64."""
+    for seed, (B, F, D) in enumerate([(3, 5, 7), (2, 1, 16), (4, 12, 33)]):
+        _, _, _, dense = _rand_case(seed, B, 1, 1, D, 1)
+        emb = np.random.default_rng(100 + seed).normal(0, 0.3, (B, F, D)).astype(np.float32)
+        T = torch.cat([torch.from_numpy(dense).double().unsqueeze(1),
+                       torch.from_numpy(emb).double()], dim=1)
+        Z = torch.bmm(T, T.transpose(1, 2))
+        li, lj = torch.tril_indices(F + 1, F + 1, -1)
+        ref = Z[:, li, lj].numpy()
+        z32, z64, bound = orc.interact_lower_tri(dense, emb, with_f64=True)
+        assert np.all(np.abs(z64 - ref) <= 1e-13 * bound + 1e-300), (B, F, D)
+        assert np.array_equal(z32, ref.astype(np.float32)) or \
+            np.all(np.abs(z32 - ref) <= U32 * np.abs(ref) + 1e-13 * bound)
+        # S_ij is the sum of |v_i v_j|, which bounds |z| and equals it for v_i = v_j
+        absT = T.abs()
+        Sref = torch.bmm(absT, absT.transpose(1, 2))[:, li, lj].numpy()
+        assert np.allclose(bound, Sref, rtol=1e-12, atol=0)
+
+
+def pin_interaction_exact_rational(orc):
+    """Brute force on tiny inputs with exact rationals: fp64 within gamma_D, f32 within 1 ulp."""
+    rng = np.random.default_rng(7)
+    B, F, D = 2, 3, 5
+    dense = rng.normal(0, 1, (B, D)).astype(np.float32)
+    emb = rng.normal(0, 1, (B, F, D)).astype(np.float32)
+    z32, z64, _ = orc.interact_lower_tri(dense, emb, with_f64=True)
+    for b in range(B):
+        feats = [dense[b]] + [emb[b, k] for k in range(F)]
+        p = 0
+        for i in range(1, F + 1):
+            for j in range(i):
+                prods = [Fraction(float(x)) * Fraction(float(y))
+                         for x, y in zip(feats[i], feats[j])]
+                exact = sum(prods)
+                # fp64 summation of D exact products: error <= D * 2^-53 * sum|prod|
+                bound64 = Fraction(D, 2 ** 53) * sum(abs(t) for t in prods)
+                assert abs(Fraction(float(z64[b, p])) - exact) <= bound64, (b, p)
+                ulp = np.spacing(np.float32(abs(float(exact)) or 1e-38))
+                assert abs(Fraction(float(z32[b, p])) - exact) <= Fraction(float(ulp)), (b, p)
+                p += 1
+
+
+def pin_concat_layout(orc):
+    """With concat, row b is [dense[b] | dots of b], both parts bit-exact."""
+    _, _, _, dense = _rand_case(3, 4, 1, 1, 6, 1)
+    emb = np.random.default_rng(4).normal(0, 1, (4, 3, 6)).astype(np.float32)
+    z = orc.interact_lower_tri(dense, emb)
+    zc = orc.interact_lower_tri(dense, emb, concat_dense=True)
+    assert zc.shape == (4, 6 + 6)
+    assert np.array_equal(zc[:, :6].view(np.uint32), dense.view(np.uint32))
+    assert np.array_equal(zc[:, 6:].view(np.uint32), z.view(np.uint32))
+
+
+def pin_scale_dense(orc):
+    """Doubling dense doubles exactly the dots that involve feature 0, nothing else."""
+    _, _, _, dense = _rand_case(5, 3, 1, 1, 9, 1)
+    emb = np.random.default_rng(6).normal(0, 1, (3, 4, 9)).astype(np.float32)
+    z = orc.interact_lower_tri(dense, emb)
+    z2 = orc.interact_lower_tri(dense * np.float32(2), emb)
+    _, rj = np.tril_indices(5, -1)
+    assert np.array_equal(z2[:, rj == 0], z[:, rj == 0] * np.float32(2))
+    assert np.array_equal(z2[:, rj != 0], z[:, rj != 0])
+
+
+# --------------------------------------------------------------------------- pooled sums
+
+def pin_embbag_vs_torch(orc):
+    """Pooled sums equal torch.nn.functional.embedding_bag(mode='sum') in fp64.
+
+    Covers ragged bags (offsets not a fixed stride), empty bags and tables with
+    different row counts.
+    """
+    rng = np.random.default_rng(11)
+    B, F, D, L = 6, 3, 5, 4
+    rows = [7, 13, 5]
+    ws = [rng.normal(0, 0.1, (rows[k], D)).astype(np.float32) for k in range(F)]
+    idx = np.stack([rng.integers(0, rows[k], B * L) for k in range(F)]).astype(np.int32)
+    offs = np.array([[0, 4, 8, 12, 16, 20],
+                     [0, 0, 3, 10, 10, 23],
+                     [0, 1, 2, 3, 24, 24]], dtype=np.int32)
+    out, o64, absum = orc.embbag_sum_multi(ws, idx, offs, B, L, with_f64=True)
+    for k in range(F):
+        ref = torch.nn.functional.embedding_bag(
+            torch.from_numpy(idx[k]).long(), torch.from_numpy(ws[k]).double(),
+            torch.from_numpy(offs[k]).long(), mode="sum").numpy()
+        assert np.allclose(o64[:, k, :], ref, rtol=1e-14, atol=1e-300), k
+        n_in_bag = np.diff(np.append(offs[k], B * L))
+        tol = (n_in_bag[:, None] * U32) * absum[:, k, :]
+        assert np.all(np.abs(out[:, k, :] - ref) <= tol), k
+
+
+def pin_embbag_sequential_order(orc):
+    """The f32 pooled sum accumulates from 0 in bag order, one rounding per add.
+
+    With rows 1.0 and 2^-24: in bag order [1, t, t] each add of t ties back to
+    1.0 (round half to even), so the sum is exactly 1.0; in order [t, t, 1] the
+    two small terms first make 2^-23 and the sum is 1 + 2^-23.
+    """
+    W = np.array([[1.0], [2.0 ** -24]], dtype=np.float32)
+    idx = np.array([[0, 1, 1, 1, 1, 0]], dtype=np.int32)
+    offs = np.array([[0, 3]], dtype=np.int32)
+    out = orc.embbag_sum_multi([W], idx, offs, 2, 3)
+    assert out[0, 0, 0] == np.float32(1.0)
+    assert out[1, 0, 0] == np.float32(1.0 + 2.0 ** -23)
+
+
+def pin_l_copies(orc):
+    """A bag of L copies of row r pools to exactly L * W[r] on dyadic tables."""
+    rng = np.random.default_rng(12)
+    for L in (1, 4, 20, 33):
+        N, D, B, F = 9, 6, 5, 2
+        ws = [_dyadic_table(rng, N, D) for _ in range(F)]
+        r = rng.integers(0, N, size=(F, B))
+        idx = np.repeat(r, L, axis=1).astype(np.int32)
+        out = orc.embbag_sum_multi(ws, idx, _fixed_offsets(F, B, L), B, L)
+        for k in range(F):
+            assert np.array_equal(out[:, k, :], ws[k][r[k]] * np.float32(L)), (L, k)
+
+
+def pin_one_hot_tables(orc):
+    """Row r of a one-hot table is e_(r mod D): pooled values are index counts.
+
+    The counts come from numpy's bincount and the dots from an integer einsum,
+    so both parts of the stage are checked exactly.
+    """
+    rng = np.random.default_rng(13)
+    B, F, N, D, L = 7, 4, 50, 8, 10
+    eye = np.eye(D, dtype=np.float32)
+    ws = [eye[np.arange(N) % D] for _ in range(F)]
+    idx = rng.integers(0, N, size=(F, B * L)).astype(np.int32)
+    pooled = orc.embbag_sum_multi(ws, idx, _fixed_offsets(F, B, L), B, L)
+    counts = np.zeros((B, F, D), dtype=np.int64)
+    for k in range(F):
+        for b in range(B):
+            counts[b, k] = np.bincount(idx[k, b * L:(b + 1) * L] % D, minlength=D)
+    assert np.array_equal(pooled, counts.astype(np.float32))
+    dense_i = rng.integers(-3, 4, size=(B, D))
+    z = orc.interact_lower_tri(dense_i.astype(np.float32), pooled)
+    feats = np.concatenate([dense_i[:, None, :], counts], axis=1)
+    gram = np.einsum("bid,bjd->bij", feats, feats)
+    ri, rj = np.tril_indices(F + 1, -1)
+    assert np.array_equal(z, gram[:, ri, rj].astype(np.float32))
+
+
+def pin_brute_force_tiny(orc):
+    """Tiny random case against exact rational sums (pooled) in plain Python."""
+    rng = np.random.default_rng(14)
+    B, F, N, D, L = 3, 2, 6, 4, 3
+    ws = [rng.normal(0, 0.1, (N, D)).astype(np.float32) for _ in range(F)]
+    idx = rng.integers(0, N, size=(F, B * L)).astype(np.int32)
+    out = orc.embbag_sum_multi(ws, idx, _fixed_offsets(F, B, L), B, L)
+    for b in range(B):
+        for k in range(F):
+            for d in range(D):
+                terms = [float(ws[k][idx[k, b * L + l], d]) for l in range(L)]
+                exact = sum(Fraction(t) for t in terms)
+                bound = Fraction(L) * Fraction(U32) * sum(abs(Fraction(t)) for t in terms)
+                assert abs(Fraction(float(out[b, k, d])) - exact) <= bound, (b, k, d)
+
+
+def pin_bag_permutation(orc):
+    """Permuting entries inside bags leaves dyadic pooled sums bit-identical."""
+    rng = np.random.default_rng(15)
+    B, F, N, D, L = 4, 3, 11, 5, 7
+    ws = [_dyadic_table(rng, N, D) for _ in range(F)]
+    idx = rng.integers(0, N, size=(F, B * L)).astype(np.int32)
+    perm = idx.reshape(F, B, L)[:, :, rng.permutation(L)].reshape(F, B * L)
+    offs = _fixed_offsets(F, B, L)
+    a = orc.embbag_sum_multi(ws, idx, offs, B, L)
+    b = orc.embbag_sum_multi(ws, np.ascontiguousarray(perm), offs, B, L)
+    assert np.array_equal(a, b)
+
+
+def pin_swap_tables(orc):
+    """Swapping two tables (with their indices) swaps their pooled slots and dots."""
+    ws, idx, offs, dense = _rand_case(16, 3, 3, 10, 4, 5)
+    pooled, inter = orc.sparse_interact(ws, idx, offs, dense, 3, 5)
+    ws2 = [ws[1], ws[0], ws[2]]
+    idx2 = np.ascontiguousarray(idx[[1, 0, 2]])
+    pooled2, inter2 = orc.sparse_interact(ws2, idx2, offs, dense, 3, 5)
+    assert np.array_equal(pooled2, pooled[:, [1, 0, 2], :])
+    # feature m of the swapped run is feature sigma(m) of the original
+    sigma = [0, 2, 1, 3]
+    ri, rj = np.tril_indices(4, -1)
+    col = {(int(i), int(j)): p for p, (i, j) in enumerate(zip(ri, rj))}
+    for p, (i, j) in enumerate(zip(ri, rj)):
+        a, b = sigma[i], sigma[j]
+        q = col[(max(a, b), min(a, b))]
+        assert np.array_equal(inter2[:, p], inter[:, q]), (i, j)
+
+
+def pin_empty_bags_are_positive_zero(orc):
+    """An empty bag (L = 0, or equal consecutive offsets) pools to +0.0."""
+    rng = np.random.default_rng(17)
+    ws = [rng.normal(0, 1, (4, 3)).astype(np.float32)]
+    out = orc.embbag_sum_multi(ws, np.zeros((1, 0), np.int32), np.zeros((1, 5), np.int32), 5, 0)
+    assert np.array_equal(out.view(np.uint32), np.zeros((5, 1, 3), np.uint32))
+    idx = np.array([[1, 2, 3, 0]], dtype=np.int32)
+    out = orc.embbag_sum_multi(ws, idx, np.array([[0, 2, 2, 4]], np.int32), 4, 1)
+    assert np.array_equal(out[1].view(np.uint32), np.zeros((1, 3), np.uint32))
+    assert np.array_equal(out[3].view(np.uint32), np.zeros((1, 3), np.uint32))
+    assert np.array_equal(out[2, 0], ws[0][3] + ws[0][0])
+
+
+def pin_rejects_bad_input(orc):
+    """Offsets out of order or range, indices outside [0, rows), bad shapes."""
+    from oracle import BAD_ARG, BAD_OFFSETS, INDEX_OOB
+
+    ws = [np.zeros((5, 2), np.float32), np.zeros((3, 2), np.float32)]
+    good_idx = np.array([[0, 1, 2, 3], [0, 1, 2, 0]], np.int32)
+    offs = _fixed_offsets(2, 2, 2)
+    orc.embbag_sum_multi(ws, good_idx, offs, 2, 2)
+    for bad in ([[2, 1], [0, 2]], [[-1, 2], [0, 2]], [[0, 5], [0, 2]], [[0, 2], [3, 2]]):
+        _expect_code(lambda: orc.embbag_sum_multi(ws, good_idx, np.array(bad, np.int32), 2, 2),
+                     BAD_OFFSETS)
+    for bad in ([[0, 1, 2, 5], [0, 1, 2, 0]], [[0, 1, 2, 3], [0, 3, 2, 0]],
+                [[0, -1, 2, 3], [0, 1, 2, 0]]):
+        _expect_code(lambda: orc.embbag_sum_multi(ws, np.array(bad, np.int32), offs, 2, 2),
+                     INDEX_OOB)
+    _expect_code(lambda: orc.embbag_sum_multi(ws, good_idx, offs, 2, -1), BAD_ARG)
+    dense = np.zeros((2, 2), np.float32)
+    _expect_code(lambda: orc.interact_lower_tri(dense, np.zeros((2, 257, 2), np.float32)),
+                 BAD_ARG)
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
+
+
+def run_all(orc) -> int:
+    """Run every pin; print the failures; return how many failed."""
+    failed = 0
+    for pin in ALL_PINS:
+        try:
+            pin(orc)
+        except Exception as e:  # noqa: BLE001 - a mutant may fail in any way
+            failed += 1
+            print(f"FAIL {pin.__name__}: {type(e).__name__}: {e}", file=sys.stderr)
+    return failed

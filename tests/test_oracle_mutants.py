@@ -1,0 +1,79 @@
+"""Planted mistakes in the oracle (CPU only) must each fail at least one pin.
+
+Every mutant below is a copy of ``oracle/dlrm_oracle.c`` with one plausible
+mistake -- a dropped term, a wrong sign, index or operand, a transposed layout,
+a missing check -- compiled with the oracle's flags into a temporary library.
+The pins of ``oracle_pins.py`` then run against it in a child process (a
+mutant may write out of bounds), which must report at least one failure. The
+unmodified source, compiled the same way, must pass every pin.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+TESTS = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(TESTS)
+
+MUTANTS = {
+    "pooled_drops_running_sum": [("acc = acc + w;", "acc = w;")],
+    "pooled_wrong_sign": [("acc = acc + w;", "acc = acc - w;")],
+    "pooled_skips_first_entry": [("for (int64_t t = s; t < e; ++t) {\n                    float w",
+                                  "for (int64_t t = s + 1; t < e; ++t) {\n                    float w")],
+    "pooled_layout_transposed": [("int64_t o = ((int64_t)b * F + k) * D + d;",
+                                  "int64_t o = ((int64_t)k * B + b) * D + d;")],
+    "pooled_all_tables_use_table0_indices": [("indices ? indices + (int64_t)k * seg : NULL",
+                                              "indices")],
+    "pooled_all_tables_use_weight0": [("const float* W = weights[k];",
+                                       "const float* W = weights[0];")],
+    "last_bag_ignores_segment_end": [("(int64_t)offsets[(int64_t)k * B + b + 1] : seg;",
+                                      "(int64_t)offsets[(int64_t)k * B + b + 1] : s + L;")],
+    "offsets_order_unchecked": [("if (s < 0 || s > e || e > seg)", "if (s < 0 || e > seg)")],
+    "index_bound_off_by_one": [("(int64_t)r >= rows[k]", "(int64_t)r > rows[k]")],
+    "dot_wrong_operand": [("(double)a[d] * (double)b[d]", "(double)a[d] * (double)a[d]")],
+    "dot_drops_first_term": [("for (int d = 0; d < D; ++d) {\n        double t",
+                              "for (int d = 1; d < D; ++d) {\n        double t")],
+    "dot_stores_abs_sum": [("z[p] = (float)s;", "z[p] = (float)m;")],
+    "features_in_reverse_table_order": [("emb + ((int64_t)b * F + (i - 1)) * D;",
+                                         "emb + ((int64_t)b * F + (F - i)) * D;")],
+    "pair_list_transposed": [("if (pi) pi[p] = i;", "if (pi) pi[p] = j;"),
+                             ("if (pj) pj[p] = j;", "if (pj) pj[p] = i;")],
+    "pairs_include_diagonal": [("for (int j = 0; j < i; ++j) {\n                const float* vj",
+                                "for (int j = 0; j <= i; ++j) {\n                const float* vj")],
+    "concat_drops_dense": [("row[d] = dense[(int64_t)b * D + d];", "row[d] = 0.0f;")],
+}
+
+_RUNNER = (
+    "import sys; sys.path[:0] = [{root!r}, {tests!r}]\n"
+    "import oracle, oracle_pins\n"
+    "sys.exit(min(100, oracle_pins.run_all(oracle.Oracle({lib!r}))))\n"
+)
+
+
+def _build_and_run(tmp_path, name, edits):
+    with open(oracle.SOURCE) as fh:
+        src = fh.read()
+    for old, new in edits:
+        assert src.count(old) == 1, f"mutant {name}: pattern must occur exactly once: {old!r}"
+        src = src.replace(old, new)
+    csrc = tmp_path / f"{name}.c"
+    csrc.write_text(src)
+    lib = str(tmp_path / f"lib{name}.so")
+    oracle.compile_source(str(csrc), lib)
+    code = _RUNNER.format(root=ROOT, tests=TESTS, lib=lib)
+    return subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                          timeout=300)
+
+
+def test_unmutated_copy_passes_every_pin(tmp_path):
+    r = _build_and_run(tmp_path, "control", [])
+    assert r.returncode == 0, r.stderr[-2000:]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_fails_a_pin(tmp_path, name):
+    r = _build_and_run(tmp_path, name, MUTANTS[name])
+    assert r.returncode != 0, f"mutant {name} passed every pin:\n{r.stderr[-2000:]}"
