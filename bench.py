@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark of the fused DLRMv1 sparse/interaction stage on B200.
+
+One step = one call of ``dlrm_sparse_interact`` over one batch: the
+multi-table EmbeddingBag sum of all F tables, the pooled vectors written to
+HBM, and the strict-lower-triangle dots over [dense, pooled]. Default
+workload: B=2048, F=32 tables of 1e6 x 64 f32, L=16, Zipf(1.05) indices.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). Under torchrun each rank is an independent
+replica with its own batch (no collective on the data path); the timing is
+the max over ranks. ``--impl reference`` times the CPU oracle on the host
+cores on bounded samples of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dlrm_embedding_bag_b200 import synthetic as syn  # noqa: E402
+
+PROFILES = os.path.join(ROOT, "profiles")
+CSRC = os.path.join(ROOT, "dlrm_embedding_bag_b200", "csrc")
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "pooled lookups/s (fused EmbeddingBag-sum + lower-triangle interaction)"
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="c3", choices=sorted(syn.CONFIGS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU time budget of the oracle baseline sample")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return args
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def algorithmic_bytes(w: syn.Workload, write_pooled: bool = True) -> int:
+    """Bytes the fused step must move once: rows, indices, offsets, dense, outputs."""
+    B, F, L, D, P = w.B, w.F, w.L, w.D, w.P
+    rows = B * F * L * D * 4
+    idx = B * F * L * 4
+    offs = B * F * 4
+    dense = B * D * 4
+    pooled = B * F * D * 4 if write_pooled else 0
+    inter = B * ((D + P) if w.concat_dense else P) * 4
+    return rows + idx + offs + dense + pooled + inter
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            return json.load(fh)
+    except OSError:
+        return None
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for d in (CSRC, os.path.join(ROOT, "include")):
+        for name in sorted(os.listdir(d)):
+            with open(os.path.join(d, name), "rb") as fh:
+                h.update(name.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    path = os.path.join(PROFILES, "traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)
+    except OSError:
+        return None
+    ent = rec.get(workload)
+    if not ent or ent.get("source_digest") != source_digest():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML in a thread."""
+
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+             0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+             0x100: "display_clock_setting"}
+    BAD = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.period = period_s
+        self.ok = False
+        try:
+            import pynvml as nv
+
+            import torch
+
+            nv.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            handle = None
+            try:
+                bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id,
+                                            props.pci_device_id)
+                handle = nv.nvmlDeviceGetHandleByPciBusId_v2(bus)
+            except Exception:  # noqa: BLE001
+                handle = nv.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv, self.h = nv, handle
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.error = repr(e)
+        self._stop = threading.Event()
+        self._t = None
+
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return fn(self.h)
+
+    def sample(self):
+        if not self.ok:
+            return
+        nv = self.nv
+        try:
+            self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                 nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0, self._reasons()))
+        except Exception:  # noqa: BLE001
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(self.period)
+
+    def start(self):
+        self.sample()
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+        self.sample()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": getattr(self, "error", "nvml unavailable")}
+        if not self.samples:
+            return {"samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for s in self.samples:
+            bits |= int(s[2])
+        reasons = sorted(n for b, n in self.NAMES.items() if bits & b)
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(mhz), "power_w_max": max(s[1] for s in self.samples),
+                "samples": len(self.samples), "reasons": reasons}
+
+    def bad(self):
+        return bool(set(self.summary().get("reasons", [])) & self.BAD)
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+
+def host_tables_for(w: syn.Workload, idx_sub: np.ndarray, source=None, seed: int = 0):
+    """Full-size host tables in which only the rows the sample references hold data.
+
+    The tables are allocated zeroed (so untouched pages stay unmapped) and
+    the referenced rows are filled -- from the device tables when given
+    (same values as the GPU run), else from N(0, 0.1). The oracle then reads
+    the same row addresses in the same 4*N*D-byte tables as the full workload.
+    """
+    import torch
+
+    tables = []
+    rng = np.random.default_rng(seed)
+    for k in range(w.F):
+        t = np.zeros((w.N, w.D), dtype=np.float32)
+        rows = np.unique(idx_sub[k])
+        if source is not None:
+            vals = source[k].index_select(0, torch.from_numpy(rows.astype(np.int64)).to(
+                source[k].device)).cpu().numpy()
+        else:
+            vals = rng.normal(0.0, 0.1, (rows.size, w.D)).astype(np.float32)
+        t[rows] = vals
+        tables.append(t)
+    return tables
+
+
+def oracle_sample(w: syn.Workload, S: int, replica: int = 0, source=None):
+    """The first S samples of the workload's batch, ready for the oracle."""
+    idx = syn.make_indices(w, replica)[:, : S * w.L]
+    idx = np.ascontiguousarray(idx)
+    sub = w.scaled(B=S)
+    off = syn.make_offsets(sub)
+    rng = np.random.default_rng(3000)
+    dense = rng.normal(0.0, 1.0, (S, w.D)).astype(np.float32)
+    tables = host_tables_for(w, idx, source=source)
+    return tables, idx, off, dense
+
+
+def time_oracle(orc, tables, idx, off, dense, S, L, concat, budget_s, min_calls=1):
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while len(times) < min_calls or time.perf_counter() < t_end:
+        t0 = time.perf_counter()
+        orc.sparse_interact(tables, idx, off, dense, S, L, concat_dense=concat)
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+def cpu_baseline(w: syn.Workload, source, budget_s: float):
+    import oracle  # test infrastructure: this leg times the oracle as it stands
+
+    S = min(w.B, 512)
+    tables, idx, off, dense = oracle_sample(w, S, source=source)
+    orc = oracle.default()
+    orc.sparse_interact(tables, idx, off, dense, S, w.L, concat_dense=w.concat_dense)  # warm
+    times = time_oracle(orc, tables, idx, off, dense, S, w.L, w.concat_dense, budget_s)
+    t = statistics.median(times)
+    return {"value": S * w.F * w.L / t, "unit": "lookups/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {S} of {w.B} samples of {w.name} (all {w.F} tables, L={w.L}), "
+                      f"full-size host tables holding the referenced rows; median of "
+                      f"{len(times)} single-thread oracle calls"}
+
+
+def run_reference(args, w: syn.Workload):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle  # the reference arm of this benchmark is the oracle
+
+    S = min(w.B, 128)
+    tables, idx, off, dense = oracle_sample(w, S)
+    orc = oracle.default()
+    for _ in range(args.warmup):
+        orc.sparse_interact(tables, idx, off, dense, S, w.L, concat_dense=w.concat_dense)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.sparse_interact(tables, idx, off, dense, S, w.L, concat_dense=w.concat_dense)
+    dt = time.perf_counter() - t0
+    value = args.steps * S * w.F * w.L / dt
+    sample = (f"each step: first {S} of {w.B} samples of {w.name}, full-size host tables "
+              f"holding the referenced rows, one single-thread oracle call")
+    line = {"metric": METRIC, "value": value, "unit": "lookups/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(w, args.gpus), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "lookups/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "lookups/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w: syn.Workload, n: int):
+    return {"workload": w.name, "B": w.B, "F": w.F, "N": w.N, "D": w.D, "L": w.L,
+            "index_dist": (f"zipf(alpha={w.alpha}) over rows, rank->row permuted"
+                           if w.dist == "zipf" else "uniform"),
+            "offsets": "fixed stride b*L",
+            "outputs": "pooled (B,F,D) f32 + interaction (B,%s) f32" %
+                       ("D+P" if w.concat_dense else "P"),
+            "l2": "flushed before every step (256 MiB write outside the per-step events)",
+            "parallelism": "replicas" if n > 1 else "single GPU"}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, w: syn.Workload):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    from dlrm_embedding_bag_b200 import ops
+
+    # inputs resident in HBM before timing: tables, this replica's batch, outputs
+    weights = syn.make_weights(w, dev)
+    idx_np = syn.make_indices(w, replica=rank)
+    off_np = syn.make_offsets(w)
+    idx = torch.from_numpy(idx_np).to(dev)
+    off = torch.from_numpy(off_np).to(dev)
+    dense = syn.make_dense(w, dev)
+    pooled = torch.empty((w.B, w.F, w.D), dtype=torch.float32, device=dev)
+    inter = torch.empty((w.B, (w.D + w.P) if w.concat_dense else w.P), dtype=torch.float32,
+                        device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+
+    def step():
+        ops.sparse_interact(weights, idx, off, dense, w.L, concat_dense=w.concat_dense,
+                            pooled_out=pooled, inter_out=inter)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed_region():
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        sampler = ClockSampler(local)
+        barrier()
+        sampler.start()
+        n0 = ops.launch_count()
+        w0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record()
+            step()
+            ends[i].record()
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - w0
+        launches = ops.launch_count() - n0
+        barrier()
+        sampler.stop()
+        per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+        return per, wall, launches, sampler
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    per, wall, launches, sampler = timed_region()
+    remeasured = False
+    if sampler.bad():
+        per, wall, launches, sampler = timed_region()
+        remeasured = True
+
+    total_ms = float(sum(per))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    lookups = world * args.steps * w.B * w.F * w.L
+    value = lookups / (total_ms / 1e3)
+    ms_step = total_ms / args.steps
+
+    # e2e through the host-buffer entry point: inputs copied in, result copied out, every step
+    e2e = None
+    if not args.no_e2e:
+        stage = ops.HostStage(weights, w.B, w.L, concat_dense=w.concat_dense, want_pooled=True)
+        ih = torch.from_numpy(idx_np.reshape(-1)).pin_memory()
+        oh = torch.from_numpy(off_np).pin_memory()
+        dh = dense.cpu().pin_memory()
+        xh = torch.empty(tuple(inter.shape), dtype=torch.float32).pin_memory()
+        for _ in range(args.warmup):
+            stage(ih, oh, dh, xh)
+        barrier()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record()
+            stage(ih, oh, dh, xh)
+            ends[i].record()
+        barrier()
+        e2e_ms = float(sum(s.elapsed_time(e) for s, e in zip(starts, ends)))
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": lookups / (e2e_ms / 1e3), "unit": "lookups/s",
+               "h2d_bytes_per_step": stage.h2d_bytes(), "d2h_bytes_per_step": stage.d2h_bytes(),
+               "ms_per_step": e2e_ms / args.steps,
+               "path": "dlrm_sparse_interact_host: pinned indices/offsets/dense in, "
+                       "interaction rows out; pooled written to device staging"}
+
+    if rank == 0:
+        peaks = measured_peaks()
+        if peaks and peaks.get("hbm_gbs"):
+            peak, peak_src = float(peaks["hbm_gbs"]), "measured"
+        else:
+            peak, peak_src = FALLBACK_HBM_GBS, "fallback"
+        per_launch = algorithmic_bytes(w)
+        achieved = per_launch / (ms_step / 1e3) / 1e9
+        rows_gbs = w.B * w.F * w.L * w.D * 4 / (ms_step / 1e3) / 1e9
+        clocks = sampler.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": "lookups/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": workload_config(w, world),
+            "samples_per_s": world * args.steps * w.B / (total_ms / 1e3),
+            "gather_row_gbs": rows_gbs,
+            "roofline": {"bound": "hbm", "kernel": "fused_kernel (dlrm_sparse_interact)",
+                         "achieved": achieved, "peak": peak, "peak_source": peak_src,
+                         "unit": "GB/s", "frac": achieved / peak,
+                         "algorithmic_bytes_per_launch": per_launch,
+                         "traffic": recorded_traffic(w.name)},
+            "clocks": clocks, "remeasured": remeasured,
+            "gpu_launches": launches,
+            "region_wall_ms": 1e3 * wall,
+            "step_ms_p50": statistics.median(per), "step_ms_min": min(per),
+            "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, weights, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    w = syn.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,243 @@
+// C ABI of the DLRMv1 sparse/interaction stage (declared in dlrm_sparse.h):
+// host-side argument checks, packing of the table pointers into the kernel
+// parameter block, and the launches. Nothing here allocates memory.
+#include <climits>
+#include <cstdint>
+#include <cstring>
+
+#include "dlrm_sparse.h"
+#include "launch.h"
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return DLRM_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Per-block opt-in shared-memory limit of the current device.
+int64_t smem_limit_current_device(int* err) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    *err = cuda_fail(e);
+    return 0;
+  }
+  int v = 0;
+  e = cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) {
+    *err = cuda_fail(e);
+    return 0;
+  }
+  *err = DLRM_OK;
+  return v;
+}
+
+// Checks shared by every gather entry point; fills the parameter block.
+int check_gather_args(const float* const* weights, const int64_t* rows, bool need_rows,
+                      const int32_t* indices, const int32_t* offsets, int B, int F, int L, int D,
+                      dlrm::TableParams* tp, bool* tables_aligned16) {
+  if (F < 1 || F > DLRM_MAX_TABLES) return DLRM_ERR_TOO_MANY_TABLES;
+  if (B < 1 || L < 0 || D < 1) return DLRM_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * L > INT32_MAX) return DLRM_ERR_SHAPE;
+  if (weights == nullptr || offsets == nullptr) return DLRM_ERR_NULL;
+  if (L > 0 && indices == nullptr) return DLRM_ERR_NULL;
+  if (need_rows && rows == nullptr) return DLRM_ERR_NULL;
+  if (!aligned(offsets, 4) || (indices && !aligned(indices, 4))) return DLRM_ERR_ALIGN;
+  std::memset(tp, 0, sizeof(*tp));
+  bool a16 = true;
+  for (int k = 0; k < F; ++k) {
+    if (weights[k] == nullptr) return DLRM_ERR_NULL;
+    if (!aligned(weights[k], 4)) return DLRM_ERR_ALIGN;
+    a16 = a16 && aligned(weights[k], 16);
+    tp->w[k] = weights[k];
+    if (need_rows) {
+      if (rows[k] < 0) return DLRM_ERR_ARG;
+      tp->rows[k] = rows[k] > INT32_MAX ? INT32_MAX : static_cast<int32_t>(rows[k]);
+    }
+  }
+  *tables_aligned16 = a16;
+  return DLRM_OK;
+}
+
+int embbag_impl(const float* const* weights, const int64_t* rows, bool check,
+                const int32_t* indices, const int32_t* offsets, int B, int F, int L, int D,
+                float* out, int32_t* status_dev, cudaStream_t stream) {
+  dlrm::TableParams tp;
+  bool a16 = false;
+  int rc = check_gather_args(weights, rows, check, indices, offsets, B, F, L, D, &tp, &a16);
+  if (rc != DLRM_OK) return rc;
+  if (out == nullptr) return DLRM_ERR_NULL;
+  if (!aligned(out, 4) || (status_dev && !aligned(status_dev, 4))) return DLRM_ERR_ALIGN;
+  const bool vec_ok = (D % 4 == 0) && a16 && aligned(out, 16);
+  if (check && status_dev) {
+    cudaError_t e = cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  cudaError_t e = dlrm::launch_embbag(tp, indices, offsets, B, F, L, D, out,
+                                      check ? status_dev : nullptr, check, vec_ok, stream);
+  return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
+}
+
+int fused_impl(const float* const* weights, const int64_t* rows, bool check,
+               const int32_t* indices, const int32_t* offsets, const float* dense, int B, int F,
+               int L, int D, float* pooled_out, float* inter_out, int concat_dense,
+               int32_t* status_dev, cudaStream_t stream) {
+  dlrm::TableParams tp;
+  bool a16 = false;
+  int rc = check_gather_args(weights, rows, check, indices, offsets, B, F, L, D, &tp, &a16);
+  if (rc != DLRM_OK) return rc;
+  if (dense == nullptr || inter_out == nullptr) return DLRM_ERR_NULL;
+  if (!aligned(dense, 4) || !aligned(inter_out, 4) || (pooled_out && !aligned(pooled_out, 4)) ||
+      (status_dev && !aligned(status_dev, 4)))
+    return DLRM_ERR_ALIGN;
+  int err = DLRM_OK;
+  const int64_t limit = smem_limit_current_device(&err);
+  if (err != DLRM_OK) return err;
+  if (dlrm::interact_smem_per_sample(F, D) > limit) return DLRM_ERR_SHAPE;
+  const bool vec_ok = (D % 4 == 0) && a16 && aligned(dense, 16) &&
+                      (pooled_out == nullptr || aligned(pooled_out, 16));
+  if (check && status_dev) {
+    cudaError_t e = cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  cudaError_t e = dlrm::launch_fused(tp, indices, offsets, dense, B, F, L, D, pooled_out,
+                                     inter_out, concat_dense ? 1 : 0,
+                                     check ? status_dev : nullptr, check, vec_ok, limit, stream);
+  return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int embbag_sum_multi(const float* const* weights, const int32_t* indices, const int32_t* offsets,
+                     int B, int F, int L, int D, float* out, dlrm_stream_t stream) {
+  return embbag_impl(weights, nullptr, false, indices, offsets, B, F, L, D, out, nullptr,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int embbag_sum_multi_ex(const float* const* weights, const int64_t* rows, const int32_t* indices,
+                        const int32_t* offsets, int B, int F, int L, int D, float* out,
+                        int32_t* status_dev, dlrm_stream_t stream) {
+  return embbag_impl(weights, rows, true, indices, offsets, B, F, L, D, out, status_dev,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int interact_lower_tri(const float* dense, const float* emb, int B, int F, int D, float* out,
+                       dlrm_stream_t stream) {
+  if (F < 1 || F > DLRM_MAX_TABLES) return DLRM_ERR_TOO_MANY_TABLES;
+  if (B < 1 || D < 1) return DLRM_ERR_SHAPE;
+  if (dense == nullptr || emb == nullptr || out == nullptr) return DLRM_ERR_NULL;
+  if (!aligned(dense, 4) || !aligned(emb, 4) || !aligned(out, 4)) return DLRM_ERR_ALIGN;
+  int err = DLRM_OK;
+  const int64_t limit = smem_limit_current_device(&err);
+  if (err != DLRM_OK) return err;
+  if (dlrm::interact_smem_per_sample(F, D) > limit) return DLRM_ERR_SHAPE;
+  const bool vec_ok = (D % 4 == 0) && aligned(dense, 16) && aligned(emb, 16);
+  cudaError_t e = dlrm::launch_interact(dense, emb, B, F, D, out, vec_ok, limit,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
+}
+
+int dlrm_sparse_interact(const float* const* weights, const int32_t* indices,
+                         const int32_t* offsets, const float* dense, int B, int F, int L, int D,
+                         float* pooled_out, float* inter_out, int concat_dense,
+                         dlrm_stream_t stream) {
+  return fused_impl(weights, nullptr, false, indices, offsets, dense, B, F, L, D, pooled_out,
+                    inter_out, concat_dense, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dlrm_sparse_interact_ex(const float* const* weights, const int64_t* rows,
+                            const int32_t* indices, const int32_t* offsets, const float* dense,
+                            int B, int F, int L, int D, float* pooled_out, float* inter_out,
+                            int concat_dense, int32_t* status_dev, dlrm_stream_t stream) {
+  return fused_impl(weights, rows, true, indices, offsets, dense, B, F, L, D, pooled_out,
+                    inter_out, concat_dense, status_dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dlrm_sparse_interact_host(const float* const* weights, const int32_t* indices_host,
+                              const int32_t* offsets_host, const float* dense_host, int B, int F,
+                              int L, int D, int concat_dense, int32_t* indices_dev,
+                              int32_t* offsets_dev, float* dense_dev, float* pooled_dev,
+                              float* inter_dev, float* pooled_host, float* inter_host,
+                              dlrm_stream_t stream) {
+  if (F < 1 || F > DLRM_MAX_TABLES) return DLRM_ERR_TOO_MANY_TABLES;
+  if (B < 1 || L < 0 || D < 1) return DLRM_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * L > INT32_MAX) return DLRM_ERR_SHAPE;
+  if (offsets_host == nullptr || dense_host == nullptr || inter_host == nullptr ||
+      offsets_dev == nullptr || dense_dev == nullptr || inter_dev == nullptr)
+    return DLRM_ERR_NULL;
+  if (L > 0 && (indices_host == nullptr || indices_dev == nullptr)) return DLRM_ERR_NULL;
+  if (pooled_host != nullptr && pooled_dev == nullptr) return DLRM_ERR_NULL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t P = static_cast<int64_t>(F + 1) * F / 2;
+  const size_t n_idx = static_cast<size_t>(F) * B * L * sizeof(int32_t);
+  const size_t n_off = static_cast<size_t>(F) * B * sizeof(int32_t);
+  const size_t n_dense = static_cast<size_t>(B) * D * sizeof(float);
+  const size_t n_inter = static_cast<size_t>(B) * (concat_dense ? D + P : P) * sizeof(float);
+  const size_t n_pooled = static_cast<size_t>(B) * F * D * sizeof(float);
+  cudaError_t e;
+  if (n_idx > 0 &&
+      (e = cudaMemcpyAsync(indices_dev, indices_host, n_idx, cudaMemcpyHostToDevice, s)) !=
+          cudaSuccess)
+    return cuda_fail(e);
+  if ((e = cudaMemcpyAsync(offsets_dev, offsets_host, n_off, cudaMemcpyHostToDevice, s)) !=
+      cudaSuccess)
+    return cuda_fail(e);
+  if ((e = cudaMemcpyAsync(dense_dev, dense_host, n_dense, cudaMemcpyHostToDevice, s)) !=
+      cudaSuccess)
+    return cuda_fail(e);
+  int rc = fused_impl(weights, nullptr, false, indices_dev, offsets_dev, dense_dev, B, F, L, D,
+                      pooled_dev, inter_dev, concat_dense, nullptr, s);
+  if (rc != DLRM_OK) return rc;
+  if ((e = cudaMemcpyAsync(inter_host, inter_dev, n_inter, cudaMemcpyDeviceToHost, s)) !=
+      cudaSuccess)
+    return cuda_fail(e);
+  if (pooled_host &&
+      (e = cudaMemcpyAsync(pooled_host, pooled_dev, n_pooled, cudaMemcpyDeviceToHost, s)) !=
+          cudaSuccess)
+    return cuda_fail(e);
+  return DLRM_OK;
+}
+
+int dlrm_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_t* j_out,
+                     dlrm_stream_t stream) {
+  if (p0 < 0 || count < 0 || p0 + count > (int64_t{1} << 31)) return DLRM_ERR_ARG;
+  if (count > 0 && (i_out == nullptr || j_out == nullptr)) return DLRM_ERR_NULL;
+  if ((i_out && !aligned(i_out, 4)) || (j_out && !aligned(j_out, 4))) return DLRM_ERR_ALIGN;
+  cudaError_t e =
+      dlrm::launch_pair_decode(p0, count, i_out, j_out, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
+}
+
+int dlrm_status_from_flags(int32_t flags) {
+  if (flags & DLRM_FLAG_INDEX_OOB) return DLRM_ERR_INDEX_OOB;
+  if (flags & DLRM_FLAG_OFFSETS) return DLRM_ERR_OFFSETS;
+  return DLRM_OK;
+}
+
+const char* dlrm_status_string(int status) {
+  switch (status) {
+    case DLRM_OK: return "ok";
+    case DLRM_ERR_NULL: return "a required pointer is NULL";
+    case DLRM_ERR_SHAPE: return "invalid shape (B, L, D, B*L, or shared memory needed per sample)";
+    case DLRM_ERR_ALIGN: return "a float or int32 pointer is not 4-byte aligned";
+    case DLRM_ERR_TOO_MANY_TABLES: return "table count F must be in [1, DLRM_MAX_TABLES]";
+    case DLRM_ERR_INDEX_OOB: return "an index lies outside its table";
+    case DLRM_ERR_OFFSETS: return "offsets describe a bag with start > end or outside [0, B*L]";
+    case DLRM_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case DLRM_ERR_ARG: return "invalid argument";
+    default: return "unknown status";
+  }
+}
+
+int dlrm_last_cuda_error(void) { return t_last_cuda_error; }
+
+int64_t dlrm_launch_count(void) { return dlrm::launch_count(); }
+
+}  // extern "C"

@@ -1,0 +1,287 @@
+"""Python binding of ``libdlrm_sparse.so`` (the C ABI in ``include/dlrm_sparse.h``).
+
+Argument marshalling only: every function checks tensor placement, dtype and
+contiguity, passes raw pointers and the current CUDA stream to the C entry
+point of the same name, and raises :class:`DlrmError` on a non-zero status.
+All arithmetic happens in the library's CUDA kernels. If the library is
+missing, importing this module raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_HERE, "libdlrm_sparse.so")
+
+DLRM_MAX_TABLES = 256
+STATUS = {
+    0: "DLRM_OK",
+    -1: "DLRM_ERR_NULL",
+    -2: "DLRM_ERR_SHAPE",
+    -3: "DLRM_ERR_ALIGN",
+    -4: "DLRM_ERR_TOO_MANY_TABLES",
+    -5: "DLRM_ERR_INDEX_OOB",
+    -6: "DLRM_ERR_OFFSETS",
+    -7: "DLRM_ERR_CUDA",
+    -8: "DLRM_ERR_ARG",
+}
+FLAG_INDEX_OOB = 1
+FLAG_OFFSETS = 2
+
+# Every symbol the header declares, with its ctypes signature.
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+SIGNATURES = {
+    "embbag_sum_multi": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "embbag_sum_multi_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P]),
+    "interact_lower_tri": (_I, [_P, _P, _I, _I, _I, _P, _P]),
+    "dlrm_sparse_interact": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _I, _P]),
+    "dlrm_sparse_interact_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _P]),
+    "dlrm_sparse_interact_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                                       _P, _P, _P]),
+    "dlrm_pair_decode": (_I, [_I64, _I64, _P, _P, _P]),
+    "dlrm_status_from_flags": (_I, [ctypes.c_int32]),
+    "dlrm_status_string": (ctypes.c_char_p, [_I]),
+    "dlrm_last_cuda_error": (_I, []),
+    "dlrm_launch_count": (_I64, []),
+}
+
+
+class DlrmError(RuntimeError):
+    """A library call returned a non-zero ``dlrm_status_t``."""
+
+    def __init__(self, status: int, what: str, detail: str = ""):
+        name = STATUS.get(status, str(status))
+        msg = f"{what}: {name} ({_lib.dlrm_status_string(status).decode()})"
+        if status == -7:
+            msg += f", cudaError {_lib.dlrm_last_cuda_error()}"
+        super().__init__(msg + (f"; {detail}" if detail else ""))
+        self.status = status
+
+
+def load_library(path: str = LIBRARY) -> ctypes.CDLL:
+    """Load the CUDA library and bind every declared symbol; raise if absent."""
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with `python -m dlrm_embedding_bag_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = load_library()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise DlrmError(rc, what)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str, dtype: torch.dtype) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device (got {t.device})")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype} (got {t.dtype})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _table_ptrs(weights: Sequence[torch.Tensor]):
+    F = len(weights)
+    if not 1 <= F <= DLRM_MAX_TABLES:
+        raise ValueError(f"table count must be in [1, {DLRM_MAX_TABLES}] (got {F})")
+    D = weights[0].shape[1]
+    for k, w in enumerate(weights):
+        _dev(w, f"weights[{k}]", torch.float32)
+        if w.dim() != 2 or w.shape[1] != D:
+            raise ValueError(f"weights[{k}] must be (rows, {D})")
+    arr = (ctypes.c_void_p * F)(*[w.data_ptr() for w in weights])
+    rows = (ctypes.c_int64 * F)(*[w.shape[0] for w in weights])
+    return arr, rows, F, D
+
+
+def _bag_args(weights, indices, offsets, L):
+    arr, rows, F, D = _table_ptrs(weights)
+    if offsets.dim() != 2 or offsets.shape[0] != F:
+        raise ValueError(f"offsets must be (F={F}, B)")
+    B = offsets.shape[1]
+    if indices.numel() != F * B * L:
+        raise ValueError(f"indices must hold F*B*L = {F * B * L} entries (got {indices.numel()})")
+    ip = _dev(indices, "indices", torch.int32) if indices.numel() else 0
+    op = _dev(offsets, "offsets", torch.int32)
+    return arr, rows, F, D, B, ip, op
+
+
+def embbag_sum_multi(weights: Sequence[torch.Tensor], indices: torch.Tensor,
+                     offsets: torch.Tensor, L: int, out: Optional[torch.Tensor] = None,
+                     status: Optional[torch.Tensor] = None, checked: bool = False) -> torch.Tensor:
+    """Pooled ``(B, F, D)`` sums of F EmbeddingBag(sum) tables in one launch.
+
+    ``indices`` is ``(F, B*L)`` int32, ``offsets`` ``(F, B)`` int32. With
+    ``checked`` the ``_ex`` entry point runs (indices checked against each
+    table's rows; flags OR-ed into ``status``, a 1-element int32 tensor).
+    """
+    arr, rows, F, D, B, ip, op = _bag_args(weights, indices, offsets, L)
+    if out is None:
+        out = torch.empty((B, F, D), dtype=torch.float32, device=weights[0].device)
+    outp = _dev(out, "out", torch.float32)
+    if out.numel() != B * F * D:
+        raise ValueError("out must be (B, F, D)")
+    if checked:
+        sp = _dev(status, "status", torch.int32) if status is not None else None
+        _check(_lib.embbag_sum_multi_ex(arr, rows, ip, op, B, F, L, D, outp, sp, _stream()),
+               "embbag_sum_multi_ex")
+    else:
+        _check(_lib.embbag_sum_multi(arr, ip, op, B, F, L, D, outp, _stream()),
+               "embbag_sum_multi")
+    return out
+
+
+def interact_lower_tri(dense: torch.Tensor, emb: torch.Tensor,
+                       out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """``(B, (F+1)F/2)`` strict-lower-triangle dots over ``[dense, emb_0..emb_{F-1}]``."""
+    if emb.dim() != 3:
+        raise ValueError("emb must be (B, F, D)")
+    B, F, D = emb.shape
+    if tuple(dense.shape) != (B, D):
+        raise ValueError(f"dense must be ({B}, {D})")
+    P = (F + 1) * F // 2
+    if out is None:
+        out = torch.empty((B, P), dtype=torch.float32, device=emb.device)
+    if out.numel() != B * P:
+        raise ValueError("out must be (B, P)")
+    _check(_lib.interact_lower_tri(_dev(dense, "dense", torch.float32),
+                                   _dev(emb, "emb", torch.float32), B, F, D,
+                                   _dev(out, "out", torch.float32), _stream()),
+           "interact_lower_tri")
+    return out
+
+
+def sparse_interact(weights: Sequence[torch.Tensor], indices: torch.Tensor,
+                    offsets: torch.Tensor, dense: torch.Tensor, L: int, *,
+                    concat_dense: bool = False, pooled_out=None, inter_out=None,
+                    want_pooled: bool = True, status: Optional[torch.Tensor] = None,
+                    checked: bool = False):
+    """Fused stage: returns ``(pooled or None, inter)``.
+
+    ``inter`` is ``(B, P)``, or ``(B, D+P)`` with ``concat_dense``.
+    ``want_pooled=False`` skips writing the pooled vectors to memory.
+    """
+    arr, rows, F, D, B, ip, op = _bag_args(weights, indices, offsets, L)
+    if tuple(dense.shape) != (B, D):
+        raise ValueError(f"dense must be ({B}, {D})")
+    P = (F + 1) * F // 2
+    dev = weights[0].device
+    if want_pooled and pooled_out is None:
+        pooled_out = torch.empty((B, F, D), dtype=torch.float32, device=dev)
+    if inter_out is None:
+        inter_out = torch.empty((B, D + P if concat_dense else P), dtype=torch.float32,
+                                device=dev)
+    pp = _dev(pooled_out, "pooled_out", torch.float32) if pooled_out is not None else None
+    if pooled_out is not None and pooled_out.numel() != B * F * D:
+        raise ValueError("pooled_out must be (B, F, D)")
+    if inter_out.numel() != B * (D + P if concat_dense else P):
+        raise ValueError("inter_out has the wrong size")
+    dp = _dev(dense, "dense", torch.float32)
+    xp = _dev(inter_out, "inter_out", torch.float32)
+    if checked:
+        sp = _dev(status, "status", torch.int32) if status is not None else None
+        _check(_lib.dlrm_sparse_interact_ex(arr, rows, ip, op, dp, B, F, L, D, pp, xp,
+                                            1 if concat_dense else 0, sp, _stream()),
+               "dlrm_sparse_interact_ex")
+    else:
+        _check(_lib.dlrm_sparse_interact(arr, ip, op, dp, B, F, L, D, pp, xp,
+                                         1 if concat_dense else 0, _stream()),
+               "dlrm_sparse_interact")
+    return pooled_out, inter_out
+
+
+def _host(t: torch.Tensor, name: str, dtype: torch.dtype) -> int:
+    if t.device.type != "cpu" or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} CPU tensor")
+    return t.data_ptr()
+
+
+class HostStage:
+    """The whole stage fed from host memory, through ``dlrm_sparse_interact_host``.
+
+    Holds the device staging buffers (allocated once, by torch) for batches of
+    a fixed shape; each :meth:`__call__` enqueues the host-to-device copies,
+    the fused launch and the device-to-host copies on the current stream.
+    """
+
+    def __init__(self, weights: Sequence[torch.Tensor], B: int, L: int, *,
+                 concat_dense: bool = False, want_pooled: bool = False):
+        """``want_pooled``: the kernel also writes the pooled vectors (to a
+        device staging buffer; they reach the host only if ``pooled_host`` is
+        passed to the call)."""
+        self.arr, _, self.F, self.D = _table_ptrs(weights)
+        self.weights = list(weights)
+        self.B, self.L, self.concat = B, L, concat_dense
+        dev = weights[0].device
+        self.P = (self.F + 1) * self.F // 2
+        self.row = self.D + self.P if concat_dense else self.P
+        self.idx_dev = torch.empty(self.F * B * L, dtype=torch.int32, device=dev)
+        self.off_dev = torch.empty((self.F, B), dtype=torch.int32, device=dev)
+        self.dense_dev = torch.empty((B, self.D), dtype=torch.float32, device=dev)
+        self.inter_dev = torch.empty((B, self.row), dtype=torch.float32, device=dev)
+        self.pooled_dev = (torch.empty((B, self.F, self.D), dtype=torch.float32, device=dev)
+                           if want_pooled else None)
+
+    def h2d_bytes(self) -> int:
+        return 4 * (self.F * self.B * self.L + self.F * self.B + self.B * self.D)
+
+    def d2h_bytes(self, with_pooled: bool = False) -> int:
+        n = self.B * self.row
+        if with_pooled:
+            n += self.B * self.F * self.D
+        return 4 * n
+
+    def __call__(self, indices_host, offsets_host, dense_host, inter_host, pooled_host=None):
+        F, B, L, D = self.F, self.B, self.L, self.D
+        ip = _host(indices_host, "indices_host", torch.int32) if F * B * L else None
+        rc = _lib.dlrm_sparse_interact_host(
+            self.arr, ip, _host(offsets_host, "offsets_host", torch.int32),
+            _host(dense_host, "dense_host", torch.float32), B, F, L, D,
+            1 if self.concat else 0, self.idx_dev.data_ptr(), self.off_dev.data_ptr(),
+            self.dense_dev.data_ptr(),
+            self.pooled_dev.data_ptr() if self.pooled_dev is not None else None,
+            self.inter_dev.data_ptr(),
+            _host(pooled_host, "pooled_host", torch.float32) if pooled_host is not None else None,
+            _host(inter_host, "inter_host", torch.float32), _stream())
+        _check(rc, "dlrm_sparse_interact_host")
+
+
+def pair_decode(p0: int, count: int, device="cuda"):
+    """``(i, j)`` int32 tensors from the kernels' closed-form pair decoder."""
+    i = torch.empty(count, dtype=torch.int32, device=device)
+    j = torch.empty(count, dtype=torch.int32, device=device)
+    _check(_lib.dlrm_pair_decode(p0, count, i.data_ptr() if count else None,
+                                 j.data_ptr() if count else None, _stream()),
+           "dlrm_pair_decode")
+    return i, j
+
+
+def status_from_flags(flags: int) -> int:
+    return _lib.dlrm_status_from_flags(int(flags))
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process."""
+    return int(_lib.dlrm_launch_count())

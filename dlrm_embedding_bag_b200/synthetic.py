@@ -99,10 +99,14 @@ def zipf_ranks(rng: np.random.Generator, n: int, N: int, alpha: float) -> np.nda
     return r
 
 
-def table_indices(w: Workload, k: int, n: Optional[int] = None) -> np.ndarray:
-    """Index stream of table ``k`` (``n`` entries, default ``B*L``), int32."""
+def table_indices(w: Workload, k: int, n: Optional[int] = None, replica: int = 0) -> np.ndarray:
+    """Index stream of table ``k`` (``n`` entries, default ``B*L``), int32.
+
+    ``replica`` selects an independent batch for another data-parallel replica
+    (seed ``2000 + k + 100003 * replica``); replica 0 is the standard stream.
+    """
     n = w.B * w.L if n is None else n
-    rng = np.random.Generator(np.random.PCG64(2000 + k))
+    rng = np.random.Generator(np.random.PCG64(2000 + k + 100003 * replica))
     if w.dist == "uniform":
         return rng.integers(0, w.N, size=n, dtype=np.int64).astype(np.int32)
     if w.dist == "zipf":
@@ -112,11 +116,11 @@ def table_indices(w: Workload, k: int, n: Optional[int] = None) -> np.ndarray:
     raise ValueError(f"unknown index distribution {w.dist!r}")
 
 
-def make_indices(w: Workload) -> np.ndarray:
+def make_indices(w: Workload, replica: int = 0) -> np.ndarray:
     """``(F, B*L)`` int32 index matrix, table-major."""
     out = np.empty((w.F, w.B * w.L), dtype=np.int32)
     for k in range(w.F):
-        out[k] = table_indices(w, k)
+        out[k] = table_indices(w, k, replica=replica)
     return out
 
 

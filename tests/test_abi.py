@@ -1,0 +1,115 @@
+"""The C-ABI library on the CPU: it loads, exports exactly what the header
+declares, and rejects bad arguments on the host before any CUDA call.
+
+None of these calls reaches a kernel launch: every one fails a host-side check
+that runs before the library touches the CUDA runtime.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dlrm_sparse.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"DLRM_API\s+[\w\s\*]+?\b(\w+)\s*\(", src))
+
+
+@pytest.fixture(scope="module")
+def ops():
+    from dlrm_embedding_bag_b200 import build, ops as _ops
+
+    build.build()
+    return _ops
+
+
+def test_header_declares_the_stage_entry_points():
+    names = _declared()
+    assert {"embbag_sum_multi", "interact_lower_tri", "dlrm_sparse_interact"} <= names
+    assert len(names) == 11
+
+
+def test_library_exports_every_declared_symbol(ops):
+    names = _declared()
+    out = subprocess.run(["nm", "-D", "--defined-only", ops.LIBRARY], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    assert names == exported
+    assert names == set(ops.SIGNATURES)
+    for n in names:
+        assert getattr(ops._lib, n) is not None
+
+
+def _ptrs(*vals):
+    return (ctypes.c_void_p * len(vals))(*vals)
+
+
+def test_status_strings_and_flags(ops):
+    lib = ops._lib
+    for code in ops.STATUS:
+        assert lib.dlrm_status_string(code)
+    assert lib.dlrm_status_string(12345) == b"unknown status"
+    assert lib.dlrm_status_from_flags(0) == 0
+    assert lib.dlrm_status_from_flags(1) == -5
+    assert lib.dlrm_status_from_flags(2) == -6
+    assert lib.dlrm_status_from_flags(3) == -5
+    assert lib.dlrm_launch_count() == 0
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails a host check first
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(F=0), -4), (dict(F=257), -4), (dict(B=0), -2), (dict(L=-1), -2), (dict(D=0), -2),
+    (dict(B=1 << 20, L=1 << 12), -2), (dict(weights=None), -1), (dict(offsets=None), -1),
+    (dict(indices=None), -1), (dict(out=None), -1), (dict(w0=0), -1),
+    (dict(w0=FAKE + 2), -3), (dict(out=FAKE + 1), -3), (dict(offsets=FAKE + 2), -3),
+])
+def test_embbag_host_checks(ops, case, expect):
+    F = case.get("F", 2)
+    w0 = case.get("w0", FAKE)
+    weights = case.get("weights", _ptrs(*([w0] + [FAKE] * (max(F, 1) - 1))))
+    rc = ops._lib.embbag_sum_multi(weights, case.get("indices", FAKE), case.get("offsets", FAKE),
+                                   case.get("B", 4), F, case.get("L", 2), case.get("D", 8),
+                                   case.get("out", FAKE), None)
+    assert rc == expect
+
+
+def test_checked_entry_points_need_rows(ops):
+    rc = ops._lib.embbag_sum_multi_ex(_ptrs(FAKE), None, FAKE, FAKE, 4, 1, 2, 8, FAKE, None, None)
+    assert rc == -1
+    rows = (ctypes.c_int64 * 1)(-5)
+    rc = ops._lib.embbag_sum_multi_ex(_ptrs(FAKE), rows, FAKE, FAKE, 4, 1, 2, 8, FAKE, None, None)
+    assert rc == -8
+
+
+def test_fused_and_interact_host_checks(ops):
+    lib = ops._lib
+    w = _ptrs(FAKE, FAKE)
+    assert lib.dlrm_sparse_interact(w, FAKE, FAKE, None, 4, 2, 2, 8, None, FAKE, 0, None) == -1
+    assert lib.dlrm_sparse_interact(w, FAKE, FAKE, FAKE, 4, 2, 2, 8, None, None, 0, None) == -1
+    assert lib.dlrm_sparse_interact(w, FAKE, FAKE, FAKE + 1, 4, 2, 2, 8, None, FAKE, 0,
+                                    None) == -3
+    assert lib.dlrm_sparse_interact(w, FAKE, FAKE, FAKE, 4, 0, 2, 8, None, FAKE, 0, None) == -4
+    assert lib.interact_lower_tri(None, FAKE, 4, 2, 8, FAKE, None) == -1
+    assert lib.interact_lower_tri(FAKE, FAKE, 0, 2, 8, FAKE, None) == -2
+    assert lib.interact_lower_tri(FAKE, FAKE, 4, 300, 8, FAKE, None) == -4
+    assert lib.interact_lower_tri(FAKE, FAKE + 2, 4, 2, 8, FAKE, None) == -3
+    assert lib.dlrm_sparse_interact_host(w, FAKE, FAKE, FAKE, 4, 2, 2, 8, 0, FAKE, FAKE, FAKE,
+                                         None, FAKE, FAKE, None, None) == -1
+    assert lib.dlrm_pair_decode(-1, 5, FAKE, FAKE, None) == -8
+    assert lib.dlrm_pair_decode(0, -1, FAKE, FAKE, None) == -8
+    assert lib.dlrm_pair_decode((1 << 31) - 2, 5, FAKE, FAKE, None) == -8
+    assert lib.dlrm_pair_decode(0, 5, None, FAKE, None) == -1
+    assert lib.dlrm_launch_count() == 0
+
+
+def test_missing_library_fails_loudly(ops, tmp_path):
+    with pytest.raises(ImportError, match="no CPU fallback"):
+        ops.load_library(str(tmp_path / "libdlrm_sparse.so"))
