@@ -46,6 +46,9 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="c3", choices=sorted(syn.CONFIGS))
+    ap.add_argument("--rows", type=int, default=None,
+                    help="override the rows per table (a smaller case for profiling)")
+    ap.add_argument("--batch", type=int, default=None, help="override the batch size")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -326,9 +329,12 @@ def run_ours(args, w: syn.Workload):
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
 
+    call = ops.SparseInteractCall(weights, idx, off, dense, w.L, concat_dense=w.concat_dense,
+                                  pooled_out=pooled, inter_out=inter)
+    stream = torch.cuda.current_stream().cuda_stream
+
     def step():
-        ops.sparse_interact(weights, idx, off, dense, w.L, concat_dense=w.concat_dense,
-                            pooled_out=pooled, inter_out=inter)
+        call(stream)
 
     def barrier():
         if world > 1:
@@ -445,6 +451,10 @@ def run_ours(args, w: syn.Workload):
 def main(argv=None):
     args = parse_args(argv)
     w = syn.CONFIGS[args.config]
+    if args.rows or args.batch:
+        B = args.batch or w.B
+        N = args.rows or w.N
+        w = w.scaled(B=B, N=N, name=f"{w.name}_B{B}_N{N}")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -212,6 +212,47 @@ def sparse_interact(weights: Sequence[torch.Tensor], indices: torch.Tensor,
     return pooled_out, inter_out
 
 
+class SparseInteractCall:
+    """A prepared ``dlrm_sparse_interact`` call on fixed buffers.
+
+    All arguments are checked and marshalled once; each ``__call__`` is a
+    single C call on the current stream (what a serving loop or a CUDA-graph
+    capture wants). The object keeps the tensors alive; their contents may
+    change between calls, their storage must not.
+    """
+
+    def __init__(self, weights: Sequence[torch.Tensor], indices: torch.Tensor,
+                 offsets: torch.Tensor, dense: torch.Tensor, L: int, *,
+                 concat_dense: bool = False, pooled_out=None, inter_out=None,
+                 want_pooled: bool = True):
+        arr, _, F, D, B, ip, op = _bag_args(weights, indices, offsets, L)
+        if tuple(dense.shape) != (B, D):
+            raise ValueError(f"dense must be ({B}, {D})")
+        P = (F + 1) * F // 2
+        dev = weights[0].device
+        if want_pooled and pooled_out is None:
+            pooled_out = torch.empty((B, F, D), dtype=torch.float32, device=dev)
+        if inter_out is None:
+            inter_out = torch.empty((B, D + P if concat_dense else P), dtype=torch.float32,
+                                    device=dev)
+        if pooled_out is not None and pooled_out.numel() != B * F * D:
+            raise ValueError("pooled_out must be (B, F, D)")
+        if inter_out.numel() != B * (D + P if concat_dense else P):
+            raise ValueError("inter_out has the wrong size")
+        pp = _dev(pooled_out, "pooled_out", torch.float32) if pooled_out is not None else None
+        self._keep = (list(weights), indices, offsets, dense)
+        self.pooled, self.inter = pooled_out, inter_out
+        self._args = (arr, ip, op, _dev(dense, "dense", torch.float32), B, F, L, D, pp,
+                      _dev(inter_out, "inter_out", torch.float32), 1 if concat_dense else 0)
+        self._fn = _lib.dlrm_sparse_interact
+
+    def __call__(self, stream: Optional[int] = None):
+        rc = self._fn(*self._args, _stream() if stream is None else stream)
+        if rc != 0:
+            raise DlrmError(rc, "dlrm_sparse_interact")
+        return self.pooled, self.inter
+
+
 def _host(t: torch.Tensor, name: str, dtype: torch.dtype) -> int:
     if t.device.type != "cpu" or t.dtype != dtype or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous {dtype} CPU tensor")

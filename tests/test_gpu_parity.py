@@ -398,3 +398,15 @@ def test_nondefault_stream_ordering(ops):
                                        w.L, False)
     assert_bits_equal(fp, ref_p, "side stream pooled")
     check_inter(fi, ref_i, bound, w.D, False, "side stream")
+
+
+def test_prepared_call_matches_plain_call(ops):
+    w = syn.C2_CONCAT.scaled(B=333)
+    weights, idx, off, dense = _inputs(w)
+    idx_d, off_d = _dev_i32(idx), _dev_i32(off)
+    call = ops.SparseInteractCall(weights, idx_d, off_d, dense, w.L, concat_dense=True)
+    p1, i1 = call()
+    p2, i2 = ops.sparse_interact(weights, idx_d, off_d, dense, w.L, concat_dense=True)
+    torch.cuda.synchronize()
+    assert torch.equal(p1.view(torch.int32), p2.view(torch.int32))
+    assert torch.equal(i1.view(torch.int32), i2.view(torch.int32))
