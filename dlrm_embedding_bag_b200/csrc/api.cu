@@ -37,78 +37,125 @@ int64_t smem_limit_current_device(int* err) {
   return v;
 }
 
-// Checks shared by every gather entry point; fills the parameter block.
-int check_gather_args(const float* const* weights, const int64_t* rows, bool need_rows,
-                      const int32_t* indices, const int32_t* offsets, int B, int F, int L, int D,
-                      dlrm::TableParams* tp, bool* tables_aligned16) {
+// A checked set of gather arguments, ready to launch.
+struct Prepared {
+  dlrm::TableParams tp;
+  dlrm::BagParams bp;
+  int pool;
+  bool tables_aligned16;
+  int elem_size;
+};
+
+// Checks shared by every gather entry point; fills the parameter blocks.
+int prepare(const void* const* weights, int dtype, const int64_t* rows, const dlrm_bags_t* bags,
+            int B, int F, int D, int32_t* status_dev, Prepared* pr) {
+  if (bags == nullptr) return DLRM_ERR_NULL;
   if (F < 1 || F > DLRM_MAX_TABLES) return DLRM_ERR_TOO_MANY_TABLES;
-  if (B < 1 || L < 0 || D < 1) return DLRM_ERR_SHAPE;
-  if (static_cast<int64_t>(B) * L > INT32_MAX) return DLRM_ERR_SHAPE;
-  if (weights == nullptr || offsets == nullptr) return DLRM_ERR_NULL;
-  if (L > 0 && indices == nullptr) return DLRM_ERR_NULL;
-  if (need_rows && rows == nullptr) return DLRM_ERR_NULL;
-  if (!aligned(offsets, 4) || (indices && !aligned(indices, 4))) return DLRM_ERR_ALIGN;
-  std::memset(tp, 0, sizeof(*tp));
+  if (B < 1 || D < 1 || bags->T < 0 || bags->T > INT32_MAX) return DLRM_ERR_SHAPE;
+  if (dtype != DLRM_TABLE_F32 && dtype != DLRM_TABLE_BF16) return DLRM_ERR_ARG;
+  if (bags->mode != DLRM_POOL_SUM && bags->mode != DLRM_POOL_MEAN && bags->mode != DLRM_POOL_MAX)
+    return DLRM_ERR_ARG;
+  if (bags->per_sample_weights != nullptr && bags->mode != DLRM_POOL_SUM) return DLRM_ERR_ARG;
+  if (weights == nullptr || bags->offsets == nullptr) return DLRM_ERR_NULL;
+  if (bags->T > 0 && bags->indices == nullptr) return DLRM_ERR_NULL;
+  if (!aligned(bags->offsets, 4) || (bags->indices && !aligned(bags->indices, 4)) ||
+      (bags->per_sample_weights && !aligned(bags->per_sample_weights, 4)) ||
+      (status_dev && !aligned(status_dev, 4)))
+    return DLRM_ERR_ALIGN;
+  const int esz = dtype == DLRM_TABLE_BF16 ? 2 : 4;
+  std::memset(&pr->tp, 0, sizeof(pr->tp));
   bool a16 = true;
   for (int k = 0; k < F; ++k) {
     if (weights[k] == nullptr) return DLRM_ERR_NULL;
-    if (!aligned(weights[k], 4)) return DLRM_ERR_ALIGN;
+    if (!aligned(weights[k], esz)) return DLRM_ERR_ALIGN;
     a16 = a16 && aligned(weights[k], 16);
-    tp->w[k] = weights[k];
-    if (need_rows) {
+    pr->tp.w[k] = weights[k];
+    if (rows != nullptr) {
       if (rows[k] < 0) return DLRM_ERR_ARG;
-      tp->rows[k] = rows[k] > INT32_MAX ? INT32_MAX : static_cast<int32_t>(rows[k]);
+      pr->tp.rows[k] = rows[k] > INT32_MAX ? INT32_MAX : static_cast<int32_t>(rows[k]);
     }
   }
-  *tables_aligned16 = a16;
+  pr->bp.indices = bags->indices;
+  pr->bp.offsets = bags->offsets;
+  pr->bp.psw = bags->per_sample_weights;
+  pr->bp.T = static_cast<int>(bags->T);
+  pr->bp.ilo = bags->include_last_offset ? 1 : 0;
+  pr->bp.mean = bags->mode == DLRM_POOL_MEAN ? 1 : 0;
+  pr->bp.check = rows != nullptr ? 1 : 0;
+  pr->bp.status = status_dev;
+  pr->pool = bags->per_sample_weights ? dlrm::kPoolWeighted
+             : bags->mode == DLRM_POOL_MAX ? dlrm::kPoolMax
+                                          : dlrm::kPoolSum;
+  pr->tables_aligned16 = a16;
+  pr->elem_size = esz;
   return DLRM_OK;
 }
 
-int embbag_impl(const float* const* weights, const int64_t* rows, bool check,
-                const int32_t* indices, const int32_t* offsets, int B, int F, int L, int D,
-                float* out, int32_t* status_dev, cudaStream_t stream) {
-  dlrm::TableParams tp;
-  bool a16 = false;
-  int rc = check_gather_args(weights, rows, check, indices, offsets, B, F, L, D, &tp, &a16);
-  if (rc != DLRM_OK) return rc;
-  if (out == nullptr) return DLRM_ERR_NULL;
-  if (!aligned(out, 4) || (status_dev && !aligned(status_dev, 4))) return DLRM_ERR_ALIGN;
-  const bool vec_ok = (D % 4 == 0) && a16 && aligned(out, 16);
-  if (check && status_dev) {
-    cudaError_t e = cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream);
-    if (e != cudaSuccess) return cuda_fail(e);
-  }
-  cudaError_t e = dlrm::launch_embbag(tp, indices, offsets, B, F, L, D, out,
-                                      check ? status_dev : nullptr, check, vec_ok, stream);
+// The vector loader needs whole 16-byte chunks per row and 16-byte aligned
+// tables and float destinations.
+int pick_loader(int dtype, int D, bool vec_ok) {
+  if (dtype == DLRM_TABLE_BF16)
+    return (vec_ok && D % 8 == 0) ? dlrm::kLdBF16x8 : dlrm::kLdBF16x1;
+  return (vec_ok && D % 4 == 0) ? dlrm::kLdF32x4 : dlrm::kLdF32x1;
+}
+
+int clear_status(int32_t* status_dev, cudaStream_t stream) {
+  if (status_dev == nullptr) return DLRM_OK;
+  cudaError_t e = cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream);
   return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
 }
 
-int fused_impl(const float* const* weights, const int64_t* rows, bool check,
-               const int32_t* indices, const int32_t* offsets, const float* dense, int B, int F,
-               int L, int D, float* pooled_out, float* inter_out, int concat_dense,
-               int32_t* status_dev, cudaStream_t stream) {
-  dlrm::TableParams tp;
-  bool a16 = false;
-  int rc = check_gather_args(weights, rows, check, indices, offsets, B, F, L, D, &tp, &a16);
+int pool_impl(const void* const* weights, int dtype, const int64_t* rows, const dlrm_bags_t* bags,
+              int B, int F, int D, float* out, int32_t* status_dev, cudaStream_t stream) {
+  Prepared pr;
+  int rc = prepare(weights, dtype, rows, bags, B, F, D, status_dev, &pr);
+  if (rc != DLRM_OK) return rc;
+  if (out == nullptr) return DLRM_ERR_NULL;
+  if (!aligned(out, 4)) return DLRM_ERR_ALIGN;
+  const int loader = pick_loader(dtype, D, pr.tables_aligned16 && aligned(out, 16));
+  if ((rc = clear_status(status_dev, stream)) != DLRM_OK) return rc;
+  cudaError_t e = dlrm::launch_embbag(pr.tp, pr.bp, B, F, D, out, pr.pool, loader, stream);
+  return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
+}
+
+int fused_impl(const void* const* weights, int dtype, const int64_t* rows,
+               const dlrm_bags_t* bags, const float* dense, int B, int F, int D,
+               float* pooled_out, float* inter_out, int concat_dense, int32_t* status_dev,
+               cudaStream_t stream) {
+  Prepared pr;
+  int rc = prepare(weights, dtype, rows, bags, B, F, D, status_dev, &pr);
   if (rc != DLRM_OK) return rc;
   if (dense == nullptr || inter_out == nullptr) return DLRM_ERR_NULL;
-  if (!aligned(dense, 4) || !aligned(inter_out, 4) || (pooled_out && !aligned(pooled_out, 4)) ||
-      (status_dev && !aligned(status_dev, 4)))
+  if (!aligned(dense, 4) || !aligned(inter_out, 4) || (pooled_out && !aligned(pooled_out, 4)))
     return DLRM_ERR_ALIGN;
   int err = DLRM_OK;
   const int64_t limit = smem_limit_current_device(&err);
   if (err != DLRM_OK) return err;
   if (dlrm::interact_smem_per_sample(F, D) > limit) return DLRM_ERR_SHAPE;
-  const bool vec_ok = (D % 4 == 0) && a16 && aligned(dense, 16) &&
-                      (pooled_out == nullptr || aligned(pooled_out, 16));
-  if (check && status_dev) {
-    cudaError_t e = cudaMemsetAsync(status_dev, 0, sizeof(int32_t), stream);
-    if (e != cudaSuccess) return cuda_fail(e);
-  }
-  cudaError_t e = dlrm::launch_fused(tp, indices, offsets, dense, B, F, L, D, pooled_out,
-                                     inter_out, concat_dense ? 1 : 0,
-                                     check ? status_dev : nullptr, check, vec_ok, limit, stream);
+  const bool vec_ok = pr.tables_aligned16 && (pooled_out == nullptr || aligned(pooled_out, 16));
+  const int loader = pick_loader(dtype, D, vec_ok);
+  if ((rc = clear_status(status_dev, stream)) != DLRM_OK) return rc;
+  cudaError_t e = dlrm::launch_fused(pr.tp, pr.bp, dense, B, F, D, pooled_out, inter_out,
+                                     concat_dense ? 1 : 0, pr.pool, loader, limit, stream);
   return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
+}
+
+// The fixed-stride, unweighted-sum, f32 case of the general entry points.
+int fixed_stride_bags(const int32_t* indices, const int32_t* offsets, int B, int L,
+                      dlrm_bags_t* bags) {
+  if (B < 1 || L < 0) return DLRM_ERR_SHAPE;
+  if (static_cast<int64_t>(B) * L > INT32_MAX) return DLRM_ERR_SHAPE;
+  bags->indices = indices;
+  bags->offsets = offsets;
+  bags->per_sample_weights = nullptr;
+  bags->T = static_cast<int64_t>(B) * L;
+  bags->include_last_offset = 0;
+  bags->mode = DLRM_POOL_SUM;
+  return DLRM_OK;
+}
+
+const void* const* as_void(const float* const* w) {
+  return reinterpret_cast<const void* const*>(w);
 }
 
 }  // namespace
@@ -117,15 +164,31 @@ extern "C" {
 
 int embbag_sum_multi(const float* const* weights, const int32_t* indices, const int32_t* offsets,
                      int B, int F, int L, int D, float* out, dlrm_stream_t stream) {
-  return embbag_impl(weights, nullptr, false, indices, offsets, B, F, L, D, out, nullptr,
-                     reinterpret_cast<cudaStream_t>(stream));
+  if (F < 1 || F > DLRM_MAX_TABLES) return DLRM_ERR_TOO_MANY_TABLES;
+  dlrm_bags_t bags;
+  int rc = fixed_stride_bags(indices, offsets, B, L, &bags);
+  if (rc != DLRM_OK) return rc;
+  return pool_impl(as_void(weights), DLRM_TABLE_F32, nullptr, &bags, B, F, D, out, nullptr,
+                   reinterpret_cast<cudaStream_t>(stream));
 }
 
 int embbag_sum_multi_ex(const float* const* weights, const int64_t* rows, const int32_t* indices,
                         const int32_t* offsets, int B, int F, int L, int D, float* out,
                         int32_t* status_dev, dlrm_stream_t stream) {
-  return embbag_impl(weights, rows, true, indices, offsets, B, F, L, D, out, status_dev,
-                     reinterpret_cast<cudaStream_t>(stream));
+  if (F < 1 || F > DLRM_MAX_TABLES) return DLRM_ERR_TOO_MANY_TABLES;
+  if (rows == nullptr) return DLRM_ERR_NULL;
+  dlrm_bags_t bags;
+  int rc = fixed_stride_bags(indices, offsets, B, L, &bags);
+  if (rc != DLRM_OK) return rc;
+  return pool_impl(as_void(weights), DLRM_TABLE_F32, rows, &bags, B, F, D, out, status_dev,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+int embbag_pool_multi(const void* const* weights, int table_dtype, const int64_t* rows,
+                      const dlrm_bags_t* bags, int B, int F, int D, float* out,
+                      int32_t* status_dev, dlrm_stream_t stream) {
+  return pool_impl(weights, table_dtype, rows, bags, B, F, D, out, status_dev,
+                   reinterpret_cast<cudaStream_t>(stream));
 }
 
 int interact_lower_tri(const float* dense, const float* emb, int B, int F, int D, float* out,
@@ -148,16 +211,34 @@ int dlrm_sparse_interact(const float* const* weights, const int32_t* indices,
                          const int32_t* offsets, const float* dense, int B, int F, int L, int D,
                          float* pooled_out, float* inter_out, int concat_dense,
                          dlrm_stream_t stream) {
-  return fused_impl(weights, nullptr, false, indices, offsets, dense, B, F, L, D, pooled_out,
-                    inter_out, concat_dense, nullptr, reinterpret_cast<cudaStream_t>(stream));
+  if (F < 1 || F > DLRM_MAX_TABLES) return DLRM_ERR_TOO_MANY_TABLES;
+  dlrm_bags_t bags;
+  int rc = fixed_stride_bags(indices, offsets, B, L, &bags);
+  if (rc != DLRM_OK) return rc;
+  return fused_impl(as_void(weights), DLRM_TABLE_F32, nullptr, &bags, dense, B, F, D,
+                    pooled_out, inter_out, concat_dense, nullptr,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dlrm_sparse_interact_ex(const float* const* weights, const int64_t* rows,
                             const int32_t* indices, const int32_t* offsets, const float* dense,
                             int B, int F, int L, int D, float* pooled_out, float* inter_out,
                             int concat_dense, int32_t* status_dev, dlrm_stream_t stream) {
-  return fused_impl(weights, rows, true, indices, offsets, dense, B, F, L, D, pooled_out,
+  if (F < 1 || F > DLRM_MAX_TABLES) return DLRM_ERR_TOO_MANY_TABLES;
+  if (rows == nullptr) return DLRM_ERR_NULL;
+  dlrm_bags_t bags;
+  int rc = fixed_stride_bags(indices, offsets, B, L, &bags);
+  if (rc != DLRM_OK) return rc;
+  return fused_impl(as_void(weights), DLRM_TABLE_F32, rows, &bags, dense, B, F, D, pooled_out,
                     inter_out, concat_dense, status_dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dlrm_sparse_interact_pool(const void* const* weights, int table_dtype, const int64_t* rows,
+                              const dlrm_bags_t* bags, const float* dense, int B, int F, int D,
+                              float* pooled_out, float* inter_out, int concat_dense,
+                              int32_t* status_dev, dlrm_stream_t stream) {
+  return fused_impl(weights, table_dtype, rows, bags, dense, B, F, D, pooled_out, inter_out,
+                    concat_dense, status_dev, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dlrm_sparse_interact_host(const float* const* weights, const int32_t* indices_host,
@@ -192,8 +273,8 @@ int dlrm_sparse_interact_host(const float* const* weights, const int32_t* indice
   if ((e = cudaMemcpyAsync(dense_dev, dense_host, n_dense, cudaMemcpyHostToDevice, s)) !=
       cudaSuccess)
     return cuda_fail(e);
-  int rc = fused_impl(weights, nullptr, false, indices_dev, offsets_dev, dense_dev, B, F, L, D,
-                      pooled_dev, inter_dev, concat_dense, nullptr, s);
+  int rc = dlrm_sparse_interact(weights, indices_dev, offsets_dev, dense_dev, B, F, L, D,
+                                pooled_dev, inter_dev, concat_dense, stream);
   if (rc != DLRM_OK) return rc;
   if ((e = cudaMemcpyAsync(inter_host, inter_dev, n_inter, cudaMemcpyDeviceToHost, s)) !=
       cudaSuccess)
@@ -225,11 +306,11 @@ const char* dlrm_status_string(int status) {
   switch (status) {
     case DLRM_OK: return "ok";
     case DLRM_ERR_NULL: return "a required pointer is NULL";
-    case DLRM_ERR_SHAPE: return "invalid shape (B, L, D, B*L, or shared memory needed per sample)";
-    case DLRM_ERR_ALIGN: return "a float or int32 pointer is not 4-byte aligned";
+    case DLRM_ERR_SHAPE: return "invalid shape (B, L, D, T, or shared memory needed per sample)";
+    case DLRM_ERR_ALIGN: return "a pointer is not aligned to its element size";
     case DLRM_ERR_TOO_MANY_TABLES: return "table count F must be in [1, DLRM_MAX_TABLES]";
     case DLRM_ERR_INDEX_OOB: return "an index lies outside its table";
-    case DLRM_ERR_OFFSETS: return "offsets describe a bag with start > end or outside [0, B*L]";
+    case DLRM_ERR_OFFSETS: return "offsets describe a bag with start > end or outside [0, T]";
     case DLRM_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case DLRM_ERR_ARG: return "invalid argument";
     default: return "unknown status";

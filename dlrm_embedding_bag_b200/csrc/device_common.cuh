@@ -16,42 +16,78 @@ constexpr int kBlockThreads = 256;
 // counts) travel by value in the kernel's parameter block (__grid_constant__),
 // so a launch needs no device-side pointer array and no host-to-device copy.
 struct TableParams {
-  const float* w[DLRM_MAX_TABLES];
+  const void* w[DLRM_MAX_TABLES];
   int32_t rows[DLRM_MAX_TABLES];
 };
 
-// 128-bit and 32-bit read-only loads of table rows.
-__device__ __forceinline__ float4 load_row_chunk(const float* p, float4*) {
-  return __ldg(reinterpret_cast<const float4*>(p));
-}
-__device__ __forceinline__ float load_row_chunk(const float* p, float*) { return __ldg(p); }
-
-__device__ __forceinline__ void acc_add(float4& a, const float4& v) {
-  a.x = __fadd_rn(a.x, v.x);
-  a.y = __fadd_rn(a.y, v.y);
-  a.z = __fadd_rn(a.z, v.z);
-  a.w = __fadd_rn(a.w, v.w);
-}
-__device__ __forceinline__ void acc_add(float& a, const float& v) { a = __fadd_rn(a, v); }
-
-__device__ __forceinline__ void set_zero(float4& a) { a = make_float4(0.f, 0.f, 0.f, 0.f); }
-__device__ __forceinline__ void set_zero(float& a) { a = 0.f; }
-
-template <int VEC>
-struct VecOf;
-template <>
-struct VecOf<4> {
-  using T = float4;
-};
-template <>
-struct VecOf<1> {
-  using T = float;
+// Where the bags are and how they pool.
+struct BagParams {
+  const int32_t* indices;  // (F, T) table-major
+  const int32_t* offsets;  // (F, B) or (F, B + 1) with include_last_offset
+  const float* psw;        // (F, T) per-sample weights, or null
+  int T;                   // index entries per table
+  int ilo;                 // include_last_offset
+  int mean;                // divide each pooled sum by the bag's entry count
+  int check;               // skip (and flag) indices outside [0, rows[k])
+  int32_t* status;         // device flags, or null
 };
 
-__device__ __forceinline__ void store_vec(float* p, const float4& v) {
-  *reinterpret_cast<float4*>(p) = v;
+// Pooling combine step, fixed per template instance.
+enum PoolKind { kPoolSum = 0, kPoolWeighted = 1, kPoolMax = 2 };
+
+// ---------------------------------------------------------------------------
+// Row loaders: one lane loads VEC consecutive table elements per request and
+// hands them out widened to f32.
+
+struct LdF32x4 {  // 128-bit loads of 4 floats
+  static constexpr int VEC = 4;
+  using Elem = float;
+  using Raw = float4;
+  __device__ __forceinline__ static Raw load(const Elem* p) {
+    return __ldg(reinterpret_cast<const float4*>(p));
+  }
+  __device__ __forceinline__ static float get(const Raw& r, int e) {
+    return e == 0 ? r.x : e == 1 ? r.y : e == 2 ? r.z : r.w;
+  }
+};
+
+struct LdF32x1 {  // scalar fallback
+  static constexpr int VEC = 1;
+  using Elem = float;
+  using Raw = float;
+  __device__ __forceinline__ static Raw load(const Elem* p) { return __ldg(p); }
+  __device__ __forceinline__ static float get(const Raw& r, int) { return r; }
+};
+
+// A bf16 value is the upper half of an f32: widening is a 16-bit shift.
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t h16) {
+  return __uint_as_float(h16 << 16);
 }
-__device__ __forceinline__ void store_vec(float* p, const float& v) { *p = v; }
+
+struct LdBF16x8 {  // 128-bit loads of 8 bf16
+  static constexpr int VEC = 8;
+  using Elem = uint16_t;
+  using Raw = uint4;
+  __device__ __forceinline__ static Raw load(const Elem* p) {
+    return __ldg(reinterpret_cast<const uint4*>(p));
+  }
+  __device__ __forceinline__ static float get(const Raw& r, int e) {
+    const uint32_t w = (e >> 1) == 0 ? r.x : (e >> 1) == 1 ? r.y : (e >> 1) == 2 ? r.z : r.w;
+    return (e & 1) ? __uint_as_float(w & 0xffff0000u) : __uint_as_float(w << 16);
+  }
+};
+
+struct LdBF16x1 {  // scalar fallback
+  static constexpr int VEC = 1;
+  using Elem = uint16_t;
+  using Raw = unsigned short;
+  __device__ __forceinline__ static Raw load(const Elem* p) {
+    return __ldg(reinterpret_cast<const unsigned short*>(p));
+  }
+  __device__ __forceinline__ static float get(const Raw& r, int) {
+    return bf16_bits_to_float(static_cast<uint32_t>(r));
+  }
+};
 
 // Flat index p of the strict lower triangle (row-major, i > j) -> (i, j):
 // i = floor((1 + sqrt(1 + 8p)) / 2), j = p - i(i-1)/2. The square root is
@@ -68,78 +104,135 @@ __device__ __forceinline__ void pair_from_flat(int64_t p, int& i_out, int& j_out
   j_out = static_cast<int>(p - i * (i - 1) / 2);
 }
 
-// Bag bounds of (table k, sample b) under the include_last_offset=False rule.
-// Invalid offsets give an empty bag and raise *bad.
-__device__ __forceinline__ void bag_bounds(const int32_t* __restrict__ offsets, int B, int BL,
-                                           int k, int b, int& start, int& n, bool& bad) {
-  const int64_t o = static_cast<int64_t>(k) * B + b;
-  const int s = __ldg(offsets + o);
-  const int e = (b + 1 < B) ? __ldg(offsets + o + 1) : BL;
-  bad = (s < 0) || (s > e) || (e > BL);
+// The same decoder for small p (< 2^24, where every int is exact in f32).
+__device__ __forceinline__ void pair_from_flat_small(int p, int& i_out, int& j_out) {
+  int i = static_cast<int>((sqrtf(8.0f * static_cast<float>(p) + 1.0f) + 1.0f) * 0.5f);
+  if (i < 1) i = 1;
+  while (i * (i - 1) / 2 > p) --i;
+  while (i * (i + 1) / 2 <= p) ++i;
+  i_out = i;
+  j_out = p - i * (i - 1) / 2;
+}
+
+// Bag bounds of (table k, sample b) under torch's offsets rule: the bag ends
+// where the next one starts, or at T for the last bag (include_last_offset=0),
+// or at offsets[k][B] (include_last_offset=1). Invalid bounds give an empty
+// bag and raise *bad.
+__device__ __forceinline__ void bag_bounds(const BagParams& bp, int B, int k, int b, int& start,
+                                           int& n, bool& bad) {
+  const int64_t o = static_cast<int64_t>(k) * (B + bp.ilo) + b;
+  const int s = __ldg(bp.offsets + o);
+  const int e = (bp.ilo || b + 1 < B) ? __ldg(bp.offsets + o + 1) : bp.T;
+  bad = (s < 0) || (s > e) || (e > bp.T);
   start = bad ? 0 : s;
   n = bad ? 0 : e - s;
 }
 
-// Pool one bag for the columns this lane owns.
+// Pool one bag for the columns this lane owns; returns the entries used.
 //
 // A lane group of G consecutive lanes handles one bag; lane q owns the column
 // chunks q, q+G, ..., q+(CPL-1)G of the current column window (a chunk is VEC
-// consecutive floats). Rows are fetched U at a time, all U loads issued before
-// any is consumed; the bag's row ids are read once, coalesced, by the group
-// and handed out with warp shuffles. Each column is then accumulated from
-// 0.0f in bag order with one rounding per add, so the result is bit-identical
-// to the sequential f32 sum.
+// consecutive elements). Rows are fetched U at a time, all U loads issued
+// before any is consumed; the bag's row ids (and weights) are read once,
+// coalesced, by the group and handed out with warp shuffles. Each column then
+// combines the rows in bag order with one rounding per step (an add, a fused
+// multiply-add, or a comparison), so the result is bit-identical to the
+// sequential definition.
 //
 // Every lane of the warp must call this with the same `nmax` (the largest n in
 // the warp), because the shuffles run over the full warp.
-template <int VEC, int G, int CPL, int U, bool CHECK>
-__device__ __forceinline__ void pool_bag(const float* __restrict__ W, int rows_k,
-                                         const int32_t* __restrict__ idx_seg, int start, int n,
-                                         int nmax, int D, int col0, int q, int gbase,
-                                         typename VecOf<VEC>::T (&acc)[CPL], bool& oob) {
-  using V = typename VecOf<VEC>::T;
+template <class LD, int G, int CPL, int U, int POOL>
+__device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W, int rows_k,
+                                        bool check, const int32_t* __restrict__ idx_seg,
+                                        const float* __restrict__ w_seg, int start, int n,
+                                        int nmax, int D, int col0, int q, int gbase,
+                                        float (&acc)[CPL][LD::VEC], bool& oob) {
+  constexpr int VEC = LD::VEC;
   constexpr int IPL = (U + G - 1) / G;  // row ids held per lane per batch of U rows
 #pragma unroll
-  for (int m = 0; m < CPL; ++m) set_zero(acc[m]);
+  for (int m = 0; m < CPL; ++m)
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[m][e] = 0.f;
+  bool colok[CPL];
+#pragma unroll
+  for (int m = 0; m < CPL; ++m) colok[m] = col0 + (q + G * m) * VEC < D;
+  int used = 0;
 
   for (int c = 0; c < nmax; c += U) {
     int my_row[IPL];
+    float my_w[IPL];
 #pragma unroll
     for (int j = 0; j < IPL; ++j) {
       const int slot = q + G * j;
-      const int t = c + slot;
-      my_row[j] = (slot < U && t < n) ? __ldg(idx_seg + start + t) : 0;
+      const bool in = (slot < U) && (c + slot < n);
+      my_row[j] = in ? __ldg(idx_seg + start + c + slot) : 0;
+      if (POOL == kPoolWeighted) my_w[j] = in ? __ldg(w_seg + start + c + slot) : 0.f;
     }
-    V v[U][CPL];
+    typename LD::Raw v[U][CPL];
     bool use[U];
+    float wt[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int r = __shfl_sync(kFullMask, my_row[u / G], gbase + (u % G));
+      if (POOL == kPoolWeighted) wt[u] = __shfl_sync(kFullMask, my_w[u / G], gbase + (u % G));
       bool ok = (c + u) < n;
-      if (CHECK) {
-        const bool in_range = (r >= 0) && (r < rows_k);
+      if (check) {
+        const bool in_range = static_cast<unsigned>(r) < static_cast<unsigned>(rows_k);
         oob |= ok && !in_range;
         ok = ok && in_range;
       }
       use[u] = ok;
-      const float* row = W + static_cast<int64_t>(r) * D;
+      const typename LD::Elem* row = W + static_cast<int64_t>(r) * D + col0 + q * VEC;
 #pragma unroll
       for (int m = 0; m < CPL; ++m) {
-        const int col = col0 + (q + G * m) * VEC;
-        if (ok && col < D) {
-          v[u][m] = load_row_chunk(row + col, static_cast<V*>(nullptr));
-        } else {
-          set_zero(v[u][m]);
-        }
+        if (ok && colok[m]) v[u][m] = LD::load(row + G * m * VEC);
       }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (use[u]) {
 #pragma unroll
-        for (int m = 0; m < CPL; ++m) acc_add(acc[m], v[u][m]);
+        for (int m = 0; m < CPL; ++m)
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            const float x = LD::get(v[u][m], e);
+            if (POOL == kPoolSum) {
+              acc[m][e] = __fadd_rn(acc[m][e], x);
+            } else if (POOL == kPoolWeighted) {
+              acc[m][e] = __fmaf_rn(wt[u], x, acc[m][e]);
+            } else {
+              acc[m][e] = (used == 0) ? x : ((x > acc[m][e]) ? x : acc[m][e]);
+            }
+          }
+        ++used;
       }
     }
+  }
+  return used;
+}
+
+// Mean pooling: one division of the sequential sum by the entries used.
+template <int CPL, int VEC>
+__device__ __forceinline__ void finish_mean(float (&acc)[CPL][VEC], int used) {
+  if (used > 0) {
+    const float cnt = static_cast<float>(used);
+#pragma unroll
+    for (int m = 0; m < CPL; ++m)
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[m][e] = __fdiv_rn(acc[m][e], cnt);
+  }
+}
+
+// Store VEC consecutive floats (16-byte aligned when VEC is 4 or 8).
+template <int VEC>
+__device__ __forceinline__ void store_floats(float* p, const float (&a)[VEC]) {
+  if constexpr (VEC % 4 == 0) {
+#pragma unroll
+    for (int e = 0; e < VEC; e += 4)
+      *reinterpret_cast<float4*>(p + e) = make_float4(a[e], a[e + 1], a[e + 2], a[e + 3]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) p[e] = a[e];
   }
 }
 

@@ -6,10 +6,11 @@
 namespace dlrm {
 
 // Shared-memory feature block of one sample: F1p = 4*ceil((F+1)/4) rows (dense
-// first, then the F pooled vectors, then zero rows), each Dp = 4*ceil(D/4) + 4
-// floats long. The row length keeps every row 16-byte aligned for float4
-// reads, and the extra 4 floats shift consecutive rows by one 16-byte bank
-// group, so float4 reads of different rows at the same column do not collide.
+// first, then the F pooled vectors, then up to 3 filler rows), each
+// Dp = 4*ceil(D/4) + 4 floats long. The row length keeps every row 16-byte
+// aligned for float4 reads, and the extra 4 floats shift consecutive rows by
+// one 16-byte bank group, so float4 reads of different rows at the same
+// column do not collide.
 struct FeatLayout {
   int F1;   // features = F + 1
   int F1p;  // rows per sample, multiple of 4
@@ -32,30 +33,21 @@ struct FeatLayout {
 };
 
 // Zero what the dot phase reads but the loaders do not write: the columns
-// [D, 4*D4) of every row, and the whole rows [F1, F1p).
+// [D, 4*D4) of the feature rows, and the filler rows [F1, F1p). (The filler
+// rows only feed tile entries that are never stored; they are zeroed so that
+// nothing reads uninitialised memory.)
 __device__ __forceinline__ void zero_feature_padding(float* feat, const FeatLayout& Lf, int D,
                                                      int S_here) {
-  const int padc = 4 * Lf.D4 - D;
-  if (padc > 0) {
-    const int per = Lf.F1 * padc;
-    for (int e = threadIdx.x; e < S_here * per; e += blockDim.x) {
-      const int s = e / per;
-      const int rem = e - s * per;
-      const int f = rem / padc;
-      const int c = D + (rem - f * padc);
-      feat[(static_cast<int64_t>(s) * Lf.F1p + f) * Lf.Dp + c] = 0.f;
+  const int padc = 4 * Lf.D4 - D;  // 0..3
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int s = 0; s < S_here; ++s) {
+    float* base = feat + static_cast<int64_t>(s) * Lf.F1p * Lf.Dp;
+    if (padc > 0) {
+      for (int f = warp; f < Lf.F1; f += nwarps)
+        if (lane < padc) base[f * Lf.Dp + D + lane] = 0.f;
     }
-  }
-  const int extra_rows = Lf.F1p - Lf.F1;
-  if (extra_rows > 0) {
-    const int per = extra_rows * 4 * Lf.D4;
-    for (int e = threadIdx.x; e < S_here * per; e += blockDim.x) {
-      const int s = e / per;
-      const int rem = e - s * per;
-      const int f = Lf.F1 + rem / (4 * Lf.D4);
-      const int c = rem % (4 * Lf.D4);
-      feat[(static_cast<int64_t>(s) * Lf.F1p + f) * Lf.Dp + c] = 0.f;
-    }
+    const int n_extra = (Lf.F1p - Lf.F1) * Lf.Dp;
+    for (int e = threadIdx.x; e < n_extra; e += blockDim.x) base[Lf.F1 * Lf.Dp + e] = 0.f;
   }
 }
 
@@ -64,29 +56,34 @@ __device__ __forceinline__ void zero_feature_padding(float* feat, const FeatLayo
 // The pairs are covered by 4x4 tiles (I, J), I >= J, of the (F+1) x (F+1)
 // Gram matrix; the flat tile index t is decoded with the same closed form as
 // the pair index (tile (I, J) is pair (I+1, J) of a triangle one larger). A
-// task is (sample, tile, q): Q consecutive lanes split the D columns of one
-// tile (lane q takes float4 chunks q, q+Q, ...), keep the 16 partial dots in
-// registers (each float4 read from shared memory feeds 16 FMAs), and combine
-// them with xor shuffles. Lane q then stores the tile entries e = 4r + c with
-// e % Q == q that lie strictly below the diagonal and inside F+1.
+// task is (sample, tile, q): Q = 2^lq consecutive lanes split the D columns
+// of one tile (lane q takes float4 chunks q, q+Q, ...), keep the 16 partial
+// dots in registers (each float4 read from shared memory feeds 16 FMAs), and
+// combine them with xor shuffles. Lane q then stores the tile entries
+// e = 4r + c with e % Q == q that lie strictly below the diagonal and inside
+// F+1.
 //
-// out row of sample b starts at out + b * row_stride + col0; dot p of the row
-// is written at offset p.
+// The output row of sample b starts at out + b * row_stride + col0; dot p of
+// the row is written at offset p.
 __device__ __forceinline__ void dots_from_smem(const float* feat, const FeatLayout& Lf,
-                                               int S_here, int Q, float* __restrict__ out,
+                                               int S_here, int lq, float* __restrict__ out,
                                                int64_t b0, int64_t row_stride, int64_t col0) {
-  const int total = S_here * Lf.nT * Q;
+  const int Q = 1 << lq;
+  const int total = (S_here * Lf.nT) << lq;
   const int lane = threadIdx.x & 31;
   for (int base = threadIdx.x - lane; base < total; base += blockDim.x) {
     const int task = base + lane;
     const bool active = task < total;
     const int tt = active ? task : 0;
-    const int q = tt % Q;
-    const int rest = tt / Q;
-    const int t = rest % Lf.nT;
-    const int s = rest / Lf.nT;
+    const int q = tt & (Q - 1);
+    const int rest = tt >> lq;
+    int t = rest, s = 0;
+    if (S_here > 1) {
+      s = rest / Lf.nT;
+      t = rest - s * Lf.nT;
+    }
     int I1, J;
-    pair_from_flat(t, I1, J);
+    pair_from_flat_small(t, I1, J);
     const int I = I1 - 1;
     const float* fi = feat + (static_cast<int64_t>(s) * Lf.F1p + 4 * I) * Lf.Dp;
     const float* fj = feat + (static_cast<int64_t>(s) * Lf.F1p + 4 * J) * Lf.Dp;
@@ -124,15 +121,15 @@ __device__ __forceinline__ void dots_from_smem(const float* feat, const FeatLayo
     if (active) {
       float* orow = out + (b0 + s) * row_stride + col0;
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int r = 0; r < 4; ++r) {
+        const int i = 4 * I + r;
+        if (i >= Lf.F1) continue;
+        float* orow_i = orow + i * (i - 1) / 2 + 4 * J;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const int i = 4 * I + r;
-          const int j = 4 * J + c;
-          if (((4 * r + c) % Q) == q && i < Lf.F1 && j < i) {
-            orow[static_cast<int64_t>(i) * (i - 1) / 2 + j] = acc[r][c];
-          }
+          if (((4 * r + c) & (Q - 1)) == q && 4 * J + c < i) orow_i[c] = acc[r][c];
         }
+      }
     }
   }
 }

@@ -44,6 +44,8 @@ SIGNATURES = {
     "dlrm_sparse_interact_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _P]),
     "dlrm_sparse_interact_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
                                        _P, _P, _P]),
+    "embbag_pool_multi": (_I, [_P, _I, _P, _P, _I, _I, _I, _P, _P, _P]),
+    "dlrm_sparse_interact_pool": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _I, _P, _P]),
     "dlrm_pair_decode": (_I, [_I64, _I64, _P, _P, _P]),
     "dlrm_status_from_flags": (_I, [ctypes.c_int32]),
     "dlrm_status_string": (ctypes.c_char_p, [_I]),
@@ -209,6 +211,105 @@ def sparse_interact(weights: Sequence[torch.Tensor], indices: torch.Tensor,
         _check(_lib.dlrm_sparse_interact(arr, ip, op, dp, B, F, L, D, pp, xp,
                                          1 if concat_dense else 0, _stream()),
                "dlrm_sparse_interact")
+    return pooled_out, inter_out
+
+
+POOL_MODES = {"sum": 0, "mean": 1, "max": 2}
+TABLE_DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+
+
+class Bags(ctypes.Structure):
+    """``dlrm_bags_t``: where the bags are and how they pool."""
+
+    _fields_ = [("indices", ctypes.c_void_p), ("offsets", ctypes.c_void_p),
+                ("per_sample_weights", ctypes.c_void_p), ("T", ctypes.c_int64),
+                ("include_last_offset", ctypes.c_int), ("mode", ctypes.c_int)]
+
+
+def _general_args(weights, indices, offsets, mode, per_sample_weights, include_last_offset,
+                  checked):
+    F = len(weights)
+    if not 1 <= F <= DLRM_MAX_TABLES:
+        raise ValueError(f"table count must be in [1, {DLRM_MAX_TABLES}] (got {F})")
+    dtype = weights[0].dtype
+    if dtype not in TABLE_DTYPES:
+        raise TypeError(f"tables must be float32 or bfloat16 (got {dtype})")
+    D = weights[0].shape[1]
+    for k, w in enumerate(weights):
+        _dev(w, f"weights[{k}]", dtype)
+        if w.dim() != 2 or w.shape[1] != D:
+            raise ValueError(f"weights[{k}] must be (rows, {D})")
+    arr = (ctypes.c_void_p * F)(*[w.data_ptr() for w in weights])
+    rows = (ctypes.c_int64 * F)(*[w.shape[0] for w in weights]) if checked else None
+    if offsets.dim() != 2 or offsets.shape[0] != F:
+        raise ValueError(f"offsets must be (F={F}, B{' + 1' if include_last_offset else ''})")
+    B = offsets.shape[1] - (1 if include_last_offset else 0)
+    T = indices.numel() // F if F else 0
+    if indices.numel() != F * T:
+        raise ValueError("indices must hold F equal segments")
+    bags = Bags(_dev(indices, "indices", torch.int32) if indices.numel() else None,
+                _dev(offsets, "offsets", torch.int32),
+                _dev(per_sample_weights, "per_sample_weights", torch.float32)
+                if per_sample_weights is not None else None,
+                T, 1 if include_last_offset else 0, POOL_MODES[mode])
+    if per_sample_weights is not None and per_sample_weights.numel() != F * T:
+        raise ValueError("per_sample_weights must match indices")
+    return arr, TABLE_DTYPES[dtype], rows, bags, F, D, B
+
+
+def embbag_pool_multi(weights: Sequence[torch.Tensor], indices: torch.Tensor,
+                      offsets: torch.Tensor, *, mode: str = "sum",
+                      per_sample_weights: Optional[torch.Tensor] = None,
+                      include_last_offset: bool = False, checked: bool = False,
+                      status: Optional[torch.Tensor] = None,
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """General multi-table EmbeddingBag ``(B, F, D)`` f32 in one launch.
+
+    ``weights``: F float32 or bfloat16 tables; ``indices`` (and
+    ``per_sample_weights``) ``(F, T)``; ``offsets`` ``(F, B)`` or ``(F, B+1)``
+    with ``include_last_offset``; ``mode`` sum/mean/max. ``checked`` checks
+    indices against the table sizes (flags in ``status``).
+    """
+    arr, dt, rows, bags, F, D, B = _general_args(weights, indices, offsets, mode,
+                                                 per_sample_weights, include_last_offset,
+                                                 checked)
+    if out is None:
+        out = torch.empty((B, F, D), dtype=torch.float32, device=weights[0].device)
+    if out.numel() != B * F * D:
+        raise ValueError("out must be (B, F, D)")
+    sp = _dev(status, "status", torch.int32) if status is not None else None
+    _check(_lib.embbag_pool_multi(arr, dt, rows, ctypes.byref(bags), B, F, D,
+                                  _dev(out, "out", torch.float32), sp, _stream()),
+           "embbag_pool_multi")
+    return out
+
+
+def sparse_interact_pool(weights: Sequence[torch.Tensor], indices: torch.Tensor,
+                         offsets: torch.Tensor, dense: torch.Tensor, *, mode: str = "sum",
+                         per_sample_weights: Optional[torch.Tensor] = None,
+                         include_last_offset: bool = False, checked: bool = False,
+                         status: Optional[torch.Tensor] = None, concat_dense: bool = False,
+                         want_pooled: bool = True, pooled_out=None, inter_out=None):
+    """Fused stage over the general bag description: ``(pooled or None, inter)``."""
+    arr, dt, rows, bags, F, D, B = _general_args(weights, indices, offsets, mode,
+                                                 per_sample_weights, include_last_offset,
+                                                 checked)
+    if tuple(dense.shape) != (B, D):
+        raise ValueError(f"dense must be ({B}, {D})")
+    P = (F + 1) * F // 2
+    dev = weights[0].device
+    if want_pooled and pooled_out is None:
+        pooled_out = torch.empty((B, F, D), dtype=torch.float32, device=dev)
+    if inter_out is None:
+        inter_out = torch.empty((B, D + P if concat_dense else P), dtype=torch.float32,
+                                device=dev)
+    pp = _dev(pooled_out, "pooled_out", torch.float32) if pooled_out is not None else None
+    sp = _dev(status, "status", torch.int32) if status is not None else None
+    _check(_lib.dlrm_sparse_interact_pool(arr, dt, rows, ctypes.byref(bags),
+                                          _dev(dense, "dense", torch.float32), B, F, D, pp,
+                                          _dev(inter_out, "inter_out", torch.float32),
+                                          1 if concat_dense else 0, sp, _stream()),
+           "dlrm_sparse_interact_pool")
     return pooled_out, inter_out
 
 

@@ -82,6 +82,41 @@ typedef enum {
 #define DLRM_FLAG_INDEX_OOB 1
 #define DLRM_FLAG_OFFSETS 2
 
+/* Pooling of a bag's rows (torch.nn.EmbeddingBag modes). The pages implement
+ * only SUM and name the others as what a later model would need (movement.rs,
+ * translate_embedding_bag_forward_only). */
+typedef enum {
+    DLRM_POOL_SUM = 0,  /* sum in bag order, one rounding per add; with
+                           per-sample weights one fused multiply-add per entry */
+    DLRM_POOL_MEAN = 1, /* the SUM result divided once by the entry count */
+    DLRM_POOL_MAX = 2   /* first entry, then (x > acc ? x : acc) in bag order */
+} dlrm_pool_mode_t;     /* an empty bag gives 0 in every mode */
+
+/* Element type of the tables. A bf16 table holds the upper 16 bits of each
+ * f32 value; rows are widened to f32 exactly and pooled in f32. */
+typedef enum { DLRM_TABLE_F32 = 0, DLRM_TABLE_BF16 = 1 } dlrm_table_dtype_t;
+
+/* General bag description (ragged bags, weights, modes).
+ *   indices  : dev int32, F segments of T entries (entry t of table k at
+ *              indices[k*T + t]); may be NULL iff T == 0.
+ *   offsets  : dev int32, (F, B), or (F, B+1) when include_last_offset != 0.
+ *              Bag b of table k is [offsets[k][b], end) with end =
+ *              offsets[k][b+1], or T for the last bag when
+ *              include_last_offset == 0. Entries outside every bag are never
+ *              read.
+ *   per_sample_weights : dev f32 (F, T), same layout as indices, or NULL.
+ *              Only with DLRM_POOL_SUM (else DLRM_ERR_ARG).
+ *   T        : entries per table, 0 <= T <= INT32_MAX.
+ *   mode     : dlrm_pool_mode_t. */
+typedef struct {
+    const int32_t* indices;
+    const int32_t* offsets;
+    const float* per_sample_weights;
+    int64_t T;
+    int include_last_offset;
+    int mode;
+} dlrm_bags_t;
+
 /*
  * embbag_sum_multi -- one launch pools all F tables.
  *   weights : host array[F] of dev pointers; table k is (rows_k, D) f32.
@@ -111,6 +146,26 @@ DLRM_API int embbag_sum_multi(const float* const* weights, const int32_t* indice
 DLRM_API int embbag_sum_multi_ex(const float* const* weights, const int64_t* rows,
                         const int32_t* indices, const int32_t* offsets, int B, int F, int L,
                         int D, float* out, int32_t* status_dev, dlrm_stream_t stream);
+
+/*
+ * embbag_pool_multi -- the general multi-table EmbeddingBag in one launch.
+ *   weights     : host array[F] of dev pointers; table k is (rows_k, D) of
+ *                 table_dtype (dlrm_table_dtype_t).
+ *   rows        : host array[F] of row counts, or NULL. If given, indices
+ *                 outside [0, rows[k]) are skipped (they add nothing and do not
+ *                 count toward a mean) and flagged; if NULL, indices are
+ *                 trusted.
+ *   bags        : host pointer to the bag description, read during the call.
+ *   out         : dev f32 (B, F, D).
+ *   status_dev  : dev int32 or NULL; zeroed on `stream`, then DLRM_FLAG_* are
+ *                 OR-ed in (bad offsets always, bad indices when rows != NULL).
+ * A bag with invalid offsets (start < 0, start > end, end > T) pools as empty.
+ * With 16-byte aligned tables and output, f32 rows use 128-bit loads when
+ * D % 4 == 0 and bf16 rows when D % 8 == 0; otherwise scalar loads, same bits.
+ */
+DLRM_API int embbag_pool_multi(const void* const* weights, int table_dtype, const int64_t* rows,
+                               const dlrm_bags_t* bags, int B, int F, int D, float* out,
+                               int32_t* status_dev, dlrm_stream_t stream);
 
 /*
  * interact_lower_tri -- the pairwise-dot interaction alone.
@@ -153,6 +208,17 @@ DLRM_API int dlrm_sparse_interact_ex(const float* const* weights, const int64_t*
                             const int32_t* indices, const int32_t* offsets, const float* dense,
                             int B, int F, int L, int D, float* pooled_out, float* inter_out,
                             int concat_dense, int32_t* status_dev, dlrm_stream_t stream);
+
+/*
+ * dlrm_sparse_interact_pool -- the fused stage with the general bag
+ * description: arguments as for embbag_pool_multi, plus dense, pooled_out
+ * (nullable), inter_out and concat_dense as for dlrm_sparse_interact.
+ */
+DLRM_API int dlrm_sparse_interact_pool(const void* const* weights, int table_dtype,
+                                       const int64_t* rows, const dlrm_bags_t* bags,
+                                       const float* dense, int B, int F, int D,
+                                       float* pooled_out, float* inter_out, int concat_dense,
+                                       int32_t* status_dev, dlrm_stream_t stream);
 
 /*
  * dlrm_sparse_interact_host -- the whole stage from host memory, for callers

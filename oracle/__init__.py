@@ -11,6 +11,11 @@ ctypes and marshals numpy arrays. What each function follows on the pages
 
 * :meth:`Oracle.embbag_sum_multi` -- embedding_bag.rs, module doc comment and
   the multi-table section doc comment (pooled sum over K tables).
+* :meth:`Oracle.embbag_pool_multi` -- the same pooling generalised the way
+  torch.nn.EmbeddingBag defines it (ragged bags, include_last_offset,
+  per-sample weights, mean/max, bf16 tables), which movement.rs
+  (translate_embedding_bag_forward_only) names as the extension a later
+  model would need.
 * :meth:`Oracle.interact_lower_tri` -- dlrm_interact.rs, module doc comment
   (the strict-lower-triangle dot products) and the stacked-kernel doc comment
   (feature 0 = dense vector, features 1..N = pooled embeddings).
@@ -38,6 +43,9 @@ BAD_ARG = 1
 BAD_OFFSETS = 2
 INDEX_OOB = 3
 
+POOL_SUM, POOL_MEAN, POOL_MAX = 0, 1, 2
+MODES = {"sum": POOL_SUM, "mean": POOL_MEAN, "max": POOL_MAX}
+
 CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math"]
 
 
@@ -52,7 +60,7 @@ class OracleError(RuntimeError):
 def compile_source(src: str, lib: str) -> str:
     """Compile one C source file into a shared library with the oracle's flags."""
     tmp = lib + f".tmp{os.getpid()}"
-    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, src])
+    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, src, "-lm"])
     os.replace(tmp, lib)
     return lib
 
@@ -84,6 +92,9 @@ class Oracle:
         lib.oracle_embbag_sum_multi.restype = I
         lib.oracle_interact_lower_tri.argtypes = [P, P, I, I, I, P, I, P, P]
         lib.oracle_interact_lower_tri.restype = I
+        lib.oracle_embbag_pool_multi.argtypes = [P, I, P, P, P, P, ctypes.c_int64, I, I, I, I,
+                                                 I, P]
+        lib.oracle_embbag_pool_multi.restype = I
         lib.oracle_pair_list.argtypes = [I, P, P]
         lib.oracle_pair_list.restype = ctypes.c_int64
         self.lib = lib
@@ -114,6 +125,37 @@ class Oracle:
         if rc != OK:
             raise OracleError(rc, "embbag_sum_multi")
         return (out, o64, oab) if with_f64 else out
+
+    def embbag_pool_multi(self, weights: Sequence[np.ndarray], indices: np.ndarray,
+                          offsets: np.ndarray, B: int, *, mode: str = "sum",
+                          per_sample_weights: np.ndarray | None = None,
+                          include_last_offset: bool = False):
+        """General pooling ``(B, F, D)`` f32: ragged bags, weights, sum/mean/max.
+
+        ``weights[k]`` is ``(rows_k, D)`` float32, or uint16 holding bf16 bit
+        patterns; ``indices`` (and ``per_sample_weights``) are ``(F, T)``;
+        ``offsets`` is ``(F, B)``, or ``(F, B+1)`` with ``include_last_offset``.
+        """
+        F = len(weights)
+        bf16 = weights[0].dtype == np.uint16
+        ws = [np.ascontiguousarray(w, dtype=np.uint16 if bf16 else np.float32) for w in weights]
+        D = int(ws[0].shape[1])
+        ptrs = (ctypes.c_void_p * F)(*[w.ctypes.data for w in ws])
+        rows = np.array([w.shape[0] for w in ws], dtype=np.int64)
+        idx = np.ascontiguousarray(indices, dtype=np.int32).reshape(F, -1)
+        T = idx.shape[1]
+        off = np.ascontiguousarray(offsets, dtype=np.int32).reshape(F, B + (1 if include_last_offset else 0))
+        psw = None
+        if per_sample_weights is not None:
+            psw = np.ascontiguousarray(per_sample_weights, dtype=np.float32).reshape(F, T)
+        out = np.empty((B, F, D), dtype=np.float32)
+        rc = self.lib.oracle_embbag_pool_multi(ctypes.cast(ptrs, ctypes.c_void_p), 1 if bf16 else 0,
+                                               _ptr(rows), _ptr(idx), _ptr(off), _ptr(psw), T,
+                                               1 if include_last_offset else 0, MODES[mode], B, F,
+                                               D, _ptr(out))
+        if rc != OK:
+            raise OracleError(rc, "embbag_pool_multi")
+        return out
 
     def interact_lower_tri(self, dense: np.ndarray, emb: np.ndarray, *,
                            concat_dense: bool = False, with_f64: bool = False):
@@ -183,3 +225,7 @@ def sparse_interact(*a, **k):
 
 def pair_list(*a, **k):
     return default().pair_list(*a, **k)
+
+
+def embbag_pool_multi(*a, **k):
+    return default().embbag_pool_multi(*a, **k)

@@ -37,8 +37,10 @@
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off (no -ffast-math),
  * so every f32 addition is one IEEE single-precision round-to-nearest add.
  */
+#include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <string.h>
 
 /* Return codes of the oracle (its own; not shared with the library). */
 #define ORACLE_OK 0
@@ -124,6 +126,113 @@ int oracle_embbag_sum_multi(const float* const* weights, const int64_t* rows,
                 out[o] = acc;
                 if (out_f64) out_f64[o] = acc64;
                 if (out_absum) out_absum[o] = absum;
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------
+ * General pooling: ragged bags, include_last_offset, per-sample weights,
+ * sum / mean / max, f32 or bf16 tables.
+ *
+ * The pages support only the fixed-stride, unweighted sum over f32 tables and
+ * name the rest as what a later model would need (movement.rs,
+ * translate_embedding_bag_forward_only: mean/max and per_sample_weights are
+ * rejected with an error that says to extend it when a model needs them).
+ * The semantics below are torch.nn.EmbeddingBag's, with these readings:
+ *   - weighted sum: each step is one fused multiply-add, acc = fma(w_t, x, acc),
+ *     from 0.0f in bag order (one rounding per entry);
+ *   - mean: the f32 sum in bag order, then one division by the entry count;
+ *     an empty bag gives 0;
+ *   - max: the first entry, then acc = (x > acc) ? x : acc in bag order (ties,
+ *     including -0 vs +0, keep the earlier value); an empty bag gives 0;
+ *   - bf16 tables: a bf16 value is the upper 16 bits of an f32, so it is
+ *     widened exactly by shifting its bits up by 16 before any arithmetic.
+ * ------------------------------------------------------------------------ */
+#define ORACLE_POOL_SUM 0
+#define ORACLE_POOL_MEAN 1
+#define ORACLE_POOL_MAX 2
+#define ORACLE_TABLE_F32 0
+#define ORACLE_TABLE_BF16 1
+
+static float bf16_bits_to_f32(uint16_t h) {
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static float table_value(const void* W, int dtype, int64_t row, int D, int d) {
+    if (dtype == ORACLE_TABLE_BF16) return bf16_bits_to_f32(((const uint16_t*)W)[row * D + d]);
+    return ((const float*)W)[row * D + d];
+}
+
+/* Bag b of table k when each table's offsets row holds B (+1) entries. */
+static int bag_bounds_general(const int32_t* offsets, int B, int64_t T, int ilo, int k, int b,
+                              int64_t* start, int64_t* end) {
+    const int64_t row = (int64_t)B + (ilo ? 1 : 0);
+    int64_t s = offsets[(int64_t)k * row + b];
+    int64_t e = (ilo || b + 1 < B) ? (int64_t)offsets[(int64_t)k * row + b + 1] : T;
+    if (s < 0 || s > e || e > T) return ORACLE_BAD_OFFSETS;
+    *start = s;
+    *end = e;
+    return ORACLE_OK;
+}
+
+/*
+ * weights[k] : rows[k] x D table, f32 or bf16 (raw 16-bit patterns)
+ * indices    : (F, T) int32, table-major; psw : (F, T) f32 or NULL (sum only)
+ * offsets    : (F, B) int32, or (F, B+1) with include_last_offset
+ * out        : (B, F, D) f32
+ * Only entries covered by some bag are read and must lie in [0, rows[k]).
+ */
+int oracle_embbag_pool_multi(const void* const* weights, int dtype, const int64_t* rows,
+                             const int32_t* indices, const int32_t* offsets, const float* psw,
+                             int64_t T, int include_last_offset, int mode, int B, int F, int D,
+                             float* out) {
+    if (B < 1 || F < 1 || F > ORACLE_MAX_TABLES || D < 1 || T < 0 || T > INT32_MAX)
+        return ORACLE_BAD_ARG;
+    if (mode != ORACLE_POOL_SUM && mode != ORACLE_POOL_MEAN && mode != ORACLE_POOL_MAX)
+        return ORACLE_BAD_ARG;
+    if (dtype != ORACLE_TABLE_F32 && dtype != ORACLE_TABLE_BF16) return ORACLE_BAD_ARG;
+    if (psw && mode != ORACLE_POOL_SUM) return ORACLE_BAD_ARG;
+    if (!weights || !rows || !offsets || !out) return ORACLE_BAD_ARG;
+    if (T > 0 && !indices) return ORACLE_BAD_ARG;
+
+    for (int k = 0; k < F; ++k) {
+        if (!weights[k] || rows[k] < 0) return ORACLE_BAD_ARG;
+        for (int b = 0; b < B; ++b) {
+            int64_t s, e;
+            int rc = bag_bounds_general(offsets, B, T, include_last_offset, k, b, &s, &e);
+            if (rc) return rc;
+            for (int64_t t = s; t < e; ++t) {
+                int32_t r = indices[(int64_t)k * T + t];
+                if (r < 0 || (int64_t)r >= rows[k]) return ORACLE_INDEX_OOB;
+            }
+        }
+    }
+
+    for (int b = 0; b < B; ++b) {
+        for (int k = 0; k < F; ++k) {
+            int64_t s, e;
+            bag_bounds_general(offsets, B, T, include_last_offset, k, b, &s, &e);
+            const int32_t* idx = indices ? indices + (int64_t)k * T : NULL;
+            const float* wk = psw ? psw + (int64_t)k * T : NULL;
+            for (int d = 0; d < D; ++d) {
+                float acc = 0.0f;
+                for (int64_t t = s; t < e; ++t) {
+                    float x = table_value(weights[k], dtype, idx[t], D, d);
+                    if (mode == ORACLE_POOL_MAX) {
+                        acc = (t == s) ? x : ((x > acc) ? x : acc);
+                    } else if (wk) {
+                        acc = fmaf(wk[t], x, acc);
+                    } else {
+                        acc = acc + x;
+                    }
+                }
+                if (mode == ORACLE_POOL_MEAN && e > s) acc = acc / (float)(e - s);
+                out[((int64_t)b * F + k) * D + d] = acc;
             }
         }
     }

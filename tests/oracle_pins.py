@@ -341,6 +341,154 @@ def pin_rejects_bad_input(orc):
                  BAD_ARG)
 
 
+# --------------------------------------------------------------------------- general pooling
+
+def _ragged(rng, F, B, T, ilo):
+    off = np.sort(rng.integers(0, T + 1, (F, B + (1 if ilo else 0))), axis=1).astype(np.int32)
+    off[:, 0] = 0
+    if ilo:
+        off[:, -1] = T
+    return off
+
+
+def _torch_bag(idx_k, w_k, off_k, mode, psw_k=None, ilo=False):
+    return torch.nn.functional.embedding_bag(
+        torch.from_numpy(idx_k).long(), torch.from_numpy(w_k), torch.from_numpy(off_k).long(),
+        mode=mode, per_sample_weights=None if psw_k is None else torch.from_numpy(psw_k),
+        include_last_offset=ilo).numpy()
+
+
+def pin_pool_modes_vs_torch(orc):
+    """sum / mean / max, ragged bags, both offset conventions, against torch.
+
+    Sums and means are compared with torch in fp64 within the f32 error of a
+    sequential sum; max is exact in any precision, so it is compared bit for
+    bit with torch's f32 max mode.
+    """
+    rng = np.random.default_rng(21)
+    B, F, N, D, T = 9, 3, 40, 6, 50
+    ws = [rng.normal(0, 0.1, (N, D)).astype(np.float32) for _ in range(F)]
+    idx = rng.integers(0, N, (F, T)).astype(np.int32)
+    for ilo in (False, True):
+        off = _ragged(rng, F, B, T, ilo)
+        for mode in ("sum", "mean", "max"):
+            out = orc.embbag_pool_multi(ws, idx, off, B, mode=mode, include_last_offset=ilo)
+            for k in range(F):
+                if mode == "max":
+                    ref = _torch_bag(idx[k], ws[k], off[k], "max", ilo=ilo)
+                    assert np.array_equal(out[:, k], ref), (ilo, mode, k)
+                    continue
+                ref = _torch_bag(idx[k], ws[k].astype(np.float64), off[k], mode, ilo=ilo)
+                ends = off[k, 1:] if ilo else np.append(off[k, 1:], T)
+                n = (ends - off[k, :B]).astype(np.float64)
+                absum = _torch_bag(idx[k], np.abs(ws[k]).astype(np.float64), off[k], "sum",
+                                   ilo=ilo)
+                scale = absum / np.maximum(n, 1)[:, None] if mode == "mean" else absum
+                tol = (n[:, None] + 1) * U32 * scale
+                assert np.all(np.abs(out[:, k] - ref) <= tol), (ilo, mode, k)
+
+
+def pin_weighted_sum_vs_torch(orc):
+    """per_sample_weights: sum_t w_t * W[idx_t] against torch in fp64."""
+    rng = np.random.default_rng(22)
+    B, F, N, D, T = 7, 2, 30, 5, 40
+    ws = [rng.normal(0, 0.1, (N, D)).astype(np.float32) for _ in range(F)]
+    idx = rng.integers(0, N, (F, T)).astype(np.int32)
+    psw = rng.normal(1.0, 0.5, (F, T)).astype(np.float32)
+    off = _ragged(rng, F, B, T, False)
+    out = orc.embbag_pool_multi(ws, idx, off, B, per_sample_weights=psw)
+    for k in range(F):
+        ref = _torch_bag(idx[k], ws[k].astype(np.float64), off[k], "sum",
+                         psw[k].astype(np.float64))
+        absum = _torch_bag(idx[k], np.abs(ws[k]).astype(np.float64), off[k], "sum",
+                           np.abs(psw[k]).astype(np.float64))
+        n = np.diff(np.append(off[k], T)).astype(np.float64)
+        assert np.all(np.abs(out[:, k] - ref) <= (n[:, None] + 1) * U32 * absum), k
+
+
+def pin_weighted_sum_exact_cases(orc):
+    """Unit weights give the plain sum bit for bit; dyadic weights are exact."""
+    rng = np.random.default_rng(23)
+    B, F, N, D, L = 6, 2, 20, 4, 5
+    ws = [rng.normal(0, 0.1, (N, D)).astype(np.float32) for _ in range(F)]
+    idx = rng.integers(0, N, (F, B * L)).astype(np.int32)
+    off = _fixed_offsets(F, B, L)
+    plain = orc.embbag_pool_multi(ws, idx, off, B)
+    ones = orc.embbag_pool_multi(ws, idx, off, B, per_sample_weights=np.ones((F, B * L)))
+    assert np.array_equal(plain.view(np.uint32), ones.view(np.uint32))
+    assert np.array_equal(plain, orc.embbag_sum_multi(ws, idx, off, B, L))
+    dy = [_dyadic_table(rng, N, D) for _ in range(F)]
+    wts = (2.0 ** rng.integers(-3, 4, (F, B * L))).astype(np.float32)
+    out = orc.embbag_pool_multi(dy, idx, off, B, per_sample_weights=wts)
+    for b in range(B):
+        for k in range(F):
+            sl = slice(b * L, (b + 1) * L)
+            exact = sum(Fraction(float(wt)) * np.vectorize(Fraction)(dy[k][r].astype(np.float64))
+                        for wt, r in zip(wts[k, sl], idx[k, sl]))
+            assert all(Fraction(float(o)) == e for o, e in zip(out[b, k], exact)), (b, k)
+
+
+def pin_mean_and_max_closed_forms(orc):
+    """Mean of L copies of a dyadic row is the row; max equals numpy's maximum."""
+    rng = np.random.default_rng(24)
+    B, F, N, D, L = 5, 3, 12, 7, 6
+    dy = [_dyadic_table(rng, N, D) for _ in range(F)]
+    r = rng.integers(0, N, (F, B))
+    idx = np.repeat(r, L, axis=1).astype(np.int32)
+    off = _fixed_offsets(F, B, L)
+    mean = orc.embbag_pool_multi(dy, idx, off, B, mode="mean")
+    for k in range(F):
+        assert np.array_equal(mean[:, k], dy[k][r[k]]), k
+    ws = [rng.normal(0, 1, (N, D)).astype(np.float32) for _ in range(F)]
+    idx = rng.integers(0, N, (F, B * L)).astype(np.int32)
+    mx = orc.embbag_pool_multi(ws, idx, off, B, mode="max")
+    for k in range(F):
+        ref = ws[k][idx[k]].reshape(B, L, D).max(axis=1)
+        assert np.array_equal(mx[:, k], ref), k
+    # empty bags give 0 in every mode
+    zoff = np.zeros((F, B), np.int32)
+    for mode in ("sum", "mean", "max"):
+        z = orc.embbag_pool_multi(ws, np.zeros((F, 0), np.int32), zoff, B, mode=mode)
+        assert np.array_equal(z.view(np.uint32), np.zeros_like(z).view(np.uint32)), mode
+
+
+def pin_bf16_tables_widen_exactly(orc):
+    """bf16 tables pool exactly like their f32 widening (done by torch)."""
+    rng = np.random.default_rng(25)
+    B, F, N, D, T = 8, 2, 25, 6, 30
+    tb = [torch.from_numpy(rng.normal(0, 0.3, (N, D)).astype(np.float32)).bfloat16()
+          for _ in range(F)]
+    bits = [t.view(torch.int16).numpy().view(np.uint16) for t in tb]
+    wide = [t.float().numpy() for t in tb]
+    idx = rng.integers(0, N, (F, T)).astype(np.int32)
+    off = _ragged(rng, F, B, T, False)
+    psw = rng.normal(0, 1, (F, T)).astype(np.float32)
+    for mode, p in (("sum", None), ("sum", psw), ("mean", None), ("max", None)):
+        a = orc.embbag_pool_multi(bits, idx, off, B, mode=mode, per_sample_weights=p)
+        b = orc.embbag_pool_multi(wide, idx, off, B, mode=mode, per_sample_weights=p)
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32)), mode
+
+
+def pin_general_pooling_rejects(orc):
+    """Weights outside sum mode, bad offsets and covered out-of-range indices."""
+    from oracle import BAD_ARG, BAD_OFFSETS, INDEX_OOB
+
+    ws = [np.zeros((5, 2), np.float32)]
+    idx = np.array([[0, 1, 2, 3, 99]], np.int32)  # entry 4 lies in no bag
+    off = np.array([[0, 2, 4]], np.int32)
+    orc.embbag_pool_multi(ws, idx, off, 2, include_last_offset=True)
+    _expect_code(lambda: orc.embbag_pool_multi(ws, idx, off[:, :2], 2), INDEX_OOB)
+    _expect_code(lambda: orc.embbag_pool_multi(ws, np.array([[0, 5, 2, 3, 0]], np.int32), off, 2,
+                                               include_last_offset=True), INDEX_OOB)
+    _expect_code(lambda: orc.embbag_pool_multi(ws, np.array([[0, 1, -1, 3, 0]], np.int32), off,
+                                               2, include_last_offset=True), INDEX_OOB)
+    _expect_code(lambda: orc.embbag_pool_multi(ws, idx, np.array([[0, 3, 2]], np.int32), 2,
+                                               include_last_offset=True), BAD_OFFSETS)
+    _expect_code(lambda: orc.embbag_pool_multi(ws, idx, off, 2, include_last_offset=True,
+                                               mode="mean",
+                                               per_sample_weights=np.ones((1, 5))), BAD_ARG)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 

@@ -32,7 +32,7 @@ def ops():
 def test_header_declares_the_stage_entry_points():
     names = _declared()
     assert {"embbag_sum_multi", "interact_lower_tri", "dlrm_sparse_interact"} <= names
-    assert len(names) == 11
+    assert len(names) == 13
 
 
 def test_library_exports_every_declared_symbol(ops):
@@ -107,6 +107,38 @@ def test_fused_and_interact_host_checks(ops):
     assert lib.dlrm_pair_decode(0, -1, FAKE, FAKE, None) == -8
     assert lib.dlrm_pair_decode((1 << 31) - 2, 5, FAKE, FAKE, None) == -8
     assert lib.dlrm_pair_decode(0, 5, None, FAKE, None) == -1
+    assert lib.dlrm_launch_count() == 0
+
+
+def test_general_pooling_host_checks(ops):
+    lib = ops._lib
+    w = _ptrs(FAKE, FAKE)
+    bags = ops.Bags(FAKE, FAKE, None, 8, 0, 0)
+    assert lib.embbag_pool_multi(w, 0, None, None, 4, 2, 8, FAKE, None, None) == -1
+    assert lib.embbag_pool_multi(w, 2, None, ctypes.byref(bags), 4, 2, 8, FAKE, None, None) == -8
+    bad_mode = ops.Bags(FAKE, FAKE, None, 8, 0, 7)
+    assert lib.embbag_pool_multi(w, 0, None, ctypes.byref(bad_mode), 4, 2, 8, FAKE, None,
+                                 None) == -8
+    psw_mean = ops.Bags(FAKE, FAKE, FAKE, 8, 0, 1)
+    assert lib.embbag_pool_multi(w, 0, None, ctypes.byref(psw_mean), 4, 2, 8, FAKE, None,
+                                 None) == -8
+    neg_t = ops.Bags(FAKE, FAKE, None, -1, 0, 0)
+    assert lib.embbag_pool_multi(w, 0, None, ctypes.byref(neg_t), 4, 2, 8, FAKE, None,
+                                 None) == -2
+    no_idx = ops.Bags(None, FAKE, None, 8, 0, 0)
+    assert lib.embbag_pool_multi(w, 0, None, ctypes.byref(no_idx), 4, 2, 8, FAKE, None,
+                                 None) == -1
+    # bf16 tables need 2-byte alignment, f32 tables 4-byte
+    w_odd = _ptrs(FAKE + 2, FAKE)
+    assert lib.embbag_pool_multi(w_odd, 0, None, ctypes.byref(bags), 4, 2, 8, FAKE, None,
+                                 None) == -3
+    assert lib.embbag_pool_multi(w_odd, 1, None, ctypes.byref(bags), 4, 2, 8, None, None,
+                                 None) == -1
+    rows = (ctypes.c_int64 * 2)(5, -1)
+    assert lib.embbag_pool_multi(w, 0, rows, ctypes.byref(bags), 4, 2, 8, FAKE, None,
+                                 None) == -8
+    assert lib.dlrm_sparse_interact_pool(w, 0, None, ctypes.byref(bags), None, 4, 2, 8, None,
+                                         FAKE, 0, None, None) == -1
     assert lib.dlrm_launch_count() == 0
 
 

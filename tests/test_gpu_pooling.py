@@ -1,0 +1,179 @@
+"""GPU parity of the general pooling entry points against the oracle.
+
+Ragged bags, include_last_offset, per-sample weights, sum / mean / max and
+bf16 tables, through ``embbag_pool_multi`` and the fused
+``dlrm_sparse_interact_pool``. Pooled values are compared bit for bit; dots
+within 1e-5 * S_ij.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dlrm_embedding_bag_b200 import synthetic as syn
+from gpu_cases import assert_bits_equal, assert_dots_close
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def ops():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from dlrm_embedding_bag_b200 import ops as _ops
+
+    return _ops
+
+
+def _host_bits(t: torch.Tensor) -> np.ndarray:
+    """Host copy of a table: f32 values, or bf16 bit patterns as uint16."""
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+    return t.cpu().numpy()
+
+
+def _case(seed, B, F, N, D, T, dtype, ilo, empty_frac=0.2):
+    rng = np.random.default_rng(seed)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    weights = [torch.empty((N, D), device=DEV).normal_(0, 0.3, generator=g).to(dtype)
+               for _ in range(F)]
+    idx = rng.integers(0, N, (F, T)).astype(np.int32)
+    nb = B + (1 if ilo else 0)
+    off = np.sort(rng.integers(0, T + 1, (F, nb)), axis=1).astype(np.int32)
+    off[:, 0] = 0
+    if ilo:
+        off[:, -1] = rng.integers(T // 2, T + 1, F)  # entries past the last bag are unused
+        off = np.minimum(off, off[:, -1:])
+    rep = rng.random((F, nb)) < empty_frac
+    for k in range(F):
+        for b in range(1, nb - (1 if ilo else 0)):
+            if rep[k, b]:
+                off[k, b] = off[k, b - 1]
+    psw = rng.normal(1.0, 0.5, (F, T)).astype(np.float32)
+    dense = torch.empty((B, D), device=DEV).normal_(0, 1, generator=g)
+    return weights, idx, off, psw, dense
+
+
+SHAPES = [  # (B, F, N, D, T)
+    (37, 3, 50, 64, 300),
+    (16, 8, 200, 128, 900),
+    (9, 5, 40, 16, 60),
+    (21, 2, 30, 24, 90),      # bf16: D % 8 == 0; f32: D % 4 == 0
+    (13, 4, 30, 20, 70),      # bf16 scalar path (D % 8 != 0), f32 vector path
+    (11, 3, 25, 7, 40),       # both scalar
+    (6, 2, 20, 264, 30),      # two column windows
+    (70, 26, 500, 64, 2000),
+]
+VARIANTS = [("sum", False), ("sum", True), ("mean", False), ("max", False)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B{}_F{}_N{}_D{}_T{}".format(*s))
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("ilo", [False, True], ids=["", "last_offset"])
+def test_general_pooling(ops, shape, dtype, ilo):
+    B, F, N, D, T = shape
+    weights, idx, off, psw, dense = _case(sum(shape) + (7 if ilo else 0), B, F, N, D, T, dtype,
+                                          ilo)
+    ws = [_host_bits(w) for w in weights]
+    idx_d = torch.from_numpy(idx).to(DEV)
+    off_d = torch.from_numpy(off).to(DEV)
+    psw_d = torch.from_numpy(psw).to(DEV)
+    for mode, weighted in VARIANTS:
+        p = psw if weighted else None
+        ref = oracle.embbag_pool_multi(ws, idx, off, B, mode=mode, per_sample_weights=p,
+                                       include_last_offset=ilo)
+        what = f"{shape} {dtype} ilo={ilo} {mode}{' weighted' if weighted else ''}"
+        out = ops.embbag_pool_multi(weights, idx_d, off_d, mode=mode,
+                                    per_sample_weights=psw_d if weighted else None,
+                                    include_last_offset=ilo)
+        fp, fi = ops.sparse_interact_pool(weights, idx_d, off_d, dense, mode=mode,
+                                          per_sample_weights=psw_d if weighted else None,
+                                          include_last_offset=ilo, concat_dense=True)
+        torch.cuda.synchronize()
+        assert_bits_equal(out, ref, what + " embbag_pool_multi")
+        assert_bits_equal(fp, ref, what + " fused pooled")
+        ref_i, _, bound = oracle.interact_lower_tri(dense.cpu().numpy(), ref, concat_dense=True,
+                                                    with_f64=True)
+        assert_bits_equal(fi[:, :D], ref_i[:, :D], what + " fused dense part")
+        assert_dots_close(fi[:, D:], ref_i[:, D:], bound, what + " fused dots")
+
+
+def test_plain_entry_points_equal_general_sum(ops):
+    w = syn.C2_CONCAT.scaled(B=200)
+    weights = syn.make_weights(w, DEV)
+    idx = torch.from_numpy(syn.make_indices(w)).to(DEV)
+    off = torch.from_numpy(syn.make_offsets(w)).to(DEV)
+    dense = syn.make_dense(w, DEV)
+    a = ops.embbag_sum_multi(weights, idx, off, w.L)
+    b = ops.embbag_pool_multi(weights, idx, off)
+    pa, ia = ops.sparse_interact(weights, idx, off, dense, w.L, concat_dense=True)
+    pb, ib = ops.sparse_interact_pool(weights, idx, off, dense, concat_dense=True)
+    torch.cuda.synchronize()
+    for x, y in ((a, b), (pa, pb), (ia, ib)):
+        assert torch.equal(x.view(torch.int32), y.view(torch.int32))
+
+
+@pytest.mark.parametrize("mode", ["sum", "mean", "max"])
+def test_checked_general_pooling_skips_bad_indices(ops, mode):
+    B, F, N, D, T = 20, 3, 15, 64, 100
+    weights, idx, off, _, dense = _case(31, B, F, N, D, T, torch.float32, False, 0.0)
+    bad = idx.copy()
+    planted = [(0, 3, N), (1, 50, -7), (2, 99, 1 << 30)]
+    for k, t, v in planted:
+        bad[k, t] = v
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = ops.embbag_pool_multi(weights, torch.from_numpy(bad).to(DEV),
+                                torch.from_numpy(off).to(DEV), mode=mode, checked=True,
+                                status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == ops.FLAG_INDEX_OOB
+    # expected: the same bags with the planted entries removed (include_last_offset form)
+    new_idx = np.zeros_like(bad)
+    new_off = np.zeros((F, B + 1), np.int32)
+    for k in range(F):
+        keep = np.ones(T, bool)
+        keep[[t for kk, t, _ in planted if kk == k]] = False
+        cum = np.concatenate([[0], np.cumsum(keep)])
+        new_off[k, :B] = cum[off[k]]
+        new_off[k, B] = cum[T]
+        kept = bad[k][keep]
+        new_idx[k, :kept.size] = kept
+    ref = oracle.embbag_pool_multi([w.cpu().numpy() for w in weights], new_idx, new_off, B,
+                                   mode=mode, include_last_offset=True)
+    assert_bits_equal(out, ref, f"checked {mode}")
+
+
+def test_bf16_full_size_sampled(ops):
+    """The c3 workload with bf16 tables (half the gathered bytes), sampled check."""
+    w = syn.C3_ZIPF
+    torch.cuda.empty_cache()
+    weights = [t.to(torch.bfloat16) for t in syn.make_weights(w, DEV)]
+    torch.cuda.empty_cache()
+    idx = syn.make_indices(w)
+    off = syn.make_offsets(w)
+    dense = syn.make_dense(w, DEV)
+    pooled, inter = ops.sparse_interact_pool(weights, torch.from_numpy(idx).to(DEV),
+                                             torch.from_numpy(off).to(DEV), dense)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(9)
+    samples = np.unique(np.concatenate([[0, w.B - 1], rng.integers(0, w.B, 30)]))
+    tables, sub_idx = [], []
+    for k in range(w.F):
+        rows = np.concatenate([idx[k, s * w.L:(s + 1) * w.L] for s in samples])
+        uniq, inv = np.unique(rows, return_inverse=True)
+        t = weights[k].index_select(0, torch.from_numpy(uniq.astype(np.int64)).to(DEV))
+        tables.append(_host_bits(t))
+        sub_idx.append(inv.astype(np.int32))
+    sub_off = np.broadcast_to((np.arange(len(samples)) * w.L).astype(np.int32),
+                              (w.F, len(samples))).copy()
+    ref = oracle.embbag_pool_multi(tables, np.stack(sub_idx), sub_off, len(samples))
+    sel = torch.from_numpy(samples).to(DEV)
+    assert_bits_equal(pooled[sel], ref, "bf16 c3 pooled (sampled)")
+    ref_i, _, bound = oracle.interact_lower_tri(dense[sel].cpu().numpy(), ref, with_f64=True)
+    assert_dots_close(inter[sel], ref_i, bound, "bf16 c3 dots (sampled)")
+    del weights, pooled, inter
+    torch.cuda.empty_cache()

@@ -32,7 +32,12 @@ MUTANTS = {
     "last_bag_ignores_segment_end": [("(int64_t)offsets[(int64_t)k * B + b + 1] : seg;",
                                       "(int64_t)offsets[(int64_t)k * B + b + 1] : s + L;")],
     "offsets_order_unchecked": [("if (s < 0 || s > e || e > seg)", "if (s < 0 || e > seg)")],
-    "index_bound_off_by_one": [("(int64_t)r >= rows[k]", "(int64_t)r > rows[k]")],
+    "index_bound_off_by_one": [
+        ("int32_t r = indices[(int64_t)k * seg + t];\n            if (r < 0 || (int64_t)r >= rows[k])",
+         "int32_t r = indices[(int64_t)k * seg + t];\n            if (r < 0 || (int64_t)r > rows[k])")],
+    "general_index_bound_off_by_one": [
+        ("int32_t r = indices[(int64_t)k * T + t];\n                if (r < 0 || (int64_t)r >= rows[k])",
+         "int32_t r = indices[(int64_t)k * T + t];\n                if (r < 0 || (int64_t)r > rows[k])")],
     "dot_wrong_operand": [("(double)a[d] * (double)b[d]", "(double)a[d] * (double)a[d]")],
     "dot_drops_first_term": [("for (int d = 0; d < D; ++d) {\n        double t",
                               "for (int d = 1; d < D; ++d) {\n        double t")],
@@ -44,6 +49,19 @@ MUTANTS = {
     "pairs_include_diagonal": [("for (int j = 0; j < i; ++j) {\n                const float* vj",
                                 "for (int j = 0; j <= i; ++j) {\n                const float* vj")],
     "concat_drops_dense": [("row[d] = dense[(int64_t)b * D + d];", "row[d] = 0.0f;")],
+    "bf16_widened_with_wrong_shift": [("((uint32_t)h) << 16", "((uint32_t)h) << 15")],
+    "weighted_sum_drops_weight": [("acc = fmaf(wk[t], x, acc);", "acc = acc + x;")],
+    "weighted_sum_uses_first_weight": [("acc = fmaf(wk[t], x, acc);",
+                                        "acc = fmaf(wk[s], x, acc);")],
+    "mean_divides_by_count_plus_one": [("acc = acc / (float)(e - s);",
+                                        "acc = acc / (float)(e - s + 1);")],
+    "max_keeps_the_minimum": [("((x > acc) ? x : acc)", "((x < acc) ? x : acc)")],
+    "max_starts_from_zero": [("acc = (t == s) ? x : ((x > acc) ? x : acc);",
+                              "acc = (x > acc) ? x : acc;")],
+    "last_offset_ignored": [("(ilo || b + 1 < B) ? (int64_t)offsets[(int64_t)k * row + b + 1]",
+                             "(b + 1 < B) ? (int64_t)offsets[(int64_t)k * row + b + 1]")],
+    "general_pooling_table_layout_transposed": [
+        ("out[((int64_t)b * F + k) * D + d] = acc;", "out[((int64_t)k * B + b) * D + d] = acc;")],
 }
 
 _RUNNER = (
