@@ -34,6 +34,7 @@ from dlrm_embedding_bag_b200 import synthetic as syn  # noqa: E402
 PROFILES = os.path.join(ROOT, "profiles")
 CSRC = os.path.join(ROOT, "dlrm_embedding_bag_b200", "csrc")
 FALLBACK_HBM_GBS = 6650.0
+E2E_BATCHES = 4
 METRIC = "pooled lookups/s (fused EmbeddingBag-sum + lower-triangle interaction)"
 
 
@@ -381,35 +382,51 @@ def run_ours(args, w: syn.Workload):
     value = lookups / (total_ms / 1e3)
     ms_step = total_ms / args.steps
 
-    # e2e through the host-buffer entry point: inputs copied in, result copied out, every step
+    # e2e through the host-buffer entry point: every step copies its batch's
+    # indices, offsets and dense rows in from pinned host memory and its
+    # interaction rows back out. Steps cycle over E2E_BATCHES distinct batches
+    # (tables 8 GB > L2) on a double-buffered two-stream pipeline, so one
+    # batch's copies overlap another's kernel; the region is timed with events.
     e2e = None
     if not args.no_e2e:
-        stage = ops.HostStage(weights, w.B, w.L, concat_dense=w.concat_dense, want_pooled=True)
-        ih = torch.from_numpy(idx_np.reshape(-1)).pin_memory()
-        oh = torch.from_numpy(off_np).pin_memory()
-        dh = dense.cpu().pin_memory()
-        xh = torch.empty(tuple(inter.shape), dtype=torch.float32).pin_memory()
-        for _ in range(args.warmup):
-            stage(ih, oh, dh, xh)
+        pipe = ops.HostPipeline(weights, w.B, w.L, concat_dense=w.concat_dense, want_pooled=True,
+                                depth=2)
+        batches = []
+        for j in range(E2E_BATCHES):
+            ij = syn.make_indices(w, replica=rank * E2E_BATCHES + j) if j else idx_np
+            batches.append((torch.from_numpy(ij.reshape(-1)).pin_memory(),
+                            torch.from_numpy(off_np).pin_memory(), dense.cpu().pin_memory()))
+        outs = [torch.empty(tuple(inter.shape), dtype=torch.float32).pin_memory()
+                for _ in range(2)]
+        for i in range(args.warmup):
+            pipe.submit(*batches[i % E2E_BATCHES], outs[i % 2])
+        pipe.drain()
         barrier()
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        cur = torch.cuda.current_stream()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(cur)
+        for _, st, _ in pipe.slots:
+            st.wait_event(t0)
         for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            starts[i].record()
-            stage(ih, oh, dh, xh)
-            ends[i].record()
+            pipe.submit(*batches[i % E2E_BATCHES], outs[i % 2])
+        for _, st, _ in pipe.slots:
+            ev = torch.cuda.Event()
+            ev.record(st)
+            cur.wait_event(ev)
+        t1.record(cur)
         barrier()
-        e2e_ms = float(sum(s.elapsed_time(e) for s, e in zip(starts, ends)))
+        e2e_ms = t0.elapsed_time(t1)
         if world > 1:
             t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e2e_ms = float(t.item())
         e2e = {"value": lookups / (e2e_ms / 1e3), "unit": "lookups/s",
-               "h2d_bytes_per_step": stage.h2d_bytes(), "d2h_bytes_per_step": stage.d2h_bytes(),
+               "h2d_bytes_per_step": pipe.h2d_bytes(), "d2h_bytes_per_step": pipe.d2h_bytes(),
                "ms_per_step": e2e_ms / args.steps,
-               "path": "dlrm_sparse_interact_host: pinned indices/offsets/dense in, "
-                       "interaction rows out; pooled written to device staging"}
+               "path": f"dlrm_sparse_interact_host via ops.HostPipeline (2 streams): pinned "
+                       f"indices/offsets/dense in, interaction rows out, {E2E_BATCHES} distinct "
+                       f"batches in rotation; pooled written to device staging"}
 
     if rank == 0:
         peaks = measured_peaks()

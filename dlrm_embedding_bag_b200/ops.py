@@ -410,6 +410,51 @@ class HostStage:
         _check(rc, "dlrm_sparse_interact_host")
 
 
+class HostPipeline:
+    """Batches from host memory, overlapped across ``depth`` CUDA streams.
+
+    Each slot owns a :class:`HostStage` (its own device staging buffers) and a
+    stream; batch i goes to slot ``i % depth``, so the host-to-device copies of
+    one batch run while another batch's kernel and device-to-host copy run.
+    :meth:`submit` returns the slot's completion event; the host outputs of a
+    batch are valid once its event has completed (:meth:`wait`). A slot is
+    reused only after its previous batch completed, so outputs are never
+    overwritten while in flight.
+    """
+
+    def __init__(self, weights: Sequence[torch.Tensor], B: int, L: int, *,
+                 concat_dense: bool = False, want_pooled: bool = False, depth: int = 2):
+        dev = weights[0].device
+        self.slots = []
+        for _ in range(depth):
+            stage = HostStage(weights, B, L, concat_dense=concat_dense, want_pooled=want_pooled)
+            self.slots.append((stage, torch.cuda.Stream(device=dev), torch.cuda.Event()))
+        self.n = 0
+
+    def h2d_bytes(self) -> int:
+        return self.slots[0][0].h2d_bytes()
+
+    def d2h_bytes(self) -> int:
+        return self.slots[0][0].d2h_bytes()
+
+    def submit(self, indices_host, offsets_host, dense_host, inter_host, pooled_host=None):
+        stage, stream, done = self.slots[self.n % len(self.slots)]
+        self.n += 1
+        done.synchronize()  # the slot's previous batch (and its host outputs) is finished
+        with torch.cuda.stream(stream):
+            stage(indices_host, offsets_host, dense_host, inter_host, pooled_host)
+            done.record(stream)
+        return done
+
+    @staticmethod
+    def wait(event: "torch.cuda.Event"):
+        event.synchronize()
+
+    def drain(self):
+        for _, stream, _ in self.slots:
+            stream.synchronize()
+
+
 def pair_decode(p0: int, count: int, device="cuda"):
     """``(i, j)`` int32 tensors from the kernels' closed-form pair decoder."""
     i = torch.empty(count, dtype=torch.int32, device=device)

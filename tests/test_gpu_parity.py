@@ -400,6 +400,26 @@ def test_nondefault_stream_ordering(ops):
     check_inter(fi, ref_i, bound, w.D, False, "side stream")
 
 
+def test_host_pipeline_overlapped_batches(ops):
+    w = syn.C2_CONCAT.scaled(B=257)
+    weights = syn.make_weights(w, DEV)
+    dense = syn.make_dense(w, DEV)
+    off = syn.make_offsets(w)
+    pipe = ops.HostPipeline(weights, w.B, w.L, concat_dense=True, depth=2)
+    batches = [syn.make_indices(w, replica=r) for r in range(5)]
+    outs = [torch.empty((w.B, w.D + w.P)).pin_memory() for _ in range(5)]
+    events = [pipe.submit(torch.from_numpy(b.reshape(-1)).pin_memory(),
+                          torch.from_numpy(off).pin_memory(), dense.cpu().pin_memory(), o)
+              for b, o in zip(batches, outs)]
+    for ev, b, o in zip(events, batches, outs):
+        pipe.wait(ev)
+        _, ref = ops.sparse_interact(weights, _dev_i32(b), _dev_i32(off), dense, w.L,
+                                     concat_dense=True)
+        torch.cuda.synchronize()
+        assert torch.equal(o.view(torch.int32), ref.cpu().view(torch.int32))
+    pipe.drain()
+
+
 def test_prepared_call_matches_plain_call(ops):
     w = syn.C2_CONCAT.scaled(B=333)
     weights, idx, off, dense = _inputs(w)
