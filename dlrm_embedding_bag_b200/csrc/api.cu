@@ -105,6 +105,40 @@ int clear_status(int32_t* status_dev, cudaStream_t stream) {
   return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
 }
 
+// The TMA path needs whole 16-byte row chunks of 64..512 bytes, 16-byte
+// aligned tables, tensor maps for every table and at least one row per table.
+bool tma_eligible(const Prepared& pr, const int64_t* rows, int F, int D) {
+  const int row_bytes = D * pr.elem_size;
+  if (row_bytes % 16 != 0 || row_bytes < 64 || row_bytes > 512) return false;
+  if (!pr.tables_aligned16 || F > dlrm::kTmaMaxTables) return false;
+  if (rows != nullptr)
+    for (int k = 0; k < F; ++k)
+      if (rows[k] < 1) return false;
+  return true;
+}
+
+dlrm::GatherPlan make_plan(const Prepared& pr, const int64_t* rows, int B, int F, int D,
+                           int loader, bool tma_ok) {
+  dlrm::GatherPlan g;
+  g.tp = &pr.tp;
+  g.bp = pr.bp;
+  g.B = B;
+  g.F = F;
+  g.D = D;
+  g.pool = pr.pool;
+  g.loader = loader;
+  g.esz = pr.elem_size;
+  g.tma_ok = tma_ok;
+  g.rows = rows;
+  return g;
+}
+
+int launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return DLRM_OK;
+  if (e == cudaErrorNotSupported) return DLRM_ERR_UNSUPPORTED;
+  return cuda_fail(e);
+}
+
 int pool_impl(const void* const* weights, int dtype, const int64_t* rows, const dlrm_bags_t* bags,
               int B, int F, int D, float* out, int32_t* status_dev, cudaStream_t stream) {
   Prepared pr;
@@ -112,10 +146,12 @@ int pool_impl(const void* const* weights, int dtype, const int64_t* rows, const 
   if (rc != DLRM_OK) return rc;
   if (out == nullptr) return DLRM_ERR_NULL;
   if (!aligned(out, 4)) return DLRM_ERR_ALIGN;
-  const int loader = pick_loader(dtype, D, pr.tables_aligned16 && aligned(out, 16));
+  const bool out16 = aligned(out, 16);
+  const int loader = pick_loader(dtype, D, pr.tables_aligned16 && out16);
+  const dlrm::GatherPlan g =
+      make_plan(pr, rows, B, F, D, loader, out16 && tma_eligible(pr, rows, F, D));
   if ((rc = clear_status(status_dev, stream)) != DLRM_OK) return rc;
-  cudaError_t e = dlrm::launch_embbag(pr.tp, pr.bp, B, F, D, out, pr.pool, loader, stream);
-  return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
+  return launch_status(dlrm::launch_embbag(g, out, stream));
 }
 
 int fused_impl(const void* const* weights, int dtype, const int64_t* rows,
@@ -132,12 +168,13 @@ int fused_impl(const void* const* weights, int dtype, const int64_t* rows,
   const int64_t limit = smem_limit_current_device(&err);
   if (err != DLRM_OK) return err;
   if (dlrm::interact_smem_per_sample(F, D) > limit) return DLRM_ERR_SHAPE;
-  const bool vec_ok = pr.tables_aligned16 && (pooled_out == nullptr || aligned(pooled_out, 16));
-  const int loader = pick_loader(dtype, D, vec_ok);
+  const bool pooled16 = pooled_out == nullptr || aligned(pooled_out, 16);
+  const int loader = pick_loader(dtype, D, pr.tables_aligned16 && pooled16);
+  const dlrm::GatherPlan g =
+      make_plan(pr, rows, B, F, D, loader, pooled16 && tma_eligible(pr, rows, F, D));
   if ((rc = clear_status(status_dev, stream)) != DLRM_OK) return rc;
-  cudaError_t e = dlrm::launch_fused(pr.tp, pr.bp, dense, B, F, D, pooled_out, inter_out,
-                                     concat_dense ? 1 : 0, pr.pool, loader, limit, stream);
-  return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
+  return launch_status(dlrm::launch_fused(g, dense, pooled_out, inter_out, concat_dense ? 1 : 0,
+                                          limit, stream));
 }
 
 // The fixed-stride, unweighted-sum, f32 case of the general entry points.
@@ -296,7 +333,16 @@ int dlrm_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_t* j_out,
   return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
 }
 
+int dlrm_set_gather_path(int path) {
+  if (path != DLRM_PATH_AUTO && path != DLRM_PATH_LDG && path != DLRM_PATH_TMA)
+    return DLRM_ERR_ARG;
+  const int prev = dlrm::gather_path();
+  dlrm::set_gather_path(path);
+  return prev;
+}
+
 int dlrm_status_from_flags(int32_t flags) {
+  if (flags & DLRM_FLAG_TIMEOUT) return DLRM_ERR_TIMEOUT;
   if (flags & DLRM_FLAG_INDEX_OOB) return DLRM_ERR_INDEX_OOB;
   if (flags & DLRM_FLAG_OFFSETS) return DLRM_ERR_OFFSETS;
   return DLRM_OK;
@@ -313,6 +359,8 @@ const char* dlrm_status_string(int status) {
     case DLRM_ERR_OFFSETS: return "offsets describe a bag with start > end or outside [0, T]";
     case DLRM_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case DLRM_ERR_ARG: return "invalid argument";
+    case DLRM_ERR_TIMEOUT: return "a bounded wait on an asynchronous copy ran out";
+    case DLRM_ERR_UNSUPPORTED: return "the requested gather path cannot serve this call";
     default: return "unknown status";
   }
 }

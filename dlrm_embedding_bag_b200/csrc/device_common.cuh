@@ -148,7 +148,10 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
                                         int nmax, int D, int col0, int q, int gbase,
                                         float (&acc)[CPL][LD::VEC], bool& oob) {
   constexpr int VEC = LD::VEC;
-  constexpr int IPL = (U + G - 1) / G;  // row ids held per lane per batch of U rows
+  // Row ids are fetched NB at a time (one coalesced load per lane), rows U at
+  // a time out of those, so a bag of up to NB rows costs one id round trip.
+  constexpr int NB = U > G ? U : G;
+  constexpr int IPL = NB / G;  // row ids held per lane
 #pragma unroll
   for (int m = 0; m < CPL; ++m)
 #pragma unroll
@@ -158,53 +161,59 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
   for (int m = 0; m < CPL; ++m) colok[m] = col0 + (q + G * m) * VEC < D;
   int used = 0;
 
-  for (int c = 0; c < nmax; c += U) {
+  for (int c = 0; c < nmax; c += NB) {
     int my_row[IPL];
     float my_w[IPL];
 #pragma unroll
     for (int j = 0; j < IPL; ++j) {
-      const int slot = q + G * j;
-      const bool in = (slot < U) && (c + slot < n);
-      my_row[j] = in ? __ldg(idx_seg + start + c + slot) : 0;
-      if (POOL == kPoolWeighted) my_w[j] = in ? __ldg(w_seg + start + c + slot) : 0.f;
-    }
-    typename LD::Raw v[U][CPL];
-    bool use[U];
-    float wt[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int r = __shfl_sync(kFullMask, my_row[u / G], gbase + (u % G));
-      if (POOL == kPoolWeighted) wt[u] = __shfl_sync(kFullMask, my_w[u / G], gbase + (u % G));
-      bool ok = (c + u) < n;
-      if (check) {
-        const bool in_range = static_cast<unsigned>(r) < static_cast<unsigned>(rows_k);
-        oob |= ok && !in_range;
-        ok = ok && in_range;
-      }
-      use[u] = ok;
-      const typename LD::Elem* row = W + static_cast<int64_t>(r) * D + col0 + q * VEC;
-#pragma unroll
-      for (int m = 0; m < CPL; ++m) {
-        if (ok && colok[m]) v[u][m] = LD::load(row + G * m * VEC);
-      }
+      const int t = c + q + G * j;
+      const bool in = t < n;
+      my_row[j] = in ? __ldg(idx_seg + start + t) : 0;
+      if (POOL == kPoolWeighted) my_w[j] = in ? __ldg(w_seg + start + t) : 0.f;
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (use[u]) {
+    for (int cu = 0; cu < NB; cu += U) {
+      if (c + cu >= nmax) break;  // warp-uniform
+      typename LD::Raw v[U][CPL];
+      bool use[U];
+      float wt[U];
 #pragma unroll
-        for (int m = 0; m < CPL; ++m)
+      for (int u = 0; u < U; ++u) {
+        const int slot = cu + u;
+        const int r = __shfl_sync(kFullMask, my_row[slot / G], gbase + (slot % G));
+        if (POOL == kPoolWeighted)
+          wt[u] = __shfl_sync(kFullMask, my_w[slot / G], gbase + (slot % G));
+        bool ok = (c + slot) < n;
+        if (check) {
+          const bool in_range = static_cast<unsigned>(r) < static_cast<unsigned>(rows_k);
+          oob |= ok && !in_range;
+          ok = ok && in_range;
+        }
+        use[u] = ok;
+        const typename LD::Elem* row = W + static_cast<int64_t>(r) * D + col0 + q * VEC;
 #pragma unroll
-          for (int e = 0; e < VEC; ++e) {
-            const float x = LD::get(v[u][m], e);
-            if (POOL == kPoolSum) {
-              acc[m][e] = __fadd_rn(acc[m][e], x);
-            } else if (POOL == kPoolWeighted) {
-              acc[m][e] = __fmaf_rn(wt[u], x, acc[m][e]);
-            } else {
-              acc[m][e] = (used == 0) ? x : ((x > acc[m][e]) ? x : acc[m][e]);
+        for (int m = 0; m < CPL; ++m) {
+          if (ok && colok[m]) v[u][m] = LD::load(row + G * m * VEC);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (use[u]) {
+#pragma unroll
+          for (int m = 0; m < CPL; ++m)
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+              const float x = LD::get(v[u][m], e);
+              if (POOL == kPoolSum) {
+                acc[m][e] = __fadd_rn(acc[m][e], x);
+              } else if (POOL == kPoolWeighted) {
+                acc[m][e] = __fmaf_rn(wt[u], x, acc[m][e]);
+              } else {
+                acc[m][e] = (used == 0) ? x : ((x > acc[m][e]) ? x : acc[m][e]);
+              }
             }
-          }
-        ++used;
+          ++used;
+        }
       }
     }
   }

@@ -36,10 +36,12 @@ struct FeatLayout {
 // [D, 4*D4) of the feature rows, and the filler rows [F1, F1p). (The filler
 // rows only feed tile entries that are never stored; they are zeroed so that
 // nothing reads uninitialised memory.)
+//
+// Run by the `nthreads` threads tid = 0 .. nthreads-1 (a multiple of 32).
 __device__ __forceinline__ void zero_feature_padding(float* feat, const FeatLayout& Lf, int D,
-                                                     int S_here) {
+                                                     int S_here, int tid, int nthreads) {
   const int padc = 4 * Lf.D4 - D;  // 0..3
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  const int warp = tid >> 5, lane = tid & 31, nwarps = nthreads >> 5;
   for (int s = 0; s < S_here; ++s) {
     float* base = feat + static_cast<int64_t>(s) * Lf.F1p * Lf.Dp;
     if (padc > 0) {
@@ -47,7 +49,7 @@ __device__ __forceinline__ void zero_feature_padding(float* feat, const FeatLayo
         if (lane < padc) base[f * Lf.Dp + D + lane] = 0.f;
     }
     const int n_extra = (Lf.F1p - Lf.F1) * Lf.Dp;
-    for (int e = threadIdx.x; e < n_extra; e += blockDim.x) base[Lf.F1 * Lf.Dp + e] = 0.f;
+    for (int e = tid; e < n_extra; e += nthreads) base[Lf.F1 * Lf.Dp + e] = 0.f;
   }
 }
 
@@ -64,14 +66,16 @@ __device__ __forceinline__ void zero_feature_padding(float* feat, const FeatLayo
 // F+1.
 //
 // The output row of sample b starts at out + b * row_stride + col0; dot p of
-// the row is written at offset p.
+// the row is written at offset p. Run by the `nthreads` threads tid = 0 ..
+// nthreads-1 (a multiple of 32, whole warps).
 __device__ __forceinline__ void dots_from_smem(const float* feat, const FeatLayout& Lf,
                                                int S_here, int lq, float* __restrict__ out,
-                                               int64_t b0, int64_t row_stride, int64_t col0) {
+                                               int64_t b0, int64_t row_stride, int64_t col0,
+                                               int tid, int nthreads) {
   const int Q = 1 << lq;
   const int total = (S_here * Lf.nT) << lq;
-  const int lane = threadIdx.x & 31;
-  for (int base = threadIdx.x - lane; base < total; base += blockDim.x) {
+  const int lane = tid & 31;
+  for (int base = tid - lane; base < total; base += nthreads) {
     const int task = base + lane;
     const bool active = task < total;
     const int tt = active ? task : 0;

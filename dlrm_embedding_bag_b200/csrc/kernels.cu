@@ -10,6 +10,7 @@
 
 #include "interact_common.cuh"
 #include "launch.h"
+#include "tma_kernels.cuh"
 
 namespace dlrm {
 
@@ -42,10 +43,10 @@ __global__ void __launch_bounds__(kBlockThreads)
       }
     }
   }
-  zero_feature_padding(feat, Lf, D, S_here);
+  zero_feature_padding(feat, Lf, D, S_here, threadIdx.x, blockDim.x);
   __syncthreads();
   const int P = Lf.F1 * (Lf.F1 - 1) / 2;
-  dots_from_smem(feat, Lf, S_here, lq, out, b0, P, 0);
+  dots_from_smem(feat, Lf, S_here, lq, out, b0, P, 0, threadIdx.x, blockDim.x);
 }
 
 __global__ void pair_decode_kernel(int64_t p0, int64_t count, int32_t* __restrict__ i_out,
@@ -115,10 +116,93 @@ static cudaError_t counted(cudaError_t e) {
   return e;
 }
 
-cudaError_t launch_embbag(const TableParams& tp, const BagParams& bp, int B, int F, int D,
-                          float* out, int pool, int loader, cudaStream_t stream) {
-  GatherLaunch a{&tp, bp, B, F, D, out, pool, choose_gather_shape(D, loader), stream};
-  switch (loader) {
+// --------------------------------------------------------------------------
+// Path choice and the TMA path's tensor maps.
+
+static std::atomic<int> g_path{DLRM_PATH_AUTO};
+int gather_path() { return g_path.load(std::memory_order_relaxed); }
+void set_gather_path(int path) { g_path.store(path, std::memory_order_relaxed); }
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime.
+static EncodeTiledFn encode_tiled() {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// One map per table: a 2-D tensor {D, rows} with row pitch D*esz, box {D, 1},
+// out-of-range rows read as zeros.
+static cudaError_t make_tma_params(const GatherPlan& g, TmaParams* tp) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  const int row_bytes = g.D * g.esz;
+  const CUtensorMapL2promotion promo = row_bytes >= 256   ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+                                       : row_bytes >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                                          : CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
+  for (int k = 0; k < g.F; ++k) {
+    const int64_t rows = g.rows ? g.rows[k] : INT32_MAX;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(g.D), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(g.D), 1};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r =
+        enc(&tp->map[k], g.esz == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+            2, const_cast<void*>(g.tp->w[k]), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, promo,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    tp->rows[k] = g.tp->rows[k];
+  }
+  return cudaSuccess;
+}
+
+static int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n;
+}
+
+static int tma_lanes(const GatherPlan& g) {
+  return std::min(32, std::max(4, pow2_ceil(g.D * g.esz / 16)));
+}
+
+cudaError_t launch_embbag(const GatherPlan& g, float* out, cudaStream_t stream) {
+  const int path = gather_path();
+  if (path == DLRM_PATH_TMA && !g.tma_ok) return cudaErrorNotSupported;
+  if (g.tma_ok && path != DLRM_PATH_LDG) {
+    TmaParams tp;
+    cudaError_t e = make_tma_params(g, &tp);
+    if (e != cudaSuccess) return e;
+    TmaLaunch a{};
+    a.tp = &tp;
+    a.bp = g.bp;
+    a.B = g.B;
+    a.F = g.F;
+    a.D = g.D;
+    a.G = tma_lanes(g);
+    a.pool = g.pool;
+    a.out = out;
+    a.sms = sm_count();
+    a.stream = stream;
+    return counted(g.esz == 4 ? launch_tma_gather_f32(a) : launch_tma_gather_bf16(a));
+  }
+  GatherLaunch a{g.tp, g.bp, g.B, g.F, g.D, out, g.pool, choose_gather_shape(g.D, g.loader),
+                 stream};
+  switch (g.loader) {
     case kLdF32x4: return counted(launch_gather_f32x4(a));
     case kLdF32x1: return counted(launch_gather_f32x1(a));
     case kLdBF16x8: return counted(launch_gather_bf16x8(a));
@@ -127,23 +211,60 @@ cudaError_t launch_embbag(const TableParams& tp, const BagParams& bp, int B, int
   }
 }
 
-cudaError_t launch_fused(const TableParams& tp, const BagParams& bp, const float* dense, int B,
-                         int F, int D, float* pooled_out, float* inter_out, int concat_dense,
-                         int pool, int loader, int64_t smem_limit, cudaStream_t stream) {
+cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_out,
+                         float* inter_out, int concat_dense, int64_t smem_limit,
+                         cudaStream_t stream) {
+  const int path = gather_path();
+  const FeatLayout Lf = FeatLayout::make(g.F, g.D);
+  bool tma_ok = g.tma_ok && (reinterpret_cast<uintptr_t>(dense) % 16 == 0);
+  TmaLaunch t{};
+  if (tma_ok) {
+    t.G = tma_lanes(g);
+    const int units = kTmaGatherWarps * (32 / t.G);
+    // about two bags per unit per tile; the dot warps take (S * nT) << lq tasks
+    t.S = std::max(1, std::min(16, (2 * units + g.F - 1) / g.F));
+    t.S = std::min(t.S, g.B);
+    const int64_t per = Lf.floats_per_sample() * 4;
+    while (t.S > 1 && TmaSmem::make(t.G, g.D * g.esz, 2 * t.S * per).total > smem_limit) --t.S;
+    tma_ok = TmaSmem::make(t.G, g.D * g.esz, 2 * t.S * per).total <= smem_limit;
+    const int qmax = std::max(1, kTmaDotWarps * 32 / (t.S * Lf.nT));
+    t.lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), 5});
+  }
+  if (path == DLRM_PATH_TMA && !tma_ok) return cudaErrorNotSupported;
+  if (tma_ok && path != DLRM_PATH_LDG) {
+    TmaParams tp;
+    cudaError_t e = make_tma_params(g, &tp);
+    if (e != cudaSuccess) return e;
+    t.tp = &tp;
+    t.bp = g.bp;
+    t.B = g.B;
+    t.F = g.F;
+    t.D = g.D;
+    t.pool = g.pool;
+    t.dense = dense;
+    t.pooled_out = pooled_out;
+    t.inter_out = inter_out;
+    t.concat_dense = concat_dense;
+    t.smem_limit = smem_limit;
+    t.sms = sm_count();
+    t.stream = stream;
+    return counted(g.esz == 4 ? launch_tma_fused_f32(t) : launch_tma_fused_bf16(t));
+  }
   FusedLaunch a;
-  a.g = GatherLaunch{&tp, bp, B, F, D, nullptr, pool, choose_gather_shape(D, loader), stream};
+  a.g = GatherLaunch{g.tp, g.bp, g.B, g.F, g.D, nullptr, g.pool,
+                     choose_gather_shape(g.D, g.loader), stream};
   a.dense = dense;
   a.pooled_out = pooled_out;
   a.inter_out = inter_out;
   a.concat_dense = concat_dense;
   // enough samples that every lane group has a bag in the gather phase
   const int groups = kBlockThreads / a.g.shape.G;
-  const int want = std::max(1, (groups + F - 1) / F);
-  choose_dot_shape(F, D, B, std::min(want, 16), std::min<int64_t>(smem_limit, 64 * 1024), a.S,
-                   a.lq);
-  a.smem = a.S * interact_smem_per_sample(F, D);
+  const int want = std::max(1, (groups + g.F - 1) / g.F);
+  choose_dot_shape(g.F, g.D, g.B, std::min(want, 16), std::min<int64_t>(smem_limit, 64 * 1024),
+                   a.S, a.lq);
+  a.smem = a.S * interact_smem_per_sample(g.F, g.D);
   if (a.smem > smem_limit) return cudaErrorInvalidValue;
-  switch (loader) {
+  switch (g.loader) {
     case kLdF32x4: return counted(launch_fused_f32x4(a));
     case kLdF32x1: return counted(launch_fused_f32x1(a));
     case kLdBF16x8: return counted(launch_fused_bf16x8(a));

@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kBlockThreads, kFusedMinBlocks)
       for (int c = threadIdx.x; c < D; c += blockDim.x) dst[c] = __ldg(src + c);
     }
   }
-  zero_feature_padding(feat, Lf, D, S_here);
+  zero_feature_padding(feat, Lf, D, S_here, threadIdx.x, blockDim.x);
 
   // bags (s, k) -> feature row k + 1; every group runs the same number of rounds
   bool oob = false, bad_any = false;
@@ -169,7 +169,8 @@ __global__ void __launch_bounds__(kBlockThreads, kFusedMinBlocks)
       for (int d = threadIdx.x; d < D; d += blockDim.x) dst[d] = src[d];
     }
   }
-  dots_from_smem(feat, Lf, S_here, lq, inter_out, b0, row_stride, concat_dense ? D : 0);
+  dots_from_smem(feat, Lf, S_here, lq, inter_out, b0, row_stride, concat_dense ? D : 0,
+                 threadIdx.x, blockDim.x);
 }
 
 // --------------------------------------------------------------------------

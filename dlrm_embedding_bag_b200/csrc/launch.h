@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "device_common.cuh"
@@ -38,6 +39,37 @@ struct FusedLaunch {
   int64_t smem;
 };
 
+// Tensor maps of the TMA gather path: one 2-D map per table ({D, rows},
+// box {D, 1}), passed by value in the kernel's parameter block.
+constexpr int kTmaMaxTables = 64;
+struct alignas(64) TmaParams {
+  CUtensorMap map[kTmaMaxTables];
+  int32_t rows[kTmaMaxTables];
+};
+
+struct TmaLaunch {
+  const TmaParams* tp;
+  BagParams bp;
+  int B, F, D;
+  int G;     // lanes per bag: pow2ceil(row bytes / 16), 4..32
+  int pool;  // PoolKind
+  float* out;  // gather-only output
+  // fused
+  const float* dense;
+  float* pooled_out;
+  float* inter_out;
+  int concat_dense;
+  int S, lq;
+  int64_t smem_limit;
+  int sms;
+  cudaStream_t stream;
+};
+
+cudaError_t launch_tma_gather_f32(const TmaLaunch& a);
+cudaError_t launch_tma_gather_bf16(const TmaLaunch& a);
+cudaError_t launch_tma_fused_f32(const TmaLaunch& a);
+cudaError_t launch_tma_fused_bf16(const TmaLaunch& a);
+
 // One pair of launchers per loader (inst_*.cu).
 cudaError_t launch_gather_f32x4(const GatherLaunch& a);
 cudaError_t launch_gather_f32x1(const GatherLaunch& a);
@@ -51,13 +83,28 @@ cudaError_t launch_fused_bf16x1(const FusedLaunch& a);
 // Shared-memory bytes that one sample's features take in the dot phase.
 int64_t interact_smem_per_sample(int F, int D);
 
-// Picks the shape and launches; `loader` from the table dtype and alignment.
-cudaError_t launch_embbag(const TableParams& tp, const BagParams& bp, int B, int F, int D,
-                          float* out, int pool, int loader, cudaStream_t stream);
+// Everything a gather launch needs besides its outputs.
+struct GatherPlan {
+  const TableParams* tp;
+  BagParams bp;
+  int B, F, D;
+  int pool;             // PoolKind
+  int loader;           // LoaderKind of the register (LDG) path
+  int esz;              // table element bytes (4 or 2)
+  bool tma_ok;          // tables and shape qualify for the TMA gather path
+  const int64_t* rows;  // host row counts, or null (then the maps span INT32_MAX rows)
+};
 
-cudaError_t launch_fused(const TableParams& tp, const BagParams& bp, const float* dense, int B,
-                         int F, int D, float* pooled_out, float* inter_out, int concat_dense,
-                         int pool, int loader, int64_t smem_limit, cudaStream_t stream);
+// Process-wide choice of gather path (dlrm_set_gather_path).
+int gather_path();
+void set_gather_path(int path);
+
+// Picks the path and shape, then launches.
+cudaError_t launch_embbag(const GatherPlan& g, float* out, cudaStream_t stream);
+
+cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_out,
+                         float* inter_out, int concat_dense, int64_t smem_limit,
+                         cudaStream_t stream);
 
 cudaError_t launch_interact(const float* dense, const float* emb, int B, int F, int D, float* out,
                             bool vec_ok, int64_t smem_limit, cudaStream_t stream);

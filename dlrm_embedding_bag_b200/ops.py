@@ -28,9 +28,13 @@ STATUS = {
     -6: "DLRM_ERR_OFFSETS",
     -7: "DLRM_ERR_CUDA",
     -8: "DLRM_ERR_ARG",
+    -9: "DLRM_ERR_TIMEOUT",
+    -10: "DLRM_ERR_UNSUPPORTED",
 }
+GATHER_PATHS = {"auto": 0, "ldg": 1, "tma": 2}
 FLAG_INDEX_OOB = 1
 FLAG_OFFSETS = 2
+FLAG_TIMEOUT = 4
 
 # Every symbol the header declares, with its ctypes signature.
 _P = ctypes.c_void_p
@@ -47,6 +51,7 @@ SIGNATURES = {
     "embbag_pool_multi": (_I, [_P, _I, _P, _P, _I, _I, _I, _P, _P, _P]),
     "dlrm_sparse_interact_pool": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _I, _P, _P]),
     "dlrm_pair_decode": (_I, [_I64, _I64, _P, _P, _P]),
+    "dlrm_set_gather_path": (_I, [_I]),
     "dlrm_status_from_flags": (_I, [ctypes.c_int32]),
     "dlrm_status_string": (ctypes.c_char_p, [_I]),
     "dlrm_last_cuda_error": (_I, []),
@@ -463,6 +468,14 @@ def pair_decode(p0: int, count: int, device="cuda"):
                                  j.data_ptr() if count else None, _stream()),
            "dlrm_pair_decode")
     return i, j
+
+
+def set_gather_path(path: str) -> str:
+    """Choose the gather path for later calls ("auto", "ldg" or "tma"); returns the old one."""
+    prev = _lib.dlrm_set_gather_path(GATHER_PATHS[path])
+    if prev < 0:
+        raise DlrmError(prev, "dlrm_set_gather_path")
+    return {v: k for k, v in GATHER_PATHS.items()}[prev]
 
 
 def status_from_flags(flags: int) -> int:

@@ -75,12 +75,22 @@ typedef enum {
                                       or end > B*L */
     DLRM_ERR_CUDA = -7,            /* a CUDA runtime call or launch failed; see
                                       dlrm_last_cuda_error() */
-    DLRM_ERR_ARG = -8              /* any other invalid argument (e.g. count < 0) */
+    DLRM_ERR_ARG = -8,             /* any other invalid argument (e.g. count < 0) */
+    DLRM_ERR_TIMEOUT = -9,         /* (device flag) a bounded wait on an asynchronous
+                                      copy ran out; the results are not valid */
+    DLRM_ERR_UNSUPPORTED = -10     /* the requested gather path cannot serve this call */
 } dlrm_status_t;
 
 /* Bits that the checked (_ex) entry points OR into *status_dev. */
 #define DLRM_FLAG_INDEX_OOB 1
 #define DLRM_FLAG_OFFSETS 2
+#define DLRM_FLAG_TIMEOUT 4
+
+/* Gather paths (dlrm_set_gather_path). */
+#define DLRM_PATH_AUTO 0 /* TMA gather when the call qualifies, else register loads */
+#define DLRM_PATH_LDG 1  /* always the register-load (128-bit ld.global.nc) gather */
+#define DLRM_PATH_TMA 2  /* always the TMA tile::gather4 gather; DLRM_ERR_UNSUPPORTED
+                            for calls it cannot serve */
 
 /* Pooling of a bag's rows (torch.nn.EmbeddingBag modes). The pages implement
  * only SUM and name the others as what a later model would need (movement.rs,
@@ -253,6 +263,23 @@ DLRM_API int dlrm_sparse_interact_host(const float* const* weights, const int32_
  */
 DLRM_API int dlrm_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_t* j_out,
                      dlrm_stream_t stream);
+
+/*
+ * dlrm_set_gather_path -- which gather serves later gather and fused calls of
+ * this process (all threads): DLRM_PATH_AUTO (default), DLRM_PATH_LDG or
+ * DLRM_PATH_TMA. Returns the previous setting, or DLRM_ERR_ARG for an unknown
+ * value. Both paths give bit-identical pooled results; the choice exists for
+ * testing and tuning.
+ *
+ * The TMA path serves a call when each table row is 64..512 bytes and a
+ * multiple of 16 bytes (f32: D in 16..128, D % 4 == 0; bf16: D in 32..256,
+ * D % 8 == 0), every table, the pooled output and the dense rows are 16-byte
+ * aligned, F <= 64, and (fused) two tiles of features fit in shared memory.
+ * It builds one tensor map per table on the host for every call. When row
+ * counts are given (the calls that take `rows`), an index outside its table
+ * reads zeros on this path instead of other memory.
+ */
+DLRM_API int dlrm_set_gather_path(int path);
 
 /* Status of a *status_dev value written by an _ex call (DLRM_OK if 0). */
 DLRM_API int dlrm_status_from_flags(int32_t flags);

@@ -32,7 +32,7 @@ def ops():
 def test_header_declares_the_stage_entry_points():
     names = _declared()
     assert {"embbag_sum_multi", "interact_lower_tri", "dlrm_sparse_interact"} <= names
-    assert len(names) == 13
+    assert len(names) == 14
 
 
 def test_library_exports_every_declared_symbol(ops):
@@ -59,6 +59,9 @@ def test_status_strings_and_flags(ops):
     assert lib.dlrm_status_from_flags(1) == -5
     assert lib.dlrm_status_from_flags(2) == -6
     assert lib.dlrm_status_from_flags(3) == -5
+    assert lib.dlrm_status_from_flags(4) == -9
+    assert lib.dlrm_set_gather_path(7) == -8
+    assert lib.dlrm_set_gather_path(1) == 0 and lib.dlrm_set_gather_path(0) == 1
     assert lib.dlrm_launch_count() == 0
 
 

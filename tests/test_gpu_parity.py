@@ -28,6 +28,15 @@ def ops():
     return _ops
 
 
+@pytest.fixture(params=["auto", "ldg"], autouse=True)
+def gather_path(request, ops):
+    """Every test runs on the default path (TMA where the call qualifies) and on
+    the register-load path."""
+    prev = ops.set_gather_path(request.param)
+    yield request.param
+    ops.set_gather_path(prev)
+
+
 def _inputs(w: syn.Workload):
     weights = syn.make_weights(w, DEV)
     idx = syn.make_indices(w)
@@ -418,6 +427,22 @@ def test_host_pipeline_overlapped_batches(ops):
         torch.cuda.synchronize()
         assert torch.equal(o.view(torch.int32), ref.cpu().view(torch.int32))
     pipe.drain()
+
+
+def test_forced_tma_path(ops):
+    """The TMA gather serves qualifying calls bit-identically and refuses the rest."""
+    prev = ops.set_gather_path("tma")
+    try:
+        for (B, F, N, D, L) in [(70, 5, 300, 64, 16), (33, 26, 200, 128, 20), (19, 2, 50, 16, 4),
+                                (9, 3, 40, 48, 11)]:
+            weights, idx, off, dense = _random_case(B + F, B, F, N, D, L)
+            _check_against_oracle(ops, weights, idx, off, dense, B, L, True,
+                                  f"tma B{B} F{F} D{D} L{L}")
+        weights, idx, off, dense = _random_case(3, 8, 2, 20, 6, 3)  # 24-byte rows
+        with pytest.raises(ops.DlrmError, match="DLRM_ERR_UNSUPPORTED"):
+            ops.embbag_sum_multi(weights, _dev_i32(idx), _dev_i32(off), 3)
+    finally:
+        ops.set_gather_path(prev)
 
 
 def test_prepared_call_matches_plain_call(ops):

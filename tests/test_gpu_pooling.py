@@ -28,6 +28,15 @@ def ops():
     return _ops
 
 
+@pytest.fixture(params=["auto", "ldg"], autouse=True)
+def gather_path(request, ops):
+    """Every test runs on the default path (TMA where the call qualifies) and on
+    the register-load path."""
+    prev = ops.set_gather_path(request.param)
+    yield request.param
+    ops.set_gather_path(prev)
+
+
 def _host_bits(t: torch.Tensor) -> np.ndarray:
     """Host copy of a table: f32 values, or bf16 bit patterns as uint16."""
     if t.dtype == torch.bfloat16:
