@@ -133,11 +133,7 @@ dlrm::GatherPlan make_plan(const Prepared& pr, const int64_t* rows, int B, int F
   return g;
 }
 
-int launch_status(cudaError_t e) {
-  if (e == cudaSuccess) return DLRM_OK;
-  if (e == cudaErrorNotSupported) return DLRM_ERR_UNSUPPORTED;
-  return cuda_fail(e);
-}
+int launch_status(cudaError_t e) { return e == cudaSuccess ? DLRM_OK : cuda_fail(e); }
 
 int pool_impl(const void* const* weights, int dtype, const int64_t* rows, const dlrm_bags_t* bags,
               int B, int F, int D, float* out, int32_t* status_dev, cudaStream_t stream) {
@@ -341,6 +337,8 @@ int dlrm_set_gather_path(int path) {
   return prev;
 }
 
+int dlrm_last_gather_path(void) { return dlrm::last_path(); }
+
 int dlrm_status_from_flags(int32_t flags) {
   if (flags & DLRM_FLAG_TIMEOUT) return DLRM_ERR_TIMEOUT;
   if (flags & DLRM_FLAG_INDEX_OOB) return DLRM_ERR_INDEX_OOB;
@@ -360,7 +358,6 @@ const char* dlrm_status_string(int status) {
     case DLRM_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case DLRM_ERR_ARG: return "invalid argument";
     case DLRM_ERR_TIMEOUT: return "a bounded wait on an asynchronous copy ran out";
-    case DLRM_ERR_UNSUPPORTED: return "the requested gather path cannot serve this call";
     default: return "unknown status";
   }
 }

@@ -120,8 +120,10 @@ static cudaError_t counted(cudaError_t e) {
 // Path choice and the TMA path's tensor maps.
 
 static std::atomic<int> g_path{DLRM_PATH_AUTO};
+static thread_local int t_last_path = 0;
 int gather_path() { return g_path.load(std::memory_order_relaxed); }
 void set_gather_path(int path) { g_path.store(path, std::memory_order_relaxed); }
+int last_path() { return t_last_path; }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -176,14 +178,14 @@ static int sm_count() {
   return n;
 }
 
-static int tma_lanes(const GatherPlan& g) {
-  return std::min(32, std::max(4, pow2_ceil(g.D * g.esz / 16)));
-}
 
+// DLRM_PATH_AUTO takes the register-load path: on B200 it is faster than the
+// TMA path on the measured workloads (L1 serves the hot rows of skewed index
+// streams, which TMA loads bypass).
 cudaError_t launch_embbag(const GatherPlan& g, float* out, cudaStream_t stream) {
   const int path = gather_path();
-  if (path == DLRM_PATH_TMA && !g.tma_ok) return cudaErrorNotSupported;
-  if (g.tma_ok && path != DLRM_PATH_LDG) {
+  if (g.tma_ok && path == DLRM_PATH_TMA) {
+    t_last_path = DLRM_PATH_TMA;
     TmaParams tp;
     cudaError_t e = make_tma_params(g, &tp);
     if (e != cudaSuccess) return e;
@@ -193,13 +195,15 @@ cudaError_t launch_embbag(const GatherPlan& g, float* out, cudaStream_t stream) 
     a.B = g.B;
     a.F = g.F;
     a.D = g.D;
-    a.G = tma_lanes(g);
+    a.G = tma_unit_lanes(g.D * g.esz);
+    a.cpl = tma_chunks_per_lane(g.D * g.esz);
     a.pool = g.pool;
     a.out = out;
     a.sms = sm_count();
     a.stream = stream;
     return counted(g.esz == 4 ? launch_tma_gather_f32(a) : launch_tma_gather_bf16(a));
   }
+  t_last_path = DLRM_PATH_LDG;
   GatherLaunch a{g.tp, g.bp, g.B, g.F, g.D, out, g.pool, choose_gather_shape(g.D, g.loader),
                  stream};
   switch (g.loader) {
@@ -219,7 +223,8 @@ cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_
   bool tma_ok = g.tma_ok && (reinterpret_cast<uintptr_t>(dense) % 16 == 0);
   TmaLaunch t{};
   if (tma_ok) {
-    t.G = tma_lanes(g);
+    t.G = tma_unit_lanes(g.D * g.esz);
+    t.cpl = tma_chunks_per_lane(g.D * g.esz);
     const int units = kTmaGatherWarps * (32 / t.G);
     // about two bags per unit per tile; the dot warps take (S * nT) << lq tasks
     t.S = std::max(1, std::min(16, (2 * units + g.F - 1) / g.F));
@@ -230,8 +235,8 @@ cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_
     const int qmax = std::max(1, kTmaDotWarps * 32 / (t.S * Lf.nT));
     t.lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), 5});
   }
-  if (path == DLRM_PATH_TMA && !tma_ok) return cudaErrorNotSupported;
-  if (tma_ok && path != DLRM_PATH_LDG) {
+  if (tma_ok && path == DLRM_PATH_TMA) {
+    t_last_path = DLRM_PATH_TMA;
     TmaParams tp;
     cudaError_t e = make_tma_params(g, &tp);
     if (e != cudaSuccess) return e;
@@ -250,6 +255,7 @@ cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_
     t.stream = stream;
     return counted(g.esz == 4 ? launch_tma_fused_f32(t) : launch_tma_fused_bf16(t));
   }
+  t_last_path = DLRM_PATH_LDG;
   FusedLaunch a;
   a.g = GatherLaunch{g.tp, g.bp, g.B, g.F, g.D, nullptr, g.pool,
                      choose_gather_shape(g.D, g.loader), stream};

@@ -51,7 +51,8 @@ struct TmaLaunch {
   const TmaParams* tp;
   BagParams bp;
   int B, F, D;
-  int G;     // lanes per bag: pow2ceil(row bytes / 16), 4..32
+  int G;     // lanes per unit (8 or 16)
+  int cpl;   // 16-byte row chunks per lane (1 or 2)
   int pool;  // PoolKind
   float* out;  // gather-only output
   // fused
@@ -98,6 +99,8 @@ struct GatherPlan {
 // Process-wide choice of gather path (dlrm_set_gather_path).
 int gather_path();
 void set_gather_path(int path);
+// The path (DLRM_PATH_LDG / DLRM_PATH_TMA) of this thread's last gather launch.
+int last_path();
 
 // Picks the path and shape, then launches.
 cudaError_t launch_embbag(const GatherPlan& g, float* out, cudaStream_t stream);

@@ -3,12 +3,15 @@
 // Rows are fetched with the tensor-map tile::gather4 load: one instruction
 // brings four arbitrary rows of a table into shared memory and reports their
 // bytes on an mbarrier. A lane group ("unit") of G lanes pools one bag at a
-// time and keeps its own ring of kTmaBufs segment buffers (kTmaSegRows rows
+// time; lane q owns the 16-byte chunks q, q+G, ... (CPL of them) of a row.
+// Each unit keeps its own ring of kTmaBufs segment buffers (kTmaSegRows rows
 // each) in flight ahead of the segment it is summing, so the bytes in flight
-// are bounded by shared memory, not by registers. Row ids (and per-sample
-// weights) of the next segment are fetched one step ahead with ordinary loads
-// and published in shared memory for the issuing lane and the summing lanes;
-// bag bounds are fetched one bag ahead.
+// cost shared memory, not registers. Measured on B200, the gather4 stream
+// reaches the HBM copy rate only with about 32 independently issuing units per
+// SM, so units are narrow (G = 8 for rows up to 256 bytes) and a block holds
+// 32 of them. Row ids (and per-sample weights) of the next segment are fetched
+// one step ahead with ordinary loads and published in shared memory for the
+// issuing lane and the summing lanes; bag bounds are fetched one bag ahead.
 //
 // Blocks are persistent. In the fused kernel, gather warps pool the bags of
 // tile t into one of two feature buffers while dot warps compute the
@@ -28,7 +31,7 @@ namespace dlrm {
 
 constexpr int kTmaQuadsPerSeg = 2;
 constexpr int kTmaSegRows = 4 * kTmaQuadsPerSeg;
-constexpr int kTmaBufs = 4;
+constexpr int kTmaBufs = 2;
 constexpr int kTmaGatherWarps = 8;
 constexpr int kTmaDotWarps = 4;
 constexpr long long kTmaWaitLimit = 200000000LL;  // clock cycles, about 0.1 s
@@ -142,9 +145,9 @@ struct BagOrder {
   }
 };
 
-template <int G, int POOL, int ESZ, bool FUSED>
+template <int G, int CPL, int POOL, int ESZ, bool FUSED>
 struct TmaUnit {
-  static constexpr int VEC = 16 / ESZ;                   // table elements per lane
+  static constexpr int VEC = 16 / ESZ;                   // table elements per 16-byte chunk
   static constexpr int IPL = (kTmaSegRows + G - 1) / G;  // row ids per lane
 
   unsigned char* ring;
@@ -164,9 +167,11 @@ struct TmaUnit {
   // consume side
   int c;
   uint32_t phase;
-  float acc[VEC];
+  float acc[CPL][VEC];
   int used;
   bool oob, bad, timeout;
+
+  __device__ __forceinline__ bool chunk_ok(int m) const { return (q + G * m) * 16 < box_bytes; }
 
   __device__ __forceinline__ void prefetch_rows(const BagParams& bp) {
 #pragma unroll
@@ -250,7 +255,8 @@ struct TmaUnit {
     if (cur.valid) advance(bp);
   }
 
-  __device__ __forceinline__ void combine(const uint4& raw, float w) {
+  __device__ __forceinline__ void combine(float (&a)[VEC], const uint4& raw, float w,
+                                          bool first) {
     float x[VEC];
     if constexpr (ESZ == 4) {
       x[0] = __uint_as_float(raw.x);
@@ -265,23 +271,22 @@ struct TmaUnit {
         x[2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
       }
     }
-    const bool first = used == 0;
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
       if (POOL == kPoolSum) {
-        acc[e] = __fadd_rn(acc[e], x[e]);
+        a[e] = __fadd_rn(a[e], x[e]);
       } else if (POOL == kPoolWeighted) {
-        acc[e] = __fmaf_rn(w, x[e], acc[e]);
+        a[e] = __fmaf_rn(w, x[e], a[e]);
       } else {
-        acc[e] = first ? x[e] : ((x[e] > acc[e]) ? x[e] : acc[e]);
+        a[e] = first ? x[e] : ((x[e] > a[e]) ? x[e] : a[e]);
       }
     }
   }
 
   // Consume the next buffer if it belongs to tile `lt` (fused) or exists
   // (gather); refills the previously consumed buffer first. Returns false at
-  // the end of the tile or of the sequence. On a finished bag, `out_row` gets
-  // the pooled vector's destination(s) through `store`.
+  // the end of the tile or of the sequence. A finished bag's pooled vector
+  // goes to `store(meta, chunk m, values)` for each chunk the lane owns.
   template <class Store>
   __device__ __forceinline__ bool step(int lt, const TmaParams& tp, const BagParams& bp,
                                        Store&& store) {
@@ -298,10 +303,11 @@ struct TmaUnit {
     }
     if (m.r0 == 0) {
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+      for (int mm = 0; mm < CPL; ++mm)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[mm][e] = 0.f;
       used = 0;
     }
-    const bool lane_has_cols = q * 16 < box_bytes;
     const int rows_k = bp.check ? tp.rows[m.k] : 0;
     const unsigned char* base = ring + buf * buf_bytes + q * 16;
     for (int r = 0; r < m.nrows; ++r) {
@@ -312,10 +318,14 @@ struct TmaUnit {
         oob |= !ok;
       }
       if (ok) {
-        if (lane_has_cols) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(base + (r >> 2) * quad_stride +
-                                                            (r & 3) * box_bytes);
-          combine(raw, POOL == kPoolWeighted ? wts[buf * kTmaSegRows + r] : 0.f);
+        const float w = POOL == kPoolWeighted ? wts[buf * kTmaSegRows + r] : 0.f;
+        const unsigned char* row = base + (r >> 2) * quad_stride + (r & 3) * box_bytes;
+#pragma unroll
+        for (int mm = 0; mm < CPL; ++mm) {
+          if (chunk_ok(mm)) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(row + mm * G * 16);
+            combine(acc[mm], raw, w, used == 0);
+          }
         }
         ++used;
       }
@@ -324,9 +334,13 @@ struct TmaUnit {
       if (bp.mean && used > 0) {
         const float cnt = static_cast<float>(used);
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[e] = __fdiv_rn(acc[e], cnt);
+        for (int mm = 0; mm < CPL; ++mm)
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) acc[mm][e] = __fdiv_rn(acc[mm][e], cnt);
       }
-      if (lane_has_cols) store(m, acc);
+#pragma unroll
+      for (int mm = 0; mm < CPL; ++mm)
+        if (chunk_ok(mm)) store(m, mm, acc[mm]);
     }
     __syncwarp(mask);
     fence_proxy_async_smem();  // our reads of this buffer precede its next TMA fill
@@ -343,9 +357,10 @@ __device__ __forceinline__ void store_vec_f32(float* p, const float (&a)[VEC]) {
 }
 
 // Shared set-up of the gather units of a block.
-template <int G, int POOL, int ESZ, bool FUSED>
-__device__ __forceinline__ void init_unit(TmaUnit<G, POOL, ESZ, FUSED>& U, unsigned char* smem,
-                                          const TmaSmem& L, int B, int F, int S, int my_tiles) {
+template <int G, int CPL, int POOL, int ESZ, bool FUSED>
+__device__ __forceinline__ void init_unit(TmaUnit<G, CPL, POOL, ESZ, FUSED>& U,
+                                          unsigned char* smem, const TmaSmem& L, int B, int F,
+                                          int S, int my_tiles) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int u = warp * (32 / G) + lane / G;
   U.q = lane % G;
@@ -371,11 +386,12 @@ __device__ __forceinline__ void tma_report(const BagParams& bp, bool oob, bool b
 
 // --------------------------------------------------------------------------
 // Gather only: persistent blocks of gather units writing pooled rows to `out`.
-template <int G, int POOL, int ESZ>
+template <int G, int CPL, int POOL, int ESZ>
 __global__ void __launch_bounds__(kTmaGatherWarps * 32, 1)
     tma_embbag_kernel(const __grid_constant__ TmaParams tp, const BagParams bp, int B, int F,
                       int D, float* __restrict__ out) {
   extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int VEC = 16 / ESZ;
   const TmaSmem L = TmaSmem::make(G, D * ESZ, 0);
   for (int i = threadIdx.x; i < L.units * kTmaBufs; i += blockDim.x) {
     mbar_init(reinterpret_cast<uint64_t*>(smem + L.bars_off) + i, 1);
@@ -383,13 +399,13 @@ __global__ void __launch_bounds__(kTmaGatherWarps * 32, 1)
   mbar_init_fence();
   __syncthreads();
 
-  TmaUnit<G, POOL, ESZ, false> U;
+  TmaUnit<G, CPL, POOL, ESZ, false> U;
   init_unit(U, smem, L, B, F, 1, 0);
   U.start(bp);
   for (int i = 0; i < kTmaBufs - 1; ++i) U.issue(i, tp, bp);
-  constexpr int VEC = 16 / ESZ;
-  auto store = [&](const SegMeta& m, const float (&a)[VEC]) {
-    store_vec_f32<VEC>(out + (static_cast<int64_t>(m.b) * F + m.k) * D + U.q * VEC, a);
+  auto store = [&](const SegMeta& m, int mm, const float (&a)[VEC]) {
+    store_vec_f32<VEC>(out + (static_cast<int64_t>(m.b) * F + m.k) * D + (U.q + G * mm) * VEC,
+                       a);
   };
   while (U.step(0, tp, bp, store)) {
   }
@@ -399,7 +415,7 @@ __global__ void __launch_bounds__(kTmaGatherWarps * 32, 1)
 // --------------------------------------------------------------------------
 // Fused: gather warps pool tile lt into feature buffer lt&1 while dot warps
 // finish tile lt-1; each tile holds S consecutive samples.
-template <int G, int POOL, int ESZ>
+template <int G, int CPL, int POOL, int ESZ>
 __global__ void __launch_bounds__((kTmaGatherWarps + kTmaDotWarps) * 32, 1)
     tma_fused_kernel(const __grid_constant__ TmaParams tp, const BagParams bp,
                      const float* __restrict__ dense, int B, int F, int D, int S, int lq,
@@ -427,7 +443,7 @@ __global__ void __launch_bounds__((kTmaGatherWarps + kTmaDotWarps) * 32, 1)
   const int warp = threadIdx.x >> 5;
 
   if (warp < kTmaGatherWarps) {
-    TmaUnit<G, POOL, ESZ, true> U;
+    TmaUnit<G, CPL, POOL, ESZ, true> U;
     init_unit(U, smem, L, B, F, S, my_tiles);
     U.start(bp);
     for (int i = 0; i < kTmaBufs - 1; ++i) U.issue(i, tp, bp);
@@ -437,12 +453,12 @@ __global__ void __launch_bounds__((kTmaGatherWarps + kTmaDotWarps) * 32, 1)
       float* fb = feat + p * S * sample_floats;
       const int64_t b0 = (static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(lt) *
                                                                  gridDim.x) * S;
-      auto store = [&](const SegMeta& m, const float (&a)[VEC]) {
+      auto store = [&](const SegMeta& m, int mm, const float (&a)[VEC]) {
         const int s = static_cast<int>(m.b - b0);
-        store_vec_f32<VEC>(fb + s * sample_floats + (1 + m.k) * Lf.Dp + U.q * VEC, a);
+        const int col = (U.q + G * mm) * VEC;
+        store_vec_f32<VEC>(fb + s * sample_floats + (1 + m.k) * Lf.Dp + col, a);
         if (pooled_out)
-          store_vec_f32<VEC>(pooled_out + (static_cast<int64_t>(m.b) * F + m.k) * D + U.q * VEC,
-                             a);
+          store_vec_f32<VEC>(pooled_out + (static_cast<int64_t>(m.b) * F + m.k) * D + col, a);
       };
       while (U.step(lt, tp, bp, store)) {
       }
@@ -489,9 +505,9 @@ __global__ void __launch_bounds__((kTmaGatherWarps + kTmaDotWarps) * 32, 1)
 // --------------------------------------------------------------------------
 // Host-side dispatch.
 
-template <int G, int POOL, int ESZ>
+template <int G, int CPL, int POOL, int ESZ>
 cudaError_t run_tma_gather(const TmaLaunch& a) {
-  auto* fn = &tma_embbag_kernel<G, POOL, ESZ>;
+  auto* fn = &tma_embbag_kernel<G, CPL, POOL, ESZ>;
   const TmaSmem L = TmaSmem::make(G, a.D * ESZ, 0);
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -508,9 +524,9 @@ cudaError_t run_tma_gather(const TmaLaunch& a) {
   return cudaGetLastError();
 }
 
-template <int G, int POOL, int ESZ>
+template <int G, int CPL, int POOL, int ESZ>
 cudaError_t run_tma_fused(const TmaLaunch& a) {
-  auto* fn = &tma_fused_kernel<G, POOL, ESZ>;
+  auto* fn = &tma_fused_kernel<G, CPL, POOL, ESZ>;
   const FeatLayout Lf = FeatLayout::make(a.F, a.D);
   const TmaSmem L = TmaSmem::make(G, a.D * ESZ, 2 * a.S * Lf.floats_per_sample() * 4);
   if (L.total > a.smem_limit) return cudaErrorInvalidValue;
@@ -530,21 +546,26 @@ cudaError_t run_tma_fused(const TmaLaunch& a) {
   return cudaGetLastError();
 }
 
-#define DLRM_TMA_POOLS(RUN, G_, ESZ_, a)                                         \
+// Lanes per unit and 16-byte chunks per lane for a row of `row_bytes`:
+// G = 8 (32 units per block) up to 256-byte rows, G = 16 (16 units) above.
+__host__ __device__ inline int tma_unit_lanes(int row_bytes) { return row_bytes <= 256 ? 8 : 16; }
+__host__ __device__ inline int tma_chunks_per_lane(int row_bytes) {
+  const int G = tma_unit_lanes(row_bytes);
+  return (row_bytes / 16 + G - 1) / G;
+}
+
+#define DLRM_TMA_POOLS(RUN, G_, C_, ESZ_, a)                                      \
   do {                                                                          \
-    if ((a).pool == kPoolSum) return RUN<G_, kPoolSum, ESZ_>(a);                \
-    if ((a).pool == kPoolWeighted) return RUN<G_, kPoolWeighted, ESZ_>(a);      \
-    return RUN<G_, kPoolMax, ESZ_>(a);                                          \
+    if ((a).pool == kPoolSum) return RUN<G_, C_, kPoolSum, ESZ_>(a);            \
+    if ((a).pool == kPoolWeighted) return RUN<G_, C_, kPoolWeighted, ESZ_>(a);  \
+    return RUN<G_, C_, kPoolMax, ESZ_>(a);                                      \
   } while (0)
 
 #define DLRM_TMA_DISPATCH(RUN, ESZ_, a)                                          \
   do {                                                                          \
-    switch ((a).G) {                                                            \
-      case 4: DLRM_TMA_POOLS(RUN, 4, ESZ_, a);                                  \
-      case 8: DLRM_TMA_POOLS(RUN, 8, ESZ_, a);                                  \
-      case 16: DLRM_TMA_POOLS(RUN, 16, ESZ_, a);                                \
-      default: DLRM_TMA_POOLS(RUN, 32, ESZ_, a);                                \
-    }                                                                           \
+    if ((a).G == 8 && (a).cpl == 1) DLRM_TMA_POOLS(RUN, 8, 1, ESZ_, a);          \
+    if ((a).G == 8) DLRM_TMA_POOLS(RUN, 8, 2, ESZ_, a);                         \
+    DLRM_TMA_POOLS(RUN, 16, 2, ESZ_, a);                                        \
   } while (0)
 
 }  // namespace dlrm

@@ -29,7 +29,6 @@ STATUS = {
     -7: "DLRM_ERR_CUDA",
     -8: "DLRM_ERR_ARG",
     -9: "DLRM_ERR_TIMEOUT",
-    -10: "DLRM_ERR_UNSUPPORTED",
 }
 GATHER_PATHS = {"auto": 0, "ldg": 1, "tma": 2}
 FLAG_INDEX_OOB = 1
@@ -52,6 +51,7 @@ SIGNATURES = {
     "dlrm_sparse_interact_pool": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _I, _P, _P]),
     "dlrm_pair_decode": (_I, [_I64, _I64, _P, _P, _P]),
     "dlrm_set_gather_path": (_I, [_I]),
+    "dlrm_last_gather_path": (_I, []),
     "dlrm_status_from_flags": (_I, [ctypes.c_int32]),
     "dlrm_status_string": (ctypes.c_char_p, [_I]),
     "dlrm_last_cuda_error": (_I, []),
@@ -476,6 +476,11 @@ def set_gather_path(path: str) -> str:
     if prev < 0:
         raise DlrmError(prev, "dlrm_set_gather_path")
     return {v: k for k, v in GATHER_PATHS.items()}[prev]
+
+
+def last_gather_path() -> str:
+    """The path that served this thread's last gather or fused launch ("ldg"/"tma")."""
+    return {0: "none", 1: "ldg", 2: "tma"}[_lib.dlrm_last_gather_path()]
 
 
 def status_from_flags(flags: int) -> int:

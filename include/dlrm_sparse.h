@@ -76,9 +76,8 @@ typedef enum {
     DLRM_ERR_CUDA = -7,            /* a CUDA runtime call or launch failed; see
                                       dlrm_last_cuda_error() */
     DLRM_ERR_ARG = -8,             /* any other invalid argument (e.g. count < 0) */
-    DLRM_ERR_TIMEOUT = -9,         /* (device flag) a bounded wait on an asynchronous
+    DLRM_ERR_TIMEOUT = -9          /* (device flag) a bounded wait on an asynchronous
                                       copy ran out; the results are not valid */
-    DLRM_ERR_UNSUPPORTED = -10     /* the requested gather path cannot serve this call */
 } dlrm_status_t;
 
 /* Bits that the checked (_ex) entry points OR into *status_dev. */
@@ -87,10 +86,10 @@ typedef enum {
 #define DLRM_FLAG_TIMEOUT 4
 
 /* Gather paths (dlrm_set_gather_path). */
-#define DLRM_PATH_AUTO 0 /* TMA gather when the call qualifies, else register loads */
+#define DLRM_PATH_AUTO 0 /* the path measured fastest on B200: register loads */
 #define DLRM_PATH_LDG 1  /* always the register-load (128-bit ld.global.nc) gather */
-#define DLRM_PATH_TMA 2  /* always the TMA tile::gather4 gather; DLRM_ERR_UNSUPPORTED
-                            for calls it cannot serve */
+#define DLRM_PATH_TMA 2  /* the TMA tile::gather4 gather for the calls that qualify
+                            (see dlrm_set_gather_path), register loads for the rest */
 
 /* Pooling of a bag's rows (torch.nn.EmbeddingBag modes). The pages implement
  * only SUM and name the others as what a later model would need (movement.rs,
@@ -280,6 +279,10 @@ DLRM_API int dlrm_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_t
  * reads zeros on this path instead of other memory.
  */
 DLRM_API int dlrm_set_gather_path(int path);
+
+/* The path (DLRM_PATH_LDG or DLRM_PATH_TMA) that served the calling thread's
+ * last gather or fused launch; 0 before the first one. */
+DLRM_API int dlrm_last_gather_path(void);
 
 /* Status of a *status_dev value written by an _ex call (DLRM_OK if 0). */
 DLRM_API int dlrm_status_from_flags(int32_t flags);

@@ -32,7 +32,7 @@ def ops():
 def test_header_declares_the_stage_entry_points():
     names = _declared()
     assert {"embbag_sum_multi", "interact_lower_tri", "dlrm_sparse_interact"} <= names
-    assert len(names) == 14
+    assert len(names) == 15
 
 
 def test_library_exports_every_declared_symbol(ops):

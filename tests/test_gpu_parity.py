@@ -28,10 +28,10 @@ def ops():
     return _ops
 
 
-@pytest.fixture(params=["auto", "ldg"], autouse=True)
+@pytest.fixture(params=["tma", "ldg"], autouse=True)
 def gather_path(request, ops):
-    """Every test runs on the default path (TMA where the call qualifies) and on
-    the register-load path."""
+    """Every test runs on the TMA gather path (where the call qualifies; the
+    register-load path serves the rest) and on the register-load path."""
     prev = ops.set_gather_path(request.param)
     yield request.param
     ops.set_gather_path(prev)
@@ -429,18 +429,25 @@ def test_host_pipeline_overlapped_batches(ops):
     pipe.drain()
 
 
-def test_forced_tma_path(ops):
-    """The TMA gather serves qualifying calls bit-identically and refuses the rest."""
+def test_path_choice(ops):
+    """Under "tma" qualifying calls run the TMA gather, the others register loads."""
     prev = ops.set_gather_path("tma")
     try:
         for (B, F, N, D, L) in [(70, 5, 300, 64, 16), (33, 26, 200, 128, 20), (19, 2, 50, 16, 4),
                                 (9, 3, 40, 48, 11)]:
             weights, idx, off, dense = _random_case(B + F, B, F, N, D, L)
-            _check_against_oracle(ops, weights, idx, off, dense, B, L, True,
-                                  f"tma B{B} F{F} D{D} L{L}")
+            ops.embbag_sum_multi(weights, _dev_i32(idx), _dev_i32(off), L)
+            assert ops.last_gather_path() == "tma"
+            ops.sparse_interact(weights, _dev_i32(idx), _dev_i32(off), dense, L)
+            assert ops.last_gather_path() == "tma"
         weights, idx, off, dense = _random_case(3, 8, 2, 20, 6, 3)  # 24-byte rows
-        with pytest.raises(ops.DlrmError, match="DLRM_ERR_UNSUPPORTED"):
-            ops.embbag_sum_multi(weights, _dev_i32(idx), _dev_i32(off), 3)
+        ops.embbag_sum_multi(weights, _dev_i32(idx), _dev_i32(off), 3)
+        assert ops.last_gather_path() == "ldg"
+        ops.set_gather_path("ldg")
+        weights, idx, off, dense = _random_case(4, 8, 2, 20, 64, 3)
+        ops.sparse_interact(weights, _dev_i32(idx), _dev_i32(off), dense, 3)
+        assert ops.last_gather_path() == "ldg"
+        torch.cuda.synchronize()
     finally:
         ops.set_gather_path(prev)
 

@@ -28,10 +28,10 @@ def ops():
     return _ops
 
 
-@pytest.fixture(params=["auto", "ldg"], autouse=True)
+@pytest.fixture(params=["tma", "ldg"], autouse=True)
 def gather_path(request, ops):
-    """Every test runs on the default path (TMA where the call qualifies) and on
-    the register-load path."""
+    """Every test runs on the TMA gather path (where the call qualifies; the
+    register-load path serves the rest) and on the register-load path."""
     prev = ops.set_gather_path(request.param)
     yield request.param
     ops.set_gather_path(prev)
