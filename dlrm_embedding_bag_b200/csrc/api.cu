@@ -330,7 +330,8 @@ int dlrm_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_t* j_out,
 }
 
 int dlrm_set_gather_path(int path) {
-  if (path != DLRM_PATH_AUTO && path != DLRM_PATH_LDG && path != DLRM_PATH_TMA)
+  if (path != DLRM_PATH_AUTO && path != DLRM_PATH_LDG && path != DLRM_PATH_TMA &&
+      path != DLRM_PATH_PIPE)
     return DLRM_ERR_ARG;
   const int prev = dlrm::gather_path();
   dlrm::set_gather_path(path);

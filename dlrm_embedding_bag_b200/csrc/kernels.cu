@@ -10,6 +10,7 @@
 
 #include "interact_common.cuh"
 #include "launch.h"
+#include "pipe_kernels.cuh"
 #include "tma_kernels.cuh"
 
 namespace dlrm {
@@ -179,9 +180,10 @@ static int sm_count() {
 }
 
 
-// DLRM_PATH_AUTO takes the register-load path: on B200 it is faster than the
-// TMA path on the measured workloads (L1 serves the hot rows of skewed index
-// streams, which TMA loads bypass).
+// DLRM_PATH_AUTO takes the per-block register-load kernels: on B200 they are
+// faster than the TMA path on the measured workloads (L1 serves the hot rows
+// of skewed index streams, which TMA loads bypass) and than the pipelined
+// path (whose fused kernel has fewer warps to hide latency with).
 cudaError_t launch_embbag(const GatherPlan& g, float* out, cudaStream_t stream) {
   const int path = gather_path();
   if (g.tma_ok && path == DLRM_PATH_TMA) {
@@ -203,9 +205,26 @@ cudaError_t launch_embbag(const GatherPlan& g, float* out, cudaStream_t stream) 
     a.stream = stream;
     return counted(g.esz == 4 ? launch_tma_gather_f32(a) : launch_tma_gather_bf16(a));
   }
+  const GatherShape sh = choose_gather_shape(g.D, g.loader);
+  const bool pipe_ok = (g.loader == kLdF32x4 || g.loader == kLdBF16x8) && sh.ncolwin == 1;
+  if (pipe_ok && path == DLRM_PATH_PIPE) {
+    t_last_path = DLRM_PATH_PIPE;
+    PipeLaunch a{};
+    a.tp = g.tp;
+    a.bp = g.bp;
+    a.B = g.B;
+    a.F = g.F;
+    a.D = g.D;
+    a.G = sh.G;
+    a.cpl = sh.cpl;
+    a.pool = g.pool;
+    a.out = out;
+    a.sms = sm_count();
+    a.stream = stream;
+    return counted(g.esz == 4 ? launch_pipe_gather_f32(a) : launch_pipe_gather_bf16(a));
+  }
   t_last_path = DLRM_PATH_LDG;
-  GatherLaunch a{g.tp, g.bp, g.B, g.F, g.D, out, g.pool, choose_gather_shape(g.D, g.loader),
-                 stream};
+  GatherLaunch a{g.tp, g.bp, g.B, g.F, g.D, out, g.pool, sh, stream};
   switch (g.loader) {
     case kLdF32x4: return counted(launch_gather_f32x4(a));
     case kLdF32x1: return counted(launch_gather_f32x1(a));
@@ -255,10 +274,40 @@ cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_
     t.stream = stream;
     return counted(g.esz == 4 ? launch_tma_fused_f32(t) : launch_tma_fused_bf16(t));
   }
+  const GatherShape sh = choose_gather_shape(g.D, g.loader);
+  const bool pipe_ok = (g.loader == kLdF32x4 || g.loader == kLdBF16x8) && sh.ncolwin == 1;
+  if (pipe_ok && path == DLRM_PATH_PIPE) {
+    PipeLaunch a{};
+    const int units = kPipeGatherWarps * 32 / sh.G;
+    // about two bags per unit per tile, two tiles of features in shared memory
+    a.S = std::max(1, std::min({16, (2 * units + g.F - 1) / g.F, g.B}));
+    const int64_t per = Lf.floats_per_sample() * 4;
+    while (a.S > 1 && 2 * a.S * per > smem_limit) --a.S;
+    a.smem = 2 * a.S * per;
+    if (a.smem <= smem_limit) {
+      t_last_path = DLRM_PATH_PIPE;
+      const int qmax = std::max(1, kPipeDotWarps * 32 / (a.S * Lf.nT));
+      a.lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), 5});
+      a.tp = g.tp;
+      a.bp = g.bp;
+      a.B = g.B;
+      a.F = g.F;
+      a.D = g.D;
+      a.G = sh.G;
+      a.cpl = sh.cpl;
+      a.pool = g.pool;
+      a.dense = dense;
+      a.pooled_out = pooled_out;
+      a.inter_out = inter_out;
+      a.concat_dense = concat_dense;
+      a.sms = sm_count();
+      a.stream = stream;
+      return counted(g.esz == 4 ? launch_pipe_fused_f32(a) : launch_pipe_fused_bf16(a));
+    }
+  }
   t_last_path = DLRM_PATH_LDG;
   FusedLaunch a;
-  a.g = GatherLaunch{g.tp, g.bp, g.B, g.F, g.D, nullptr, g.pool,
-                     choose_gather_shape(g.D, g.loader), stream};
+  a.g = GatherLaunch{g.tp, g.bp, g.B, g.F, g.D, nullptr, g.pool, sh, stream};
   a.dense = dense;
   a.pooled_out = pooled_out;
   a.inter_out = inter_out;

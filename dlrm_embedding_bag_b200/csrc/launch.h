@@ -66,6 +66,29 @@ struct TmaLaunch {
   cudaStream_t stream;
 };
 
+// The persistent pipelined register-load path.
+struct PipeLaunch {
+  const TableParams* tp;
+  BagParams bp;
+  int B, F, D;
+  int G, cpl;  // lanes per unit, 16-byte chunks per lane
+  int pool;
+  float* out;  // gather-only output
+  const float* dense;
+  float* pooled_out;
+  float* inter_out;
+  int concat_dense;
+  int S, lq;
+  int64_t smem;
+  int sms;
+  cudaStream_t stream;
+};
+
+cudaError_t launch_pipe_gather_f32(const PipeLaunch& a);
+cudaError_t launch_pipe_gather_bf16(const PipeLaunch& a);
+cudaError_t launch_pipe_fused_f32(const PipeLaunch& a);
+cudaError_t launch_pipe_fused_bf16(const PipeLaunch& a);
+
 cudaError_t launch_tma_gather_f32(const TmaLaunch& a);
 cudaError_t launch_tma_gather_bf16(const TmaLaunch& a);
 cudaError_t launch_tma_fused_f32(const TmaLaunch& a);

@@ -25,6 +25,7 @@
 
 #include "interact_common.cuh"
 #include "launch.h"
+#include "persist_common.cuh"
 #include "tma_common.cuh"
 
 namespace dlrm {
@@ -35,8 +36,6 @@ constexpr int kTmaBufs = 2;
 constexpr int kTmaGatherWarps = 8;
 constexpr int kTmaDotWarps = 4;
 constexpr long long kTmaWaitLimit = 200000000LL;  // clock cycles, about 0.1 s
-
-enum { kBarReady0 = 1, kBarFree0 = 3 };
 
 // What one issued segment holds; written by the unit before it issues.
 struct SegMeta {
@@ -70,78 +69,6 @@ struct TmaSmem {
     s.feat_off = ((s.wts_off + nb * kTmaSegRows * 4 + 15) / 16) * 16;
     s.total = s.feat_off + feat_bytes;
     return s;
-  }
-};
-
-// Where a unit's bags come from.
-//  fused  : the block's tiles lt = 0, 1, ... (tile t = blockIdx.x + lt*gridDim.x
-//           of S samples); within a tile, bags j = u, u + units, ... of S_t*F.
-//  gather : global bag ids g = blockIdx.x*units + u + i*gridDim.x*units.
-struct BagPos {
-  int valid, lt, j;  // j: bag within the tile (fused) or global bag id (gather)
-  int b, k, start, n;
-  bool bad;
-};
-
-template <bool FUSED>
-struct BagOrder {
-  int B, F, S, units, u, my_tiles;
-  __device__ __forceinline__ int tile_samples(int lt) const {
-    const int64_t t = static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(lt) * gridDim.x;
-    const int64_t rem = B - t * S;
-    return rem < S ? static_cast<int>(rem) : S;
-  }
-  __device__ __forceinline__ void first(BagPos& p) const {
-    if (FUSED) {
-      p.lt = 0;
-      p.j = u;
-      p.valid = 0;
-      while (p.lt < my_tiles) {
-        if (p.j < tile_samples(p.lt) * F) {
-          p.valid = 1;
-          break;
-        }
-        ++p.lt;
-      }
-    } else {
-      p.lt = 0;
-      p.j = static_cast<int>(blockIdx.x) * units + u;
-      p.valid = static_cast<int64_t>(p.j) < static_cast<int64_t>(B) * F;
-    }
-  }
-  __device__ __forceinline__ void next(const BagPos& c, BagPos& p) const {
-    p = c;
-    if (!c.valid) return;
-    if (FUSED) {
-      p.j = c.j + units;
-      while (p.lt < my_tiles && p.j >= tile_samples(p.lt) * F) {
-        ++p.lt;
-        p.j = u;
-      }
-      p.valid = p.lt < my_tiles;
-    } else {
-      const int64_t g = static_cast<int64_t>(c.j) + static_cast<int64_t>(gridDim.x) * units;
-      p.valid = g < static_cast<int64_t>(B) * F;
-      p.j = p.valid ? static_cast<int>(g) : 0;
-    }
-  }
-  // Fill b, k and start the load of the bag's bounds.
-  __device__ __forceinline__ void locate(BagPos& p, const BagParams& bp) const {
-    if (!p.valid) {
-      p.b = p.k = p.start = p.n = 0;
-      p.bad = false;
-      return;
-    }
-    if (FUSED) {
-      const int s = p.j / F;
-      p.k = p.j - s * F;
-      p.b = static_cast<int>((static_cast<int64_t>(blockIdx.x) +
-                              static_cast<int64_t>(p.lt) * gridDim.x) * S) + s;
-    } else {
-      p.b = p.j / F;
-      p.k = p.j - p.b * F;
-    }
-    bag_bounds(bp, B, p.k, p.b, p.start, p.n, p.bad);
   }
 };
 
@@ -349,13 +276,6 @@ struct TmaUnit {
   }
 };
 
-template <int VEC>
-__device__ __forceinline__ void store_vec_f32(float* p, const float (&a)[VEC]) {
-#pragma unroll
-  for (int e = 0; e < VEC; e += 4)
-    *reinterpret_cast<float4*>(p + e) = make_float4(a[e], a[e + 1], a[e + 2], a[e + 3]);
-}
-
 // Shared set-up of the gather units of a block.
 template <int G, int CPL, int POOL, int ESZ, bool FUSED>
 __device__ __forceinline__ void init_unit(TmaUnit<G, CPL, POOL, ESZ, FUSED>& U,
@@ -467,38 +387,8 @@ __global__ void __launch_bounds__((kTmaGatherWarps + kTmaDotWarps) * 32, 1)
     }
     if (U.q == 0) tma_report(bp, U.oob, U.bad, U.timeout);
   } else {
-    const int tid = threadIdx.x - kTmaGatherWarps * 32;
-    constexpr int nthr = kTmaDotWarps * 32;
-    const bool dense_vec = ((D & 3) == 0) && ((reinterpret_cast<uintptr_t>(dense) & 15) == 0);
-    for (int lt = 0; lt < my_tiles; ++lt) {
-      const int p = lt & 1;
-      float* fb = feat + p * S * sample_floats;
-      const int64_t b0 = (static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(lt) *
-                                                                 gridDim.x) * S;
-      const int S_t = (B - b0 < S) ? static_cast<int>(B - b0) : S;
-      for (int s = 0; s < S_t; ++s) {
-        const float* src = dense + (b0 + s) * D;
-        float* dst = fb + s * sample_floats;
-        if (dense_vec) {
-          for (int c4 = tid; c4 < (D >> 2); c4 += nthr)
-            reinterpret_cast<float4*>(dst)[c4] = __ldg(reinterpret_cast<const float4*>(src) + c4);
-        } else {
-          for (int c1 = tid; c1 < D; c1 += nthr) dst[c1] = __ldg(src + c1);
-        }
-      }
-      zero_feature_padding(fb, Lf, D, S_t, tid, nthr);
-      named_bar_sync(kBarReady0 + p, NT);
-      if (concat_dense) {
-        for (int s = 0; s < S_t; ++s) {
-          const float* src = fb + s * sample_floats;
-          float* dst = inter_out + (b0 + s) * row_stride;
-          for (int d = tid; d < D; d += nthr) dst[d] = src[d];
-        }
-      }
-      dots_from_smem(fb, Lf, S_t, lq, inter_out, b0, row_stride, concat_dense ? D : 0, tid,
-                     nthr);
-      if (lt + 2 < my_tiles) named_bar_arrive(kBarFree0 + p, NT);
-    }
+    fused_dot_warps<kTmaGatherWarps, kTmaDotWarps>(feat, Lf, dense, B, D, S, lq, my_tiles,
+                                                   inter_out, concat_dense);
   }
 }
 

@@ -30,7 +30,7 @@ STATUS = {
     -8: "DLRM_ERR_ARG",
     -9: "DLRM_ERR_TIMEOUT",
 }
-GATHER_PATHS = {"auto": 0, "ldg": 1, "tma": 2}
+GATHER_PATHS = {"auto": 0, "ldg": 1, "tma": 2, "pipe": 3}
 FLAG_INDEX_OOB = 1
 FLAG_OFFSETS = 2
 FLAG_TIMEOUT = 4
@@ -471,7 +471,7 @@ def pair_decode(p0: int, count: int, device="cuda"):
 
 
 def set_gather_path(path: str) -> str:
-    """Choose the gather path for later calls ("auto", "ldg" or "tma"); returns the old one."""
+    """Choose the gather path for later calls ("auto", "ldg", "tma", "pipe"); returns the old one."""
     prev = _lib.dlrm_set_gather_path(GATHER_PATHS[path])
     if prev < 0:
         raise DlrmError(prev, "dlrm_set_gather_path")
@@ -479,8 +479,8 @@ def set_gather_path(path: str) -> str:
 
 
 def last_gather_path() -> str:
-    """The path that served this thread's last gather or fused launch ("ldg"/"tma")."""
-    return {0: "none", 1: "ldg", 2: "tma"}[_lib.dlrm_last_gather_path()]
+    """The path that served this thread's last gather or fused launch."""
+    return {0: "none", 1: "ldg", 2: "tma", 3: "pipe"}[_lib.dlrm_last_gather_path()]
 
 
 def status_from_flags(flags: int) -> int:

@@ -86,10 +86,15 @@ typedef enum {
 #define DLRM_FLAG_TIMEOUT 4
 
 /* Gather paths (dlrm_set_gather_path). */
-#define DLRM_PATH_AUTO 0 /* the path measured fastest on B200: register loads */
-#define DLRM_PATH_LDG 1  /* always the register-load (128-bit ld.global.nc) gather */
+#define DLRM_PATH_AUTO 0 /* the path measured fastest on B200: DLRM_PATH_LDG */
+#define DLRM_PATH_LDG 1  /* one block per batch of bags (fused: of samples), register
+                            (128-bit ld.global.nc) loads; serves every call */
 #define DLRM_PATH_TMA 2  /* the TMA tile::gather4 gather for the calls that qualify
-                            (see dlrm_set_gather_path), register loads for the rest */
+                            (see dlrm_set_gather_path), DLRM_PATH_LDG for the rest */
+#define DLRM_PATH_PIPE 3 /* persistent register-load units that prefetch the next bag's
+                            ids and bounds; rows of whole 16-byte chunks (f32: D % 4 == 0,
+                            D <= 256; bf16: D % 8 == 0, D <= 512) and 16-byte aligned
+                            tables and outputs, DLRM_PATH_LDG for the rest */
 
 /* Pooling of a bag's rows (torch.nn.EmbeddingBag modes). The pages implement
  * only SUM and name the others as what a later model would need (movement.rs,
@@ -265,8 +270,8 @@ DLRM_API int dlrm_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_t
 
 /*
  * dlrm_set_gather_path -- which gather serves later gather and fused calls of
- * this process (all threads): DLRM_PATH_AUTO (default), DLRM_PATH_LDG or
- * DLRM_PATH_TMA. Returns the previous setting, or DLRM_ERR_ARG for an unknown
+ * this process (all threads): DLRM_PATH_AUTO (default), DLRM_PATH_LDG,
+ * DLRM_PATH_TMA or DLRM_PATH_PIPE. Returns the previous setting, or DLRM_ERR_ARG for an unknown
  * value. Both paths give bit-identical pooled results; the choice exists for
  * testing and tuning.
  *
@@ -280,7 +285,7 @@ DLRM_API int dlrm_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_t
  */
 DLRM_API int dlrm_set_gather_path(int path);
 
-/* The path (DLRM_PATH_LDG or DLRM_PATH_TMA) that served the calling thread's
+/* The path (DLRM_PATH_LDG, _TMA or _PIPE) that served the calling thread's
  * last gather or fused launch; 0 before the first one. */
 DLRM_API int dlrm_last_gather_path(void);
 

@@ -62,6 +62,7 @@ def test_status_strings_and_flags(ops):
     assert lib.dlrm_status_from_flags(4) == -9
     assert lib.dlrm_set_gather_path(7) == -8
     assert lib.dlrm_set_gather_path(1) == 0 and lib.dlrm_set_gather_path(0) == 1
+    assert lib.dlrm_set_gather_path(3) == 0 and lib.dlrm_set_gather_path(0) == 3
     assert lib.dlrm_launch_count() == 0
 
 

@@ -28,10 +28,11 @@ def ops():
     return _ops
 
 
-@pytest.fixture(params=["tma", "ldg"], autouse=True)
+@pytest.fixture(params=["pipe", "tma", "ldg"], autouse=True)
 def gather_path(request, ops):
-    """Every test runs on the TMA gather path (where the call qualifies; the
-    register-load path serves the rest) and on the register-load path."""
+    """Every test runs on the pipelined path and on the TMA gather path (each
+    where the call qualifies; the per-block register loads serve the rest) and
+    on the per-block register-load path."""
     prev = ops.set_gather_path(request.param)
     yield request.param
     ops.set_gather_path(prev)
@@ -430,7 +431,9 @@ def test_host_pipeline_overlapped_batches(ops):
 
 
 def test_path_choice(ops):
-    """Under "tma" qualifying calls run the TMA gather, the others register loads."""
+    """Under "tma" qualifying calls run the TMA gather, under "pipe" calls with
+    16-byte row chunks in one column window run the pipelined kernels, and all
+    other calls (every call under "auto") the per-block register loads."""
     prev = ops.set_gather_path("tma")
     try:
         for (B, F, N, D, L) in [(70, 5, 300, 64, 16), (33, 26, 200, 128, 20), (19, 2, 50, 16, 4),
@@ -443,6 +446,18 @@ def test_path_choice(ops):
         weights, idx, off, dense = _random_case(3, 8, 2, 20, 6, 3)  # 24-byte rows
         ops.embbag_sum_multi(weights, _dev_i32(idx), _dev_i32(off), 3)
         assert ops.last_gather_path() == "ldg"
+        for name, want in (("pipe", "pipe"), ("auto", "ldg")):
+            ops.set_gather_path(name)
+            for D in (16, 64, 128, 256):
+                weights, idx, off, dense = _random_case(D, 5, 3, 40, D, 4)
+                ops.embbag_sum_multi(weights, _dev_i32(idx), _dev_i32(off), 4)
+                assert ops.last_gather_path() == want
+                ops.sparse_interact(weights, _dev_i32(idx), _dev_i32(off), dense, 4)
+                assert ops.last_gather_path() == want
+            for D in (6, 512):  # 24-byte rows; two column windows
+                weights, idx, off, dense = _random_case(D, 5, 3, 40, D, 4)
+                ops.embbag_sum_multi(weights, _dev_i32(idx), _dev_i32(off), 4)
+                assert ops.last_gather_path() == "ldg"
         ops.set_gather_path("ldg")
         weights, idx, off, dense = _random_case(4, 8, 2, 20, 64, 3)
         ops.sparse_interact(weights, _dev_i32(idx), _dev_i32(off), dense, 3)

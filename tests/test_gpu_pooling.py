@@ -28,10 +28,11 @@ def ops():
     return _ops
 
 
-@pytest.fixture(params=["tma", "ldg"], autouse=True)
+@pytest.fixture(params=["pipe", "tma", "ldg"], autouse=True)
 def gather_path(request, ops):
-    """Every test runs on the TMA gather path (where the call qualifies; the
-    register-load path serves the rest) and on the register-load path."""
+    """Every test runs on the pipelined path and on the TMA gather path (each
+    where the call qualifies; the per-block register loads serve the rest) and
+    on the per-block register-load path."""
     prev = ops.set_gather_path(request.param)
     yield request.param
     ops.set_gather_path(prev)
