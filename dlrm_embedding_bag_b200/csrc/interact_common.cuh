@@ -53,21 +53,58 @@ __device__ __forceinline__ void zero_feature_padding(float* feat, const FeatLayo
   }
 }
 
+// Reduce-scatter of one 4x4 tile of partial dots over the Q = 2^LQ lanes of
+// a task, then the stores. Tile value v = 4r + c is the dot of rows 4I+r and
+// 4J+c. Each xor round halves what a lane holds: the lane whose mask bit is
+// clear keeps the lower half of its values and receives its partner's lower
+// half, the other keeps and receives the upper half. After LQ rounds lane q
+// holds the fully summed values v = q*(16/Q) .. q*(16/Q) + 16/Q - 1, and
+// stores the ones strictly below the diagonal and inside F+1.
+template <int LQ>
+__device__ __forceinline__ void tile_reduce_store(float (&acc)[16], int q, bool active, int I,
+                                                  int J, int F1, float* __restrict__ orow) {
+  constexpr int Q = 1 << LQ;
+  constexpr int NV = 16 >> LQ;
+#pragma unroll
+  for (int round = 0; round < LQ; ++round) {
+    const int m = Q >> (round + 1);
+    const int half = 8 >> round;
+    const bool upper = (q & m) != 0;
+#pragma unroll
+    for (int k = 0; k < half; ++k) {
+      const float lo = acc[k], hi = acc[k + half];
+      const float send = upper ? lo : hi;
+      const float keep = upper ? hi : lo;
+      acc[k] = keep + __shfl_xor_sync(kFullMask, send, m);
+    }
+  }
+  if (!active) return;
+#pragma unroll
+  for (int k = 0; k < NV; ++k) {
+    const int v = q * NV + k;
+    const int i = 4 * I + (v >> 2);
+    const int j = 4 * J + (v & 3);
+    if (i < F1 && j < i) orow[i * (i - 1) / 2 + j] = acc[k];
+  }
+}
+
 // All strict-lower-triangle dots of the block's samples, from shared memory.
 //
 // The pairs are covered by 4x4 tiles (I, J), I >= J, of the (F+1) x (F+1)
 // Gram matrix; the flat tile index t is decoded with the same closed form as
 // the pair index (tile (I, J) is pair (I+1, J) of a triangle one larger). A
-// task is (sample, tile, q): Q = 2^lq consecutive lanes split the D columns
-// of one tile (lane q takes float4 chunks q, q+Q, ...), keep the 16 partial
-// dots in registers (each float4 read from shared memory feeds 16 FMAs), and
-// combine them with xor shuffles. Lane q then stores the tile entries
-// e = 4r + c with e % Q == q that lie strictly below the diagonal and inside
-// F+1.
+// task is (sample, tile, q): Q = 2^lq consecutive lanes (lq <= 4) split the D
+// columns of one tile (lane q takes float4 chunks q, q+Q, ...) and keep the 16
+// partial dots in registers, so each float4 read from shared memory feeds 16
+// FMAs; tile_reduce_store combines and stores them.
 //
 // The output row of sample b starts at out + b * row_stride + col0; dot p of
 // the row is written at offset p. Run by the `nthreads` threads tid = 0 ..
-// nthreads-1 (a multiple of 32, whole warps).
+// nthreads-1 (a multiple of 32, whole warps). UNROLL iterations of the column
+// loop are unrolled (more loads in flight, more registers). DP > 0 fixes the
+// row length Lf.Dp at compile time, so every shared-memory read of a tile
+// step is an immediate offset from one of two base addresses.
+template <int UNROLL = 1, int DP = 0>
 __device__ __forceinline__ void dots_from_smem(const float* feat, const FeatLayout& Lf,
                                                int S_here, int lq, float* __restrict__ out,
                                                int64_t b0, int64_t row_stride, int64_t col0,
@@ -75,6 +112,7 @@ __device__ __forceinline__ void dots_from_smem(const float* feat, const FeatLayo
   const int Q = 1 << lq;
   const int total = (S_here * Lf.nT) << lq;
   const int lane = tid & 31;
+  const int rstride = DP > 0 ? (DP >> 2) : (Lf.Dp >> 2);  // float4 per feature row
   for (int base = tid - lane; base < total; base += nthreads) {
     const int task = base + lane;
     const bool active = task < total;
@@ -89,53 +127,68 @@ __device__ __forceinline__ void dots_from_smem(const float* feat, const FeatLayo
     int I1, J;
     pair_from_flat_small(t, I1, J);
     const int I = I1 - 1;
-    const float* fi = feat + (static_cast<int64_t>(s) * Lf.F1p + 4 * I) * Lf.Dp;
-    const float* fj = feat + (static_cast<int64_t>(s) * Lf.F1p + 4 * J) * Lf.Dp;
+    const float4* fi = reinterpret_cast<const float4*>(feat) +
+                       (static_cast<int64_t>(s) * Lf.F1p + 4 * I) * rstride + q;
+    const float4* fj = reinterpret_cast<const float4*>(feat) +
+                       (static_cast<int64_t>(s) * Lf.F1p + 4 * J) * rstride + q;
 
-    float acc[4][4];
+    float acc[16];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
+    for (int v = 0; v < 16; ++v) acc[v] = 0.f;
 
+#pragma unroll UNROLL
     for (int d4 = q; d4 < Lf.D4; d4 += Q) {
       float4 a[4], bv[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) a[r] = *reinterpret_cast<const float4*>(fi + r * Lf.Dp + 4 * d4);
+      for (int r = 0; r < 4; ++r) a[r] = fi[r * rstride];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) bv[c] = *reinterpret_cast<const float4*>(fj + c * Lf.Dp + 4 * d4);
+      for (int c = 0; c < 4; ++c) bv[c] = fj[c * rstride];
+      fi += Q;
+      fj += Q;
 #pragma unroll
       for (int r = 0; r < 4; ++r)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          float x = acc[r][c];
+          float x = acc[4 * r + c];
           x = fmaf(a[r].x, bv[c].x, x);
           x = fmaf(a[r].y, bv[c].y, x);
           x = fmaf(a[r].z, bv[c].z, x);
           x = fmaf(a[r].w, bv[c].w, x);
-          acc[r][c] = x;
+          acc[4 * r + c] = x;
         }
     }
-    for (int off = 1; off < Q; off <<= 1) {
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] += __shfl_xor_sync(kFullMask, acc[r][c], off);
-    }
-    if (active) {
-      float* orow = out + (b0 + s) * row_stride + col0;
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int i = 4 * I + r;
-        if (i >= Lf.F1) continue;
-        float* orow_i = orow + i * (i - 1) / 2 + 4 * J;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (((4 * r + c) & (Q - 1)) == q && 4 * J + c < i) orow_i[c] = acc[r][c];
-        }
-      }
+    float* orow = out + (b0 + s) * row_stride + col0;
+    switch (lq) {
+      case 0: tile_reduce_store<0>(acc, q, active, I, J, Lf.F1, orow); break;
+      case 1: tile_reduce_store<1>(acc, q, active, I, J, Lf.F1, orow); break;
+      case 2: tile_reduce_store<2>(acc, q, active, I, J, Lf.F1, orow); break;
+      case 3: tile_reduce_store<3>(acc, q, active, I, J, Lf.F1, orow); break;
+      default: tile_reduce_store<4>(acc, q, active, I, J, Lf.F1, orow); break;
     }
   }
+}
+
+// Ampere-style asynchronous global -> shared copies (cp.async), used to stage
+// the next group of samples while the current one is computed.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's committed groups are still pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 }  // namespace dlrm

@@ -17,37 +17,87 @@ namespace dlrm {
 
 static std::atomic<int64_t> g_launches{0};
 
-// Interaction alone: each block stages S samples' [dense, emb] rows in shared
-// memory with coalesced loads, then runs the tiled dot phase.
+// Interaction alone. Persistent blocks walk groups of S samples (group g =
+// blockIdx.x + i * gridDim.x); while the dots of one group run from one shared
+// buffer, the [dense, emb] rows of the next group are copied into the other
+// with cp.async. Warp w copies feature rows w, w + 8, ...; when a row is at
+// most 32 chunks of VEC floats and the chunk count divides 32, one warp copy
+// covers 32/DV rows.
 template <int VEC>
-__global__ void __launch_bounds__(kBlockThreads)
-    interact_kernel(const float* __restrict__ dense, const float* __restrict__ emb, int B, int F,
-                    int D, int S, int lq, float* __restrict__ out) {
-  extern __shared__ __align__(16) float feat[];
-  const FeatLayout Lf = FeatLayout::make(F, D);
-  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * S;
-  const int S_here = (B - b0 < S) ? static_cast<int>(B - b0) : S;
+__device__ __forceinline__ void stage_interact_group(float* buf, const FeatLayout& Lf,
+                                                     const float* __restrict__ dense,
+                                                     const float* __restrict__ emb, int64_t b0,
+                                                     int S_here, int F, int D) {
   const int DV = D / VEC;
-  const int per_sample = Lf.F1 * DV;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int nwarps = kBlockThreads / 32;
+  const bool packed = DV <= 32 && (32 % DV) == 0;
+  const int rpw = packed ? 32 / DV : 1;              // rows per warp copy
+  const int lr = packed ? lane / DV : 0;             // this lane's row within the copy
+  const int c0 = packed ? (lane - lr * DV) : lane;  // this lane's first chunk
+  const int cstep = packed ? DV : 32;
   for (int s = 0; s < S_here; ++s) {
-    float* base = feat + s * Lf.floats_per_sample();
-    for (int e = threadIdx.x; e < per_sample; e += blockDim.x) {
-      const int f = e / DV;
-      const int c = (e - f * DV) * VEC;
-      const float* src = (f == 0) ? dense + (b0 + s) * D + c
-                                  : emb + ((b0 + s) * F + (f - 1)) * static_cast<int64_t>(D) + c;
-      if constexpr (VEC == 4) {
-        *reinterpret_cast<float4*>(base + f * Lf.Dp + c) =
-            __ldg(reinterpret_cast<const float4*>(src));
-      } else {
-        base[f * Lf.Dp + c] = __ldg(src);
+    float* base = buf + s * Lf.floats_per_sample();
+    const int64_t b = b0 + s;
+    for (int f = warp * rpw + lr; f < Lf.F1; f += nwarps * rpw) {
+      const float* src =
+          (f == 0) ? dense + b * D : emb + (b * F + (f - 1)) * static_cast<int64_t>(D);
+      float* dst = base + f * Lf.Dp;
+      for (int c = c0; c < DV; c += cstep) {
+        if constexpr (VEC == 4) {
+          cp_async16(dst + 4 * c, src + 4 * c);
+        } else {
+          cp_async4(dst + c, src + c);
+        }
       }
     }
   }
-  zero_feature_padding(feat, Lf, D, S_here, threadIdx.x, blockDim.x);
-  __syncthreads();
+}
+
+template <int VEC, int DP>
+__global__ void __launch_bounds__(kBlockThreads, 2)
+    interact_kernel(const float* __restrict__ dense, const float* __restrict__ emb, int B, int F,
+                    int D, int S, int lq, int nbuf, float* __restrict__ out) {
+  extern __shared__ __align__(16) float feat[];
+  const FeatLayout Lf = FeatLayout::make(F, D);
+  const int64_t bstride = (nbuf > 1) ? S * Lf.floats_per_sample() : 0;  // buffer i at feat + i*bstride
+  const int64_t ngroups = (static_cast<int64_t>(B) + S - 1) / S;
   const int P = Lf.F1 * (Lf.F1 - 1) / 2;
-  dots_from_smem(feat, Lf, S_here, lq, out, b0, P, 0, threadIdx.x, blockDim.x);
+  auto samples = [&](int64_t g) {
+    const int64_t rem = B - g * S;
+    return rem < S ? static_cast<int>(rem) : S;
+  };
+  // The copies never write the padding, so it is zeroed once per buffer.
+  for (int i = 0; i < nbuf; ++i)
+    zero_feature_padding(feat + i * bstride, Lf, D, S, threadIdx.x, blockDim.x);
+  int64_t g = blockIdx.x;
+  if (nbuf == 1) {
+    for (; g < ngroups; g += gridDim.x) {
+      stage_interact_group<VEC>(feat, Lf, dense, emb, g * S, samples(g), F, D);
+      cp_async_commit();
+      cp_async_wait<0>();
+      __syncthreads();
+      dots_from_smem<2, DP>(feat, Lf, samples(g), lq, out, g * S, P, 0, threadIdx.x,
+                            blockDim.x);
+      __syncthreads();
+    }
+    return;
+  }
+  if (g < ngroups) stage_interact_group<VEC>(feat, Lf, dense, emb, g * S, samples(g), F, D);
+  cp_async_commit();
+  for (int it = 0; g < ngroups; ++it, g += gridDim.x) {
+    const int64_t gn = g + gridDim.x;
+    if (gn < ngroups)
+      stage_interact_group<VEC>(feat + ((it + 1) & 1) * bstride, Lf, dense, emb, gn * S,
+                                samples(gn), F, D);
+    cp_async_commit();
+    cp_async_wait<1>();  // group g has landed (only the copy of group gn may be pending)
+    __syncthreads();
+    dots_from_smem<2, DP>(feat + (it & 1) * bstride, Lf, samples(g), lq, out, g * S, P, 0,
+                          threadIdx.x, blockDim.x);
+    __syncthreads();  // buffer it&1 is refilled in the next iteration
+  }
+  cp_async_wait<0>();
 }
 
 __global__ void pair_decode_kernel(int64_t p0, int64_t count, int32_t* __restrict__ i_out,
@@ -109,7 +159,7 @@ static void choose_dot_shape(int F, int D, int B, int samples_wanted, int64_t sm
   S = std::min(s, B);
   const int tiles = S * Lf.nT;
   const int qmax = std::max(1, kBlockThreads / tiles);
-  lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), 5});
+  lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), 4});
 }
 
 static cudaError_t counted(cudaError_t e) {
@@ -252,7 +302,7 @@ cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_
     while (t.S > 1 && TmaSmem::make(t.G, g.D * g.esz, 2 * t.S * per).total > smem_limit) --t.S;
     tma_ok = TmaSmem::make(t.G, g.D * g.esz, 2 * t.S * per).total <= smem_limit;
     const int qmax = std::max(1, kTmaDotWarps * 32 / (t.S * Lf.nT));
-    t.lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), 5});
+    t.lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), 4});
   }
   if (tma_ok && path == DLRM_PATH_TMA) {
     t_last_path = DLRM_PATH_TMA;
@@ -287,7 +337,7 @@ cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_
     if (a.smem <= smem_limit) {
       t_last_path = DLRM_PATH_PIPE;
       const int qmax = std::max(1, kPipeDotWarps * 32 / (a.S * Lf.nT));
-      a.lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), 5});
+      a.lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), 4});
       a.tp = g.tp;
       a.bp = g.bp;
       a.B = g.B;
@@ -328,31 +378,64 @@ cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_
   }
 }
 
-cudaError_t launch_interact(const float* dense, const float* emb, int B, int F, int D, float* out,
-                            bool vec_ok, int64_t smem_limit, cudaStream_t stream) {
+// Samples per group S and lanes per tile 2^lq for the interaction kernel.
+// Measured on B200 (B=2048, F=32, D=64 and B=65536, F=26, D=128), four lanes
+// per tile beat one or two (shorter serial chains per thread), and the best
+// group is the largest that still gives one task per thread: S*nT*4 <= 256.
+// S is further capped by the shared-memory budget of two buffers.
+static void choose_interact_shape(int F, int D, int B, int64_t smem_budget, int& S, int& lq) {
   const FeatLayout Lf = FeatLayout::make(F, D);
-  // enough samples that the staging loop and the dot phase keep 256 threads busy
-  const int want = std::max(1, kBlockThreads / std::max(1, Lf.nT * std::min(Lf.D4, 4)));
+  const int64_t per = Lf.floats_per_sample() * 4;
+  lq = std::min(2, log2_floor(std::max(1, Lf.D4)));
+  S = std::max(1, kBlockThreads / std::max(1, Lf.nT << lq));
+  while (S > 1 && 2 * S * per > smem_budget) --S;
+  S = std::max(1, std::min(S, B));
+}
+
+template <int VEC, int DP>
+static cudaError_t run_interact(const float* dense, const float* emb, int B, int F, int D,
+                                float* out, int64_t smem_limit, int sms, cudaStream_t stream) {
+  const FeatLayout Lf = FeatLayout::make(F, D);
+  const int64_t per = Lf.floats_per_sample() * 4;
+  if (per > smem_limit) return cudaErrorInvalidValue;
+  auto* fn = &interact_kernel<VEC, DP>;
+  const int64_t budget = std::min<int64_t>(smem_limit, 100 * 1024);  // two blocks per SM
   int S, lq;
-  choose_dot_shape(F, D, B, std::min(want, 8), std::min<int64_t>(smem_limit, 64 * 1024), S, lq);
-  const int64_t smem = S * Lf.floats_per_sample() * 4;
-  if (smem > smem_limit) return cudaErrorInvalidValue;
-  const int64_t grid = (static_cast<int64_t>(B) + S - 1) / S;
-  const void* fn = vec_ok ? reinterpret_cast<const void*>(&interact_kernel<4>)
-                          : reinterpret_cast<const void*>(&interact_kernel<1>);
+  choose_interact_shape(F, D, B, budget, S, lq);
+  const int nbuf = (2 * S * per <= smem_limit) ? 2 : 1;
+  const int64_t smem = nbuf * S * per;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  if (vec_ok) {
-    interact_kernel<4><<<static_cast<unsigned>(grid), kBlockThreads, smem, stream>>>(
-        dense, emb, B, F, D, S, lq, out);
+  int per_sm = 0;
+  cudaError_t e =
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kBlockThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const int64_t ngroups = (static_cast<int64_t>(B) + S - 1) / S;
+  const int64_t grid = std::min<int64_t>(ngroups, static_cast<int64_t>(per_sm) * sms);
+  fn<<<static_cast<unsigned>(grid), kBlockThreads, smem, stream>>>(dense, emb, B, F, D, S, lq,
+                                                                  nbuf, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_interact(const float* dense, const float* emb, int B, int F, int D, float* out,
+                            bool vec_ok, int64_t smem_limit, cudaStream_t stream) {
+  const int sms = sm_count();
+  cudaError_t e;
+  if (vec_ok && D == 64) {
+    e = run_interact<4, 68>(dense, emb, B, F, D, out, smem_limit, sms, stream);
+  } else if (vec_ok && D == 128) {
+    e = run_interact<4, 132>(dense, emb, B, F, D, out, smem_limit, sms, stream);
+  } else if (vec_ok) {
+    e = run_interact<4, 0>(dense, emb, B, F, D, out, smem_limit, sms, stream);
   } else {
-    interact_kernel<1><<<static_cast<unsigned>(grid), kBlockThreads, smem, stream>>>(
-        dense, emb, B, F, D, S, lq, out);
+    e = run_interact<1, 0>(dense, emb, B, F, D, out, smem_limit, sms, stream);
   }
-  return counted(cudaGetLastError());
+  return counted(e);
 }
 
 cudaError_t launch_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_t* j_out,
