@@ -30,7 +30,7 @@ from __future__ import annotations
 import ctypes
 import os
 import subprocess
-from typing import Sequence
+from typing import Optional, Sequence
 
 import numpy as np
 
@@ -97,6 +97,10 @@ class Oracle:
         lib.oracle_embbag_pool_multi.restype = I
         lib.oracle_pair_list.argtypes = [I, P, P]
         lib.oracle_pair_list.restype = ctypes.c_int64
+        L64 = ctypes.c_int64
+        lib.oracle_linear_bf16.argtypes = [P, L64, L64, P, L64, L64, P, L64, P, L64, L64, I, P, P,
+                                           P]
+        lib.oracle_linear_bf16.restype = I
         self.lib = lib
         self.path = libpath
 
@@ -199,6 +203,41 @@ class Oracle:
             raise OracleError(-1, "pair_list")
         return pi, pj
 
+    def linear_bf16(self, a_lo: np.ndarray, w: np.ndarray, bias=None, act: int = 0, *,
+                    a_hi: Optional[np.ndarray] = None, k_lo: Optional[int] = None,
+                    k_hi: Optional[int] = None, k: Optional[int] = None):
+        """One MLP layer ``act(A W^T + bias)`` over bf16 operands, exactly (fp64).
+
+        ``a_lo`` ``(M, >=k_lo)``, ``a_hi`` ``(M, >=k_hi)`` (optional) and ``w``
+        ``(N, >=k_lo+k_hi)`` are uint16 arrays of bf16 bit patterns (row pitch =
+        their second dimension); ``bias`` is ``(N,)`` f32 or None; ``act`` is 0
+        (none), 1 (ReLU) or 2 (sigmoid). ``k_lo``/``k_hi`` default to the
+        widths of ``a_lo``/``a_hi``. Returns ``(out, pre, bound)``, each
+        ``(M, N)`` fp64: the activation, the pre-activation and
+        ``sum_k |a_k w_k| + |bias|``.
+        """
+        a_lo = np.ascontiguousarray(a_lo, dtype=np.uint16)
+        w = np.ascontiguousarray(w, dtype=np.uint16)
+        M, lda_lo = a_lo.shape
+        N, ldw = w.shape
+        k_lo = lda_lo if k_lo is None else k_lo
+        if a_hi is not None:
+            a_hi = np.ascontiguousarray(a_hi, dtype=np.uint16)
+            lda_hi = a_hi.shape[1]
+            k_hi = lda_hi if k_hi is None else k_hi
+        else:
+            lda_hi, k_hi = 0, 0
+        b = None if bias is None else _f32(bias)
+        out = np.empty((M, N), dtype=np.float64)
+        pre = np.empty((M, N), dtype=np.float64)
+        bnd = np.empty((M, N), dtype=np.float64)
+        rc = self.lib.oracle_linear_bf16(_ptr(a_lo), lda_lo, k_lo, _ptr(a_hi), lda_hi, k_hi,
+                                         _ptr(w), ldw, _ptr(b), M, N, act, _ptr(out), _ptr(pre),
+                                         _ptr(bnd))
+        if rc != OK:
+            raise OracleError(rc, "linear_bf16")
+        return out, pre, bnd
+
 
 _default = None
 
@@ -229,3 +268,7 @@ def pair_list(*a, **k):
 
 def embbag_pool_multi(*a, **k):
     return default().embbag_pool_multi(*a, **k)
+
+
+def linear_bf16(*a, **k):
+    return default().linear_bf16(*a, **k)

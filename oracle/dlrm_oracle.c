@@ -330,3 +330,65 @@ int oracle_sparse_interact(const float* const* weights, const int64_t* rows,
     return oracle_interact_lower_tri(dense, pooled_tmp, B, F, D, inter_out, concat_dense,
                                      NULL, bound);
 }
+
+/*
+ * One DLRMv1 MLP layer, y = act(A W^T + bias), the linear-with-bias layer the
+ * pages' matmul2d.rs page describes (linear_bias, linear_bias_relu,
+ * linear_bias_sigmoid): A is (M, K), W is (N, K) (the nn.Linear weight
+ * layout, "transpose_b"), bias is (N,), the activation is applied to
+ * acc + bias. The split form of the same page (linear_bias_split_a and its
+ * ReLU/Sigmoid variants) reads columns 0..k_lo-1 of A from a_lo and columns
+ * k_lo..K-1 from a_hi, without building the concatenation.
+ *
+ * Operands are bf16 bit patterns (the tensor-core path takes bf16 operands;
+ * see the design notes): a value is the f32 whose upper 16 bits are the
+ * pattern. Every product of two such values is exact in fp64 and the sum is
+ * taken in fp64 in ascending k, so out holds the exact layer up to fp64
+ * rounding.
+ *   a_lo  : (M, lda_lo) rows, columns [0, k_lo) used
+ *   a_hi  : (M, lda_hi) rows, columns [0, k_hi) used; NULL when k_hi == 0
+ *   w     : (N, ldw) rows, columns [0, k_lo + k_hi) used
+ *   bias  : (N,) f32, or NULL for no bias
+ *   act   : 0 none, 1 ReLU max(x, 0), 2 sigmoid 1 / (1 + exp(-x))
+ *   out   : (M, N) fp64, the activation of the exact pre-activation
+ *   pre   : nullable (M, N) fp64, the exact pre-activation acc + bias
+ *   bound : nullable (M, N) fp64, sum_k |a_k w_k| + |bias| (error scale)
+ */
+int oracle_linear_bf16(const uint16_t* a_lo, int64_t lda_lo, int64_t k_lo,
+                       const uint16_t* a_hi, int64_t lda_hi, int64_t k_hi,
+                       const uint16_t* w, int64_t ldw, const float* bias,
+                       int64_t M, int64_t N, int act, double* out, double* pre,
+                       double* bound) {
+    if (M < 1 || N < 1 || k_lo < 1 || k_hi < 0 || act < 0 || act > 2) return ORACLE_BAD_ARG;
+    if (!a_lo || !w || !out || (k_hi > 0 && !a_hi)) return ORACLE_BAD_ARG;
+    if (lda_lo < k_lo || (k_hi > 0 && lda_hi < k_hi) || ldw < k_lo + k_hi) return ORACLE_BAD_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            const uint16_t* wn = w + n * ldw;
+            double s = 0.0, mag = 0.0;
+            for (int64_t k = 0; k < k_lo; ++k) {
+                const double t = (double)bf16_bits_to_f32(a_lo[m * lda_lo + k]) *
+                                 (double)bf16_bits_to_f32(wn[k]);
+                s += t;
+                mag += (t < 0.0) ? -t : t;
+            }
+            for (int64_t k = 0; k < k_hi; ++k) {
+                const double t = (double)bf16_bits_to_f32(a_hi[m * lda_hi + k]) *
+                                 (double)bf16_bits_to_f32(wn[k_lo + k]);
+                s += t;
+                mag += (t < 0.0) ? -t : t;
+            }
+            if (bias) {
+                s += (double)bias[n];
+                mag += fabs((double)bias[n]);
+            }
+            double y = s;
+            if (act == 1) y = (s > 0.0) ? s : 0.0;
+            if (act == 2) y = 1.0 / (1.0 + exp(-s));
+            out[m * N + n] = y;
+            if (pre) pre[m * N + n] = s;
+            if (bound) bound[m * N + n] = mag;
+        }
+    }
+    return ORACLE_OK;
+}

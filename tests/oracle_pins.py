@@ -489,6 +489,120 @@ def pin_general_pooling_rejects(orc):
                                                per_sample_weights=np.ones((1, 5))), BAD_ARG)
 
 
+# ---------------------------------------------------------------------------
+# The MLP layer: act(A W^T + bias) over bf16 operands (matmul2d.rs page,
+# linear_bias / _relu / _sigmoid and the split-A forms).
+
+
+def _bf16_bits(x):
+    """bf16 bit patterns of an array (torch's round-to-nearest-even)."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _bf16_values(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def pin_linear_exact_integers(orc):
+    """Small-integer operands: the layer is an exact integer matmul (numpy int64)."""
+    rng = np.random.default_rng(71)
+    for (M, N, K) in [(1, 1, 1), (3, 5, 7), (17, 9, 40)]:
+        a = rng.integers(-8, 9, size=(M, K))
+        w = rng.integers(-8, 9, size=(N, K))
+        b = rng.integers(-50, 51, size=N)
+        out, pre, bound = orc.linear_bf16(_bf16_bits(a), _bf16_bits(w), b.astype(np.float32))
+        want = a.astype(np.int64) @ w.astype(np.int64).T + b
+        assert np.array_equal(pre, want.astype(np.float64))
+        assert np.array_equal(out, want.astype(np.float64))
+        wantb = np.abs(a).astype(np.int64) @ np.abs(w).astype(np.int64).T + np.abs(b)
+        assert np.array_equal(bound, wantb.astype(np.float64))
+
+
+def pin_linear_vs_torch_fp64(orc):
+    """Random bf16 operands against torch.nn.functional.linear in fp64."""
+    rng = np.random.default_rng(72)
+    for (M, N, K) in [(4, 3, 16), (33, 20, 100)]:
+        a = _bf16_bits(rng.normal(0, 1, size=(M, K)))
+        w = _bf16_bits(rng.normal(0, 0.1, size=(N, K)))
+        b = rng.normal(0, 0.1, size=N).astype(np.float32)
+        ta = torch.from_numpy(_bf16_values(a).astype(np.float64))
+        tw = torch.from_numpy(_bf16_values(w).astype(np.float64))
+        tb = torch.from_numpy(b.astype(np.float64))
+        want = torch.nn.functional.linear(ta, tw, tb).numpy()
+        out, _, bound = orc.linear_bf16(a, w, b, 0)
+        assert np.all(np.abs(out - want) <= 1e-12 * bound + 1e-300)
+        out, _, _ = orc.linear_bf16(a, w, None, 0)
+        want0 = torch.nn.functional.linear(ta, tw).numpy()
+        assert np.all(np.abs(out - want0) <= 1e-12 * bound + 1e-300)
+
+
+def pin_linear_activations(orc):
+    """ReLU is torch.relu and sigmoid is scipy's expit of the pre-activation."""
+    from scipy.special import expit
+
+    rng = np.random.default_rng(73)
+    a = _bf16_bits(rng.normal(0, 1, size=(9, 24)))
+    w = _bf16_bits(rng.normal(0, 0.5, size=(7, 24)))
+    b = rng.normal(0, 0.5, size=7).astype(np.float32)
+    _, pre, _ = orc.linear_bf16(a, w, b, 0)
+    relu, pre1, _ = orc.linear_bf16(a, w, b, 1)
+    sig, pre2, _ = orc.linear_bf16(a, w, b, 2)
+    assert np.array_equal(pre, pre1) and np.array_equal(pre, pre2)
+    assert (pre < 0).any() and (pre > 0).any()
+    assert np.array_equal(relu, torch.relu(torch.from_numpy(pre)).numpy())
+    assert np.allclose(sig, expit(pre), rtol=1e-15, atol=0)
+
+
+def pin_linear_split_equals_concat(orc):
+    """Split A (columns from two sources) equals the layer on the concatenation,
+    and the weight's column k_lo + k multiplies a_hi's column k."""
+    rng = np.random.default_rng(74)
+    M, N, k_lo, k_hi = 6, 5, 3, 11
+    a_lo = _bf16_bits(rng.normal(0, 1, size=(M, k_lo)))
+    a_hi = _bf16_bits(rng.normal(0, 1, size=(M, k_hi)))
+    w = _bf16_bits(rng.normal(0, 1, size=(N, k_lo + k_hi)))
+    b = rng.normal(0, 1, size=N).astype(np.float32)
+    cat = np.concatenate([a_lo, a_hi], axis=1)
+    for act in (0, 1, 2):
+        want = orc.linear_bf16(cat, w, b, act)
+        got = orc.linear_bf16(a_lo, w, b, act, a_hi=a_hi)
+        for x, y in zip(want, got):
+            assert np.array_equal(x, y)
+    # one-hot probes: a_hi = e_k picks weight column k_lo + k
+    for k in range(k_hi):
+        e = np.zeros((1, k_hi), np.float32)
+        e[0, k] = 1.0
+        _, pre, _ = orc.linear_bf16(np.zeros((1, k_lo), np.uint16), w, None, 0,
+                                    a_hi=_bf16_bits(e))
+        assert np.array_equal(pre[0], _bf16_values(w[:, k_lo + k]).astype(np.float64))
+
+
+def pin_linear_row_pitch(orc):
+    """Only the first k columns of each pitched row enter the layer."""
+    rng = np.random.default_rng(75)
+    M, N, K, pad = 4, 3, 5, 3
+    a = _bf16_bits(rng.normal(0, 1, size=(M, K)))
+    w = _bf16_bits(rng.normal(0, 1, size=(N, K)))
+    junk = _bf16_bits(np.full((M, pad), 1e30))
+    wjunk = _bf16_bits(np.full((N, pad), -1e30))
+    want = orc.linear_bf16(a, w, None, 0)
+    got = orc.linear_bf16(np.concatenate([a, junk], 1), np.concatenate([w, wjunk], 1), None, 0,
+                          k_lo=K)
+    for x, y in zip(want, got):
+        assert np.array_equal(x, y)
+
+
+def pin_linear_rejects(orc):
+    from oracle import BAD_ARG
+
+    a = np.zeros((2, 4), np.uint16)
+    w = np.zeros((3, 4), np.uint16)
+    _expect_code(lambda: orc.linear_bf16(a, w, None, 3), BAD_ARG)
+    _expect_code(lambda: orc.linear_bf16(a, np.zeros((3, 3), np.uint16), None, 0), BAD_ARG)
+    _expect_code(lambda: orc.linear_bf16(a, w, None, 0, k_lo=5), BAD_ARG)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 

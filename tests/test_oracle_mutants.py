@@ -60,6 +60,15 @@ MUTANTS = {
                               "acc = (x > acc) ? x : acc;")],
     "last_offset_ignored": [("(ilo || b + 1 < B) ? (int64_t)offsets[(int64_t)k * row + b + 1]",
                              "(b + 1 < B) ? (int64_t)offsets[(int64_t)k * row + b + 1]")],
+    "linear_weight_transposed": [("(double)bf16_bits_to_f32(wn[k]);", "(double)bf16_bits_to_f32(w[k * ldw + n]);")],
+    "linear_hi_part_reads_lo_weights": [("(double)bf16_bits_to_f32(wn[k_lo + k]);",
+                                         "(double)bf16_bits_to_f32(wn[k]);")],
+    "linear_bias_subtracted": [("s += (double)bias[n];", "s -= (double)bias[n];")],
+    "linear_relu_after_sigmoid_swapped": [("if (act == 1) y = (s > 0.0) ? s : 0.0;",
+                                           "if (act == 2) y = (s > 0.0) ? s : 0.0;")],
+    "linear_sigmoid_sign": [("y = 1.0 / (1.0 + exp(-s));", "y = 1.0 / (1.0 + exp(s));")],
+    "linear_a_row_pitch_ignored": [("bf16_bits_to_f32(a_lo[m * lda_lo + k])",
+                                    "bf16_bits_to_f32(a_lo[m * k_lo + k])")],
     "general_pooling_table_layout_transposed": [
         ("out[((int64_t)b * F + k) * D + d] = acc;", "out[((int64_t)k * B + b) * D + d] = acc;")],
 }
