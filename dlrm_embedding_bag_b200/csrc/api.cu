@@ -8,7 +8,7 @@
 #include "dlrm_sparse.h"
 #include "launch.h"
 
-namespace {
+namespace dlrm {
 
 thread_local int t_last_cuda_error = 0;
 
@@ -16,6 +16,13 @@ int cuda_fail(cudaError_t e) {
   t_last_cuda_error = static_cast<int>(e);
   return DLRM_ERR_CUDA;
 }
+
+}  // namespace dlrm
+
+namespace {
+
+using dlrm::cuda_fail;
+using dlrm::t_last_cuda_error;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

@@ -176,13 +176,8 @@ int gather_path() { return g_path.load(std::memory_order_relaxed); }
 void set_gather_path(int path) { g_path.store(path, std::memory_order_relaxed); }
 int last_path() { return t_last_path; }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
 // The driver's tensor-map encoder, looked up once through the runtime.
-static EncodeTiledFn encode_tiled() {
+EncodeTiledFn encode_tiled() {
   static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -448,5 +443,6 @@ cudaError_t launch_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_
 }
 
 int64_t launch_count() { return g_launches.load(std::memory_order_relaxed); }
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 }  // namespace dlrm

@@ -39,6 +39,17 @@ struct FusedLaunch {
   int64_t smem;
 };
 
+// cuTensorMapEncodeTiled, looked up once through the runtime's driver entry
+// point (null if the driver does not provide it).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled();
+
+// Records a failed CUDA call for dlrm_last_cuda_error() and returns DLRM_ERR_CUDA.
+int cuda_fail(cudaError_t e);
+
 // Tensor maps of the TMA gather path: one 2-D map per table ({D, rows},
 // box {D, 1}), passed by value in the kernel's parameter block.
 constexpr int kTmaMaxTables = 64;
@@ -139,5 +150,7 @@ cudaError_t launch_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_
                                cudaStream_t stream);
 
 int64_t launch_count();
+// Counts one kernel launch of this library (dlrm_launch_count).
+void note_launch();
 
 }  // namespace dlrm

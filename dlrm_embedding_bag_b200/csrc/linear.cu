@@ -1,0 +1,358 @@
+// DLRMv1 MLP layer on the sm_100a tensor cores: Y = act([A_lo | A_hi] W^T + bias)
+// (luminal compare main...vanilla-pytorch, matmul2d.rs: linear_bias,
+// linear_bias_relu, linear_bias_sigmoid and the split-A forms), plus the f32 ->
+// bf16 conversion that feeds it. Declared in dlrm_mlp.h.
+//
+// One CTA of 128 threads computes a 128 x BN tile of Y:
+//   - thread 0 streams 64-wide K blocks of A (128 x 64 bf16) and W (BN x 64)
+//     into a 4-stage shared-memory ring with 2-D TMA loads (128-byte swizzle);
+//     K blocks 0..nkb_lo-1 read A_lo, the rest read A_hi, and W's column
+//     offset follows, so the concatenation is never built;
+//   - thread 32 waits for each stage and issues four tcgen05.mma (K = 16 each)
+//     that accumulate the tile in f32 in tensor memory, then commits the
+//     stage back to the producer through an mbarrier;
+//   - after the last MMA all four warps read their 32 accumulator rows with
+//     tcgen05.ld, add the bias, apply the activation and store f32 and/or bf16.
+// Every wait on an mbarrier is bounded; a wait that runs out sets
+// DLRM_FLAG_TIMEOUT in the optional status word and the CTA still frees its
+// tensor memory and exits.
+#include <algorithm>
+#include <climits>
+#include <cstdint>
+
+#include <cuda_bf16.h>
+
+#include "dlrm_mlp.h"
+#include "launch.h"
+#include "tcgen05_common.cuh"
+
+namespace dlrm {
+namespace {
+
+constexpr int kLinBM = 128;    // rows of a tile (tcgen05 M)
+constexpr int kLinBK = 64;     // K per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int kLinStages = 4;  // shared-memory ring depth
+constexpr int kLinThreads = 128;
+constexpr long long kLinWaitLimit = 200000000LL;  // clock cycles, about 0.1 s
+
+template <int BN>
+struct LinSmem {
+  static constexpr int kA = kLinBM * kLinBK * 2;
+  static constexpr int kB = BN * kLinBK * 2;
+  static constexpr int kStage = kA + kB;
+  static constexpr int kBars = kLinStages * kStage;  // full[S], empty[S], done, tmem slot
+  static constexpr int kTotal = kBars + (2 * kLinStages + 1) * 8 + 8 + 1024;  // + alignment
+};
+
+struct LinearArgs {
+  const float* bias;
+  float* y_f32;
+  uint16_t* y_bf16;
+  int64_t ldy_f32, ldy_bf16;
+  int M, N, k_lo, nkb_lo, nkb_hi;
+  int32_t* status;
+};
+
+template <int ACT>
+__device__ __forceinline__ float activate(float x) {
+  if constexpr (ACT == DLRM_ACT_RELU) {
+    return x > 0.f ? x : 0.f;
+  } else if constexpr (ACT == DLRM_ACT_SIGMOID) {
+    return __fdiv_rn(1.f, __fadd_rn(1.f, expf(-x)));
+  } else {
+    return x;
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
+         (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
+}
+
+template <int BN, int ACT>
+__global__ void __launch_bounds__(kLinThreads, 1)
+    linear_bf16_kernel(const __grid_constant__ CUtensorMap map_a_lo,
+                       const __grid_constant__ CUtensorMap map_a_hi,
+                       const __grid_constant__ CUtensorMap map_w, const LinearArgs args) {
+  using L = LinSmem<BN>;
+  constexpr uint32_t kCols = BN < 32 ? 32 : BN;  // TMEM columns: f32 accumulator
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // 1024-byte aligned tiles
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint64_t* empty = full + kLinStages;
+  uint64_t* done = empty + kLinStages;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (warp == 0) {
+    tmem_alloc(tslot, kCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < kLinStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    mbar_init_fence();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tslot;
+
+  const int m0 = blockIdx.x * kLinBM, n0 = blockIdx.y * BN;
+  const int nkb = args.nkb_lo + args.nkb_hi;
+  bool timed_out = false;
+  if (threadIdx.x == 0) {
+    // TMA producer.
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % kLinStages;
+      if (kb >= kLinStages &&
+          !mbar_wait_bounded(&empty[s], ((kb / kLinStages) - 1) & 1, kLinWaitLimit)) {
+        timed_out = true;
+        break;
+      }
+      uint8_t* sa = smem + s * L::kStage;
+      uint8_t* sb = sa + L::kA;
+      mbar_arrive_expect_tx(&full[s], L::kStage);
+      if (kb < args.nkb_lo) {
+        tma_load_2d(sa, &map_a_lo, &full[s], kb * kLinBK, m0);
+        tma_load_2d(sb, &map_w, &full[s], kb * kLinBK, n0);
+      } else {
+        const int kh = kb - args.nkb_lo;
+        tma_load_2d(sa, &map_a_hi, &full[s], kh * kLinBK, m0);
+        tma_load_2d(sb, &map_w, &full[s], args.k_lo + kh * kLinBK, n0);
+      }
+    }
+  } else if (threadIdx.x == 32) {
+    // MMA issuer.
+    constexpr uint32_t idesc = idesc_bf16_f32(kLinBM, BN);
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % kLinStages;
+      if (!mbar_wait_bounded(&full[s], (kb / kLinStages) & 1, kLinWaitLimit)) {
+        timed_out = true;
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t sa = smem_u32(smem + s * L::kStage);
+      const uint32_t sb = sa + L::kA;
+#pragma unroll
+      for (int kk = 0; kk < kLinBK / 16; ++kk)
+        tc_mma_bf16(tmem, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32), idesc,
+                    (kb | kk) != 0 ? 1u : 0u);
+      tc_commit(&empty[s]);  // the stage is free once these MMAs have read it
+    }
+    tc_commit(done);
+  }
+  __syncwarp();
+
+  // Epilogue: warp w owns accumulator rows 32w .. 32w+31 (TMEM lanes).
+  const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(done, 0, kLinWaitLimit) ? 1 : 0);
+  tc_fence_after_sync();
+  const int row = m0 + warp * 32 + lane;
+  const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  const bool f32_vec = args.y_f32 != nullptr && (args.ldy_f32 % 4) == 0 &&
+                       (reinterpret_cast<uintptr_t>(args.y_f32) % 16) == 0;
+  const bool bf_vec = args.y_bf16 != nullptr && (args.ldy_bf16 % 8) == 0 &&
+                      (reinterpret_cast<uintptr_t>(args.y_bf16) % 16) == 0;
+  if (ok) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN && n0 + c0 < args.N; c0 += 16) {
+      float v[16];
+      tmem_ld_32x32b_x16(trow + c0, v);
+      const int nb = n0 + c0;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float b = (args.bias != nullptr && nb + j < args.N) ? __ldg(args.bias + nb + j) : 0.f;
+        v[j] = activate<ACT>(__fadd_rn(v[j], b));
+      }
+      if (row >= args.M) continue;
+      const bool whole = nb + 16 <= args.N;
+      if (args.y_f32 != nullptr) {
+        float* y = args.y_f32 + static_cast<int64_t>(row) * args.ldy_f32 + nb;
+        if (whole && f32_vec) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            reinterpret_cast<float4*>(y)[q] =
+                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (nb + j < args.N) y[j] = v[j];
+        }
+      }
+      if (args.y_bf16 != nullptr) {
+        uint16_t* y = args.y_bf16 + static_cast<int64_t>(row) * args.ldy_bf16 + nb;
+        if (whole && bf_vec) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+            reinterpret_cast<uint4*>(y)[q] =
+                make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                           pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                           pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (nb + j < args.N) y[j] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
+        }
+      }
+    }
+  }
+  if ((timed_out || !ok) && args.status != nullptr) atomicOr(args.status, DLRM_FLAG_TIMEOUT);
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kCols);
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ x, int64_t ldx, int64_t rows,
+                                   int64_t cols, uint16_t* __restrict__ y, int64_t ldy) {
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const float* xr = x + r * ldx;
+    uint16_t* yr = y + r * ldy;
+    for (int64_t c = threadIdx.x; c < cols; c += blockDim.x)
+      yr[c] = __bfloat16_as_ushort(__float2bfloat16_rn(__ldg(xr + c)));
+  }
+}
+
+// 2-D bf16 tensor map {cols, rows} with row pitch ld elements, box {64, box_rows},
+// 128-byte swizzle; elements past the tensor read as zero.
+cudaError_t encode_bf16_operand(CUtensorMap* map, const void* base, int64_t cols, int64_t rows,
+                                int64_t ld, int box_rows) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kLinBK), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int BN, int ACT>
+cudaError_t run_linear(const CUtensorMap& a_lo, const CUtensorMap& a_hi, const CUtensorMap& w,
+                       const LinearArgs& args, cudaStream_t stream) {
+  auto* fn = &linear_bf16_kernel<BN, ACT>;
+  constexpr int smem = LinSmem<BN>::kTotal;
+  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>((args.M + kLinBM - 1) / kLinBM),
+                  static_cast<unsigned>((args.N + BN - 1) / BN));
+  fn<<<grid, kLinThreads, smem, stream>>>(a_lo, a_hi, w, args);
+  return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t run_linear_act(int act, const CUtensorMap& a_lo, const CUtensorMap& a_hi,
+                           const CUtensorMap& w, const LinearArgs& args, cudaStream_t stream) {
+  switch (act) {
+    case DLRM_ACT_RELU: return run_linear<BN, DLRM_ACT_RELU>(a_lo, a_hi, w, args, stream);
+    case DLRM_ACT_SIGMOID: return run_linear<BN, DLRM_ACT_SIGMOID>(a_lo, a_hi, w, args, stream);
+    default: return run_linear<BN, DLRM_ACT_NONE>(a_lo, a_hi, w, args, stream);
+  }
+}
+
+int sm_count_current() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n;
+}
+
+// Tile width: the widest of 256, 128 whose tile count still covers every SM,
+// else 64 (more, smaller tiles for small layers).
+int choose_bn(int64_t M, int64_t N, int sms) {
+  const int64_t mt = (M + kLinBM - 1) / kLinBM;
+  if (N <= 64) return 64;
+  if (mt * ((N + 255) / 256) >= sms) return 256;
+  if (mt * ((N + 127) / 128) >= sms) return 128;
+  return 64;
+}
+
+bool is_aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+}  // namespace dlrm
+
+extern "C" {
+
+DLRM_API int dlrm_linear_bf16(const uint16_t* a_lo, int64_t lda_lo, int64_t k_lo,
+                              const uint16_t* a_hi, int64_t lda_hi, int64_t k_hi,
+                              const uint16_t* w, int64_t ldw, const float* bias, int64_t M,
+                              int64_t N, int act, float* y_f32, int64_t ldy_f32,
+                              uint16_t* y_bf16, int64_t ldy_bf16, int32_t* status_dev,
+                              dlrm_stream_t stream) {
+  using namespace dlrm;
+  if (a_lo == nullptr || w == nullptr) return DLRM_ERR_NULL;
+  if (y_f32 == nullptr && y_bf16 == nullptr) return DLRM_ERR_NULL;
+  if (k_hi > 0 && a_hi == nullptr) return DLRM_ERR_NULL;
+  if (act < DLRM_ACT_NONE || act > DLRM_ACT_SIGMOID) return DLRM_ERR_ARG;
+  if (M < 1 || N < 1 || k_lo < 1 || k_hi < 0) return DLRM_ERR_SHAPE;
+  const int64_t K = k_lo + k_hi;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return DLRM_ERR_SHAPE;
+  if (lda_lo < k_lo || (k_hi > 0 && lda_hi < k_hi) || ldw < K) return DLRM_ERR_SHAPE;
+  if ((y_f32 != nullptr && ldy_f32 < N) || (y_bf16 != nullptr && ldy_bf16 < N))
+    return DLRM_ERR_SHAPE;
+  if ((N + 63) / 64 > 65535) return DLRM_ERR_SHAPE;  // grid.y
+  if (lda_lo % 8 != 0 || (k_hi > 0 && lda_hi % 8 != 0) || ldw % 8 != 0) return DLRM_ERR_ALIGN;
+  if (k_hi > 0 && k_lo % 8 != 0) return DLRM_ERR_ALIGN;
+  if (!is_aligned(a_lo, 16) || (k_hi > 0 && !is_aligned(a_hi, 16)) || !is_aligned(w, 16))
+    return DLRM_ERR_ALIGN;
+  if ((bias != nullptr && !is_aligned(bias, 4)) || (y_f32 != nullptr && !is_aligned(y_f32, 4)) ||
+      (y_bf16 != nullptr && !is_aligned(y_bf16, 2)) ||
+      (status_dev != nullptr && !is_aligned(status_dev, 4)))
+    return DLRM_ERR_ALIGN;
+
+  const int bn = choose_bn(M, N, sm_count_current());
+  CUtensorMap ma_lo, ma_hi, mw;
+  cudaError_t e = encode_bf16_operand(&ma_lo, a_lo, k_lo, M, lda_lo, kLinBM);
+  if (e == cudaSuccess && k_hi > 0) e = encode_bf16_operand(&ma_hi, a_hi, k_hi, M, lda_hi, kLinBM);
+  if (e == cudaSuccess) e = encode_bf16_operand(&mw, w, K, N, ldw, bn);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (k_hi == 0) ma_hi = ma_lo;  // never read
+
+  LinearArgs args;
+  args.bias = bias;
+  args.y_f32 = y_f32;
+  args.y_bf16 = y_bf16;
+  args.ldy_f32 = ldy_f32;
+  args.ldy_bf16 = ldy_bf16;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.k_lo = static_cast<int>(k_lo);
+  args.nkb_lo = static_cast<int>((k_lo + kLinBK - 1) / kLinBK);
+  args.nkb_hi = static_cast<int>((k_hi + kLinBK - 1) / kLinBK);
+  args.status = status_dev;
+  auto* s = reinterpret_cast<cudaStream_t>(stream);
+  switch (bn) {
+    case 256: e = run_linear_act<256>(act, ma_lo, ma_hi, mw, args, s); break;
+    case 128: e = run_linear_act<128>(act, ma_lo, ma_hi, mw, args, s); break;
+    default: e = run_linear_act<64>(act, ma_lo, ma_hi, mw, args, s); break;
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+  note_launch();
+  return DLRM_OK;
+}
+
+DLRM_API int dlrm_f32_to_bf16(const float* x, int64_t ldx, int64_t rows, int64_t cols,
+                              uint16_t* y, int64_t ldy, dlrm_stream_t stream) {
+  using namespace dlrm;
+  if (x == nullptr || y == nullptr) return DLRM_ERR_NULL;
+  if (rows < 1 || cols < 1 || ldx < cols || ldy < cols) return DLRM_ERR_SHAPE;
+  if (!is_aligned(x, 4) || !is_aligned(y, 2)) return DLRM_ERR_ALIGN;
+  const int64_t blocks = std::min<int64_t>(rows, 148 * 32);
+  const int threads = cols >= 256 ? 256 : static_cast<int>(((cols + 31) / 32) * 32);
+  f32_to_bf16_kernel<<<static_cast<unsigned>(blocks), threads, 0,
+                       reinterpret_cast<cudaStream_t>(stream)>>>(x, ldx, rows, cols, y, ldy);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  note_launch();
+  return DLRM_OK;
+}
+
+}  // extern "C"

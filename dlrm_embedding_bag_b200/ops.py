@@ -1,4 +1,5 @@
-"""Python binding of ``libdlrm_sparse.so`` (the C ABI in ``include/dlrm_sparse.h``).
+"""Python binding of ``libdlrm_sparse.so`` (the C ABI in ``include/dlrm_sparse.h``;
+the MLP layers of ``include/dlrm_mlp.h`` are bound in :mod:`.mlp`).
 
 Argument marshalling only: every function checks tensor placement, dtype and
 contiguity, passes raw pointers and the current CUDA stream to the C entry
@@ -56,6 +57,10 @@ SIGNATURES = {
     "dlrm_status_string": (ctypes.c_char_p, [_I]),
     "dlrm_last_cuda_error": (_I, []),
     "dlrm_launch_count": (_I64, []),
+    # include/dlrm_mlp.h
+    "dlrm_linear_bf16": (_I, [_P, _I64, _I64, _P, _I64, _I64, _P, _I64, _P, _I64, _I64, _I, _P,
+                              _I64, _P, _I64, _P, _P]),
+    "dlrm_f32_to_bf16": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P]),
 }
 
 

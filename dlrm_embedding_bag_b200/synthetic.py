@@ -153,3 +153,50 @@ def make_dense(w: Workload, device="cpu") -> "torch.Tensor":
     t = torch.empty((w.B, w.D), dtype=torch.float32, device=device)
     t.normal_(0.0, 1.0, generator=g)
     return t
+
+
+# DLRMv1 MLPs around the stage. The pages give no layer widths for their DLRMv1
+# sweep; these follow the DLRM reference architecture for 13 dense features
+# and D = 64: bottom 13-512-256-D, top (D+P)-512-256-1.
+DENSE_FEATURES = 13
+BOTTOM_HIDDEN = (512, 256)
+TOP_HIDDEN = (512, 256)
+
+
+def make_mlp_layers(in_features: int, widths, seed: int, device="cpu", last: str = "relu"):
+    """Seeded layers ``(w, bias, act)`` of an MLP ``in_features -> widths...``.
+
+    ``w`` is ``(N, K)`` bf16 (round-to-nearest-even of N(0, sqrt(2/(N+K))) f32
+    draws) stored with a row pitch rounded up to 8 elements; ``bias`` is
+    ``(N,)`` f32 N(0, sqrt(1/N)); hidden layers use ReLU, the last ``last``.
+    Layer ``i`` draws from a torch generator seeded ``seed * 100 + i``.
+    """
+    import torch
+
+    layers = []
+    k = in_features
+    for i, n in enumerate(widths):
+        g = torch.Generator(device=device)
+        g.manual_seed(seed * 100 + i)
+        w32 = torch.empty((n, k), device=device).normal_(0.0, (2.0 / (n + k)) ** 0.5,
+                                                          generator=g)
+        b = torch.empty(n, device=device).normal_(0.0, (1.0 / n) ** 0.5, generator=g)
+        w = torch.empty((n, (k + 7) // 8 * 8), dtype=torch.bfloat16, device=device)[:, :k]
+        w.copy_(w32.to(torch.bfloat16))
+        act = last if i == len(widths) - 1 else "relu"
+        layers.append((w, b, act))
+        k = n
+    return layers
+
+
+def make_dense_features(B: int, device="cpu", seed: int = 5000):
+    """``(B, 13)`` bf16 dense input features (log-normal-like, as Criteo's
+    log(1 + count) features): |N(0, 1)| rounded to bf16, pitch 16."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    x = torch.empty((B, DENSE_FEATURES), device=device).normal_(0.0, 1.0, generator=g).abs_()
+    out = torch.empty((B, 16), dtype=torch.bfloat16, device=device)[:, :DENSE_FEATURES]
+    out.copy_(x.to(torch.bfloat16))
+    return out

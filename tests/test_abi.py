@@ -12,13 +12,16 @@ import subprocess
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "dlrm_sparse.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("dlrm_sparse.h", "dlrm_mlp.h")]
 
 
 def _declared():
-    src = open(HEADER).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return set(re.findall(r"DLRM_API\s+[\w\s\*]+?\b(\w+)\s*\(", src))
+    names = set()
+    for h in HEADERS:
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"DLRM_API\s+[\w\s\*]+?\b(\w+)\s*\(", src))
+    return names
 
 
 @pytest.fixture(scope="module")
@@ -32,7 +35,8 @@ def ops():
 def test_header_declares_the_stage_entry_points():
     names = _declared()
     assert {"embbag_sum_multi", "interact_lower_tri", "dlrm_sparse_interact"} <= names
-    assert len(names) == 15
+    assert {"dlrm_linear_bf16", "dlrm_f32_to_bf16"} <= names
+    assert len(names) == 17
 
 
 def test_library_exports_every_declared_symbol(ops):
@@ -149,3 +153,33 @@ def test_general_pooling_host_checks(ops):
 def test_missing_library_fails_loudly(ops, tmp_path):
     with pytest.raises(ImportError, match="no CPU fallback"):
         ops.load_library(str(tmp_path / "libdlrm_sparse.so"))
+
+
+def test_linear_host_checks(ops):
+    """Bad MLP-layer arguments are rejected before any CUDA call."""
+    lib = ops._lib
+    A = 0x10000  # a 16-byte aligned non-null address that is never dereferenced
+    W = 0x20000
+    Y = 0x30000
+
+    def call(a_lo=A, lda_lo=64, k_lo=64, a_hi=None, lda_hi=0, k_hi=0, w=W, ldw=64, bias=None,
+             M=4, N=8, act=0, y32=Y, ld32=8, y16=None, ld16=0, status=None):
+        return lib.dlrm_linear_bf16(a_lo, lda_lo, k_lo, a_hi, lda_hi, k_hi, w, ldw, bias, M, N,
+                                    act, y32, ld32, y16, ld16, status, None)
+
+    assert call(a_lo=None) == -1
+    assert call(w=None) == -1
+    assert call(y32=None) == -1
+    assert call(k_hi=8, lda_hi=8, ldw=72) == -1          # a_hi missing
+    assert call(act=3) == -8
+    assert call(M=0) == -2 and call(N=0) == -2 and call(k_lo=0) == -2
+    assert call(lda_lo=56) == -2                          # pitch < k
+    assert call(ldw=56) == -2
+    assert call(ld32=7) == -2
+    assert call(lda_lo=68, k_lo=60, ldw=64) == -3         # pitch not a multiple of 8
+    assert call(a_lo=A + 8) == -3                         # 8-byte aligned only
+    assert call(k_lo=60, ldw=72, a_hi=A, lda_hi=8, k_hi=8) == -3  # k_lo % 8 with a split
+    assert call(y32=Y + 2) == -3
+    assert lib.dlrm_f32_to_bf16(None, 4, 1, 4, Y, 4, None) == -1
+    assert lib.dlrm_f32_to_bf16(A, 3, 1, 4, Y, 4, None) == -2
+    assert lib.dlrm_f32_to_bf16(A + 2, 4, 1, 4, Y, 4, None) == -3

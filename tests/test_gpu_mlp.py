@@ -1,0 +1,224 @@
+"""The MLP layers (tcgen05 GEMM with fused bias/activation, split-A) against
+the oracle, on the GPU.
+
+Parity bar: the oracle computes each layer exactly (fp64) from the same bf16
+operand bits. The kernel's products are exact and its accumulation is f32, so
+the pre-activation may differ by at most (K + 2) * 2^-23 * sum_k |a_k w_k| +
+|bias| (K + 1 f32 roundings, each relative to a partial sum bounded by that
+magnitude); ReLU keeps that bound, sigmoid (slope <= 1/4) scales it by 1/4
+and adds the f32 exp/divide error (a few ulp of the result). The bf16 output
+must be exactly the round-to-nearest-even of the kernel's own f32 output.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dlrm_embedding_bag_b200 import mlp, ops, synthetic as syn
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+ACT_CODE = {"none": 0, "relu": 1, "sigmoid": 2}
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _rand_bf16(g, rows, cols, std=1.0, pitch=None):
+    x = torch.empty((rows, cols), device=DEV).normal_(0, std, generator=g)
+    buf = mlp.bf16_empty(rows, pitch or cols, DEV)[:, :cols]
+    buf.copy_(x.to(torch.bfloat16))
+    return buf
+
+
+def _check_layer(y32, y16, a_lo, w, bias, act, a_hi=None, rows=None, what=""):
+    """y32/y16: kernel outputs; rows: optional subset of rows to check."""
+    a = a_lo if rows is None else a_lo[rows]
+    h = None if a_hi is None else (a_hi if rows is None else a_hi[rows])
+    out, pre, bound = oracle.linear_bf16(_bits(a), _bits(w),
+                                         None if bias is None else bias.cpu().numpy(),
+                                         ACT_CODE[act], a_hi=None if h is None else _bits(h))
+    K = w.shape[1]
+    slope = 0.25 if act == "sigmoid" else 1.0
+    tol = slope * (K + 2) * 2.0 ** -23 * bound + 8 * 2.0 ** -24 * np.abs(out) + 1e-30
+    if y32 is not None:
+        got = (y32 if rows is None else y32[rows]).double().cpu().numpy()
+        err = np.abs(got - out)
+        bad = err > tol
+        assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside the bound; worst "
+                               f"err {err.max():.3e}, tol there {tol.flat[err.argmax()]:.3e}")
+    if y16 is not None and y32 is not None:
+        want16 = _bits(y32.to(torch.bfloat16))
+        assert np.array_equal(_bits(y16), want16), f"{what}: bf16 output is not RNE of f32"
+
+
+def _run(M, N, K, act="none", bias=True, seed=0, pitch_a=None, pitch_y=None, rows=None,
+         bf16=True):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    a = _rand_bf16(g, M, K, 1.0, pitch_a)
+    w = _rand_bf16(g, N, K, K ** -0.5)
+    b = torch.empty(N, device=DEV).normal_(0, 0.5, generator=g) if bias else None
+    y32 = None
+    if pitch_y:
+        y32 = torch.full((M, pitch_y), float("nan"), device=DEV)[:, :N]
+    y32, y16 = mlp.linear_bf16(a, w, b, act, out_f32=y32, bf16=bf16)
+    torch.cuda.synchronize()
+    _check_layer(y32, y16, a, w, b, act, rows=rows, what=f"M={M} N={N} K={K} {act}")
+    return y32, y16
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 8), (5, 3, 16), (128, 64, 64), (200, 96, 72),
+                                   (300, 130, 200), (129, 257, 136), (1000, 512, 592),
+                                   (64, 40, 13)])
+def test_linear_shapes(M, N, K):
+    _run(M, N, K, seed=M + N + K)
+
+
+@pytest.mark.parametrize("act", ["none", "relu", "sigmoid"])
+def test_linear_activations(act):
+    y32, _ = _run(333, 200, 96, act=act, seed=7)
+    if act == "relu":
+        assert (y32 >= 0).all() and (y32 == 0).any()
+    if act == "sigmoid":
+        assert ((y32 > 0) & (y32 < 1)).all()
+
+
+def test_linear_no_bias_bf16_only_and_pitched():
+    _run(150, 70, 80, bias=False, seed=3)
+    _run(150, 70, 80, seed=4, pitch_a=96, pitch_y=75)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(5)
+    a = _rand_bf16(g, 77, 40)
+    w = _rand_bf16(g, 33, 40)
+    y32, _ = mlp.linear_bf16(a, w, None, "relu")
+    _, y16 = mlp.linear_bf16(a, w, None, "relu", f32=False, bf16=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(y16), _bits(y32.to(torch.bfloat16)))
+
+
+@pytest.mark.parametrize("M,N,K", [(20000, 512, 128), (10000, 256, 192)])
+def test_linear_wide_tiles_sampled(M, N, K):
+    """Sizes that select 256- and 128-column tiles; the oracle checks 96 rows."""
+    rows = torch.from_numpy(np.random.default_rng(M).choice(M, 96, replace=False)).to(DEV)
+    _run(M, N, K, act="relu", seed=11, rows=rows)
+
+
+@pytest.mark.parametrize("k_lo,k_hi", [(64, 528), (128, 351), (24, 40), (8, 8), (64, 0)])
+def test_linear_split_a(k_lo, k_hi):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(k_lo * 1000 + k_hi)
+    M, N = 260, 192
+    a_lo = _rand_bf16(g, M, k_lo)
+    a_hi = _rand_bf16(g, M, k_hi) if k_hi else None
+    w = _rand_bf16(g, N, k_lo + k_hi, (k_lo + k_hi) ** -0.5)
+    b = torch.empty(N, device=DEV).normal_(0, 0.5, generator=g)
+    y32, y16 = mlp.linear_bf16(a_lo, w, b, "relu", a_hi=a_hi, bf16=True)
+    torch.cuda.synchronize()
+    _check_layer(y32, y16, a_lo, w, b, "relu", a_hi=a_hi, what=f"split {k_lo}+{k_hi}")
+    if k_hi and k_lo % 64 == 0:
+        # same K blocks as the layer on the concatenation: identical bits
+        cat = mlp.bf16_empty(M, k_lo + k_hi, DEV)
+        cat[:, :k_lo].copy_(a_lo)
+        cat[:, k_lo:].copy_(a_hi)
+        c32, _ = mlp.linear_bf16(cat, w, b, "relu")
+        torch.cuda.synchronize()
+        assert torch.equal(c32.view(torch.int32), y32.view(torch.int32))
+
+
+def test_f32_to_bf16_matches_torch_rne():
+    rng = np.random.default_rng(9)
+    bits = rng.integers(0, 2 ** 32, size=(37, 301), dtype=np.uint64).astype(np.uint32)
+    x = bits.view(np.float32).copy()
+    x[~np.isfinite(x)] = 0.0
+    x[0, :8] = [0.0, -0.0, np.inf, -np.inf, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1e-40, -1e-40]
+    xt = torch.from_numpy(x).to(DEV)
+    y = mlp.to_bf16(xt)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(y), _bits(xt.to(torch.bfloat16)))
+
+
+def _dlrm_case(seed, B, F, N, D, L, dense_in=13, bot=(64, 32), top=(64, 32)):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    bottom = mlp.MLP(syn.make_mlp_layers(dense_in, list(bot) + [D], seed, DEV))
+    P = (F + 1) * F // 2
+    top_m = mlp.MLP(syn.make_mlp_layers(D + P, list(top) + [1], seed + 1, DEV, last="sigmoid"))
+    w = syn.Workload("t", B=B, F=F, N=N, D=D, L=L)
+    weights = syn.make_weights(w, DEV)
+    idx = torch.from_numpy(syn.make_indices(w)).to(DEV)
+    off = torch.from_numpy(syn.make_offsets(w)).to(DEV)
+    x = _rand_bf16(g, B, dense_in)
+    return bottom, top_m, x, weights, idx, off
+
+
+def test_mlp_chain_per_layer():
+    bottom, _, x, *_ = _dlrm_case(21, 300, 4, 100, 64, 3)
+    (y32, _), inputs = bottom.forward(x, keep=True, last_bf16=True)
+    torch.cuda.synchronize()
+    outs = [inp[0] for inp in inputs[1:]] + [None]
+    for i, ((w, b, act), (a, _)) in enumerate(zip(bottom.layers, inputs)):
+        if outs[i] is not None:
+            # the next layer's bf16 input is this layer's bf16 output; check it
+            # against the oracle through its f32 twin recomputed with f32=True
+            r32, r16 = mlp.linear_bf16(a, w, b, act, bf16=True)
+            torch.cuda.synchronize()
+            assert torch.equal(r16.contiguous().view(torch.int16),
+                               outs[i].contiguous().view(torch.int16))
+            _check_layer(r32, r16, a, w, b, act, what=f"bottom layer {i}")
+        else:
+            _check_layer(y32, None, a, w, b, act, what=f"bottom layer {i}")
+
+
+def test_dlrm_forward_chain():
+    """Every stage of the forward against the oracle, fed the kernel's own inputs."""
+    B, F, N, D, L = 256, 8, 1000, 64, 4
+    bottom, top, x, weights, idx, off = _dlrm_case(31, B, F, N, D, L)
+    ctr, t = mlp.dlrm_forward(bottom, top, x, weights, idx, off, L, keep=True)
+    torch.cuda.synchronize()
+    assert ctr.shape == (B, 1) and ((ctr > 0) & (ctr < 1)).all()
+    # bottom: last layer's f32 and bf16 outputs agree
+    assert np.array_equal(_bits(t["dense16"]), _bits(t["dense32"].to(torch.bfloat16)))
+    # sparse stage: pooled bit-exact, z within the dot bound
+    wn = [w_.cpu().numpy() for w_ in weights]
+    pooled, inter, bound = oracle.sparse_interact(wn, idx.cpu().numpy(), off.cpu().numpy(),
+                                                  t["dense32"].cpu().numpy(), B, L,
+                                                  with_bound=True)
+    assert np.array_equal(t["pooled"].cpu().numpy().view(np.uint32), pooled.view(np.uint32))
+    assert np.all(np.abs(t["z"].cpu().numpy().astype(np.float64) - inter) <= 1e-5 * bound + 1e-30)
+    assert np.array_equal(_bits(t["z16"]), _bits(t["z"].to(torch.bfloat16)))
+    # top: first layer reads [dense | z] through the split form
+    (a0, h0) = t["top_inputs"][0]
+    w0, b0, act0 = top.layers[0]
+    r32, _ = mlp.linear_bf16(a0, w0, b0, act0, a_hi=h0)
+    torch.cuda.synchronize()
+    _check_layer(r32, None, a0, w0, b0, act0, a_hi=h0, what="top layer 0")
+    (a_last, _) = t["top_inputs"][-1]
+    wl, bl, actl = top.layers[-1]
+    _check_layer(ctr, None, a_last, wl, bl, actl, what="CTR head")
+
+
+def test_linear_graph_capture_and_launch_count():
+    g = torch.Generator(device=DEV)
+    g.manual_seed(41)
+    a = _rand_bf16(g, 512, 128)
+    w = _rand_bf16(g, 256, 128)
+    b = torch.zeros(256, device=DEV)
+    y = torch.empty((512, 256), device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    n0 = ops.launch_count()
+    mlp.linear_bf16(a, w, b, "relu", out_f32=y, status=status)
+    assert ops.launch_count() == n0 + 1
+    ref = y.clone()
+    y.zero_()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            mlp.linear_bf16(a, w, b, "relu", out_f32=y, status=status)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
+    assert int(status.item()) == 0
