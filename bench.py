@@ -52,6 +52,8 @@ def parse_args(argv=None):
     ap.add_argument("--batch", type=int, default=None, help="override the batch size")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mlp", action="store_true",
+                    help="time the DLRMv1 MLP layers (tcgen05) and the full forward instead")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU time budget of the oracle baseline sample")
     args = ap.parse_args(argv)
@@ -63,6 +65,18 @@ def parse_args(argv=None):
 def dist_env():
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
             int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The maximum of x over all ranks (x itself on one rank); every rank calls it."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def algorithmic_bytes(w: syn.Workload, write_pooled: bool = True) -> int:
@@ -86,12 +100,18 @@ def measured_peaks():
         return None
 
 
+# The sources the benchmarked fused kernel and its launch are built from: a
+# recorded DRAM traffic figure stays valid while none of them changes.
+FUSED_SOURCES = [os.path.join(CSRC, n) for n in (
+    "device_common.cuh", "interact_common.cuh", "kernels.cuh", "inst_f32x4.cu", "kernels.cu",
+    "launch.h", "api.cu")] + [os.path.join(ROOT, "include", "dlrm_sparse.h")]
+
+
 def source_digest() -> str:
     h = hashlib.sha256()
-    for d in (CSRC, os.path.join(ROOT, "include")):
-        for name in sorted(os.listdir(d)):
-            with open(os.path.join(d, name), "rb") as fh:
-                h.update(name.encode() + b"\0" + fh.read())
+    for path in FUSED_SOURCES:
+        with open(path, "rb") as fh:
+            h.update(os.path.basename(path).encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -373,11 +393,7 @@ def run_ours(args, w: syn.Workload):
         per, wall, launches, sampler = timed_region()
         remeasured = True
 
-    total_ms = float(sum(per))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(per)), world, dev)
     lookups = world * args.steps * w.B * w.F * w.L
     value = lookups / (total_ms / 1e3)
     ms_step = total_ms / args.steps
@@ -416,11 +432,7 @@ def run_ours(args, w: syn.Workload):
             cur.wait_event(ev)
         t1.record(cur)
         barrier()
-        e2e_ms = t0.elapsed_time(t1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
         e2e = {"value": lookups / (e2e_ms / 1e3), "unit": "lookups/s",
                "h2d_bytes_per_step": pipe.h2d_bytes(), "d2h_bytes_per_step": pipe.d2h_bytes(),
                "ms_per_step": e2e_ms / args.steps,
@@ -465,6 +477,108 @@ def run_ours(args, w: syn.Workload):
     return 0
 
 
+# ----------------------------------------------------------------------------- MLP layers
+
+def run_mlp(args, w: syn.Workload):
+    """Time each DLRMv1 MLP layer (bf16 tcgen05 GEMM + bias + activation) at the
+    workload's batch and at 32x that batch, and the full DLRMv1 forward
+    (bottom MLP, sparse stage, top MLP) at the workload's batch. One JSON line."""
+    import torch
+    from dlrm_embedding_bag_b200 import mlp, ops
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+
+    def timeit(fn, steps, warmup):
+        for _ in range(warmup):
+            flush.fill_(1)
+            fn()
+        torch.cuda.synchronize()
+        st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            st[i].record()
+            fn()
+            en[i].record()
+        torch.cuda.synchronize()
+        return statistics.median([a.elapsed_time(b) for a, b in zip(st, en)])
+
+    P = w.P
+    bottom_w = [syn.DENSE_FEATURES, *syn.BOTTOM_HIDDEN, w.D]
+    top_w = [w.D + P, *syn.TOP_HIDDEN, 1]
+    layers = []
+    for B in (w.B, 32 * w.B):
+        g = torch.Generator(device=dev)
+        g.manual_seed(B)
+        for name, widths, last, split in (("bottom", bottom_w, "relu", False),
+                                          ("top", top_w, "sigmoid", True)):
+            ls = syn.make_mlp_layers(widths[0], widths[1:], 7 if name == "bottom" else 8, dev,
+                                     last=last)
+            for i, (wt, b, act) in enumerate(ls):
+                K, N = wt.shape[1], wt.shape[0]
+                if split and i == 0:
+                    a_lo = mlp.bf16_empty(B, w.D, dev)
+                    a_lo.copy_(torch.randn(B, w.D, device=dev, generator=g).to(torch.bfloat16))
+                    a_hi = mlp.bf16_empty(B, P, dev)
+                    a_hi.copy_(torch.randn(B, P, device=dev, generator=g).to(torch.bfloat16))
+                else:
+                    a_lo = mlp.bf16_empty(B, K, dev)
+                    a_lo.copy_(torch.randn(B, K, device=dev, generator=g).to(torch.bfloat16))
+                    a_hi = None
+                last_layer = i == len(ls) - 1
+                y32 = torch.empty((B, N), device=dev) if last_layer else None
+                y16 = None if last_layer else mlp.bf16_empty(B, N, dev)
+
+                def fn(a_lo=a_lo, a_hi=a_hi, wt=wt, b=b, act=act, y32=y32, y16=y16):
+                    mlp.linear_bf16(a_lo, wt, b, act, a_hi=a_hi, out_f32=y32, out_bf16=y16,
+                                    f32=y32 is not None, bf16=y16 is not None)
+
+                ms = timeit(fn, args.steps, args.warmup)
+                flops = 2.0 * B * N * K
+                layers.append({"mlp": name, "layer": i, "B": B, "K": K, "N": N,
+                               "split_a": bool(split and i == 0), "act": act, "us": 1e3 * ms,
+                               "tflops": flops / (ms / 1e3) / 1e12})
+    # the full forward at the workload's batch
+    bottom = mlp.MLP(syn.make_mlp_layers(bottom_w[0], bottom_w[1:], 7, dev))
+    top = mlp.MLP(syn.make_mlp_layers(top_w[0], top_w[1:], 8, dev, last="sigmoid"))
+    weights = syn.make_weights(w, dev)
+    idx = torch.from_numpy(syn.make_indices(w)).to(dev)
+    off = torch.from_numpy(syn.make_offsets(w)).to(dev)
+    x = syn.make_dense_features(w.B, dev)
+    n0 = ops.launch_count()
+    mlp.dlrm_forward(bottom, top, x, weights, idx, off, w.L)
+    fwd_launches = ops.launch_count() - n0
+    fwd_ms = timeit(lambda: mlp.dlrm_forward(bottom, top, x, weights, idx, off, w.L),
+                    args.steps, args.warmup)
+    big = max(layers, key=lambda r: r["B"] * r["N"] * r["K"])
+    peaks = measured_peaks() or {}
+    peak = float(peaks.get("bf16_tflops") or 1590.0)
+    line = {
+        "metric": "DLRMv1 MLP layer TFLOP/s (bf16 tcgen05, f32 accumulate, fused bias+act)",
+        "value": big["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"DLRMv1 MLPs bottom {'-'.join(map(str, bottom_w))}, top "
+                               f"{'-'.join(map(str, top_w))} (top layer 0 split-A "
+                               f"[D={w.D} | P={P}]) at B={w.B} and {32 * w.B}",
+                   "l2": "flushed between steps"},
+        "roofline": {"bound": "tensor", "kernel": f"linear_bf16_kernel B={big['B']} "
+                     f"K={big['K']} N={big['N']}", "achieved": big["tflops"], "peak": peak,
+                     "peak_source": "measured (burst)" if peaks.get("bf16_tflops") else "fallback",
+                     "unit": "TFLOP/s", "frac": big["tflops"] / peak},
+        "layers": layers,
+        "forward": {"workload": w.name, "B": w.B, "us": 1e3 * fwd_ms,
+                    "samples_per_s": w.B / (fwd_ms / 1e3), "gpu_launches": fwd_launches,
+                    "steps": "bottom MLP (3 layers), fused sparse stage, z to bf16, top MLP "
+                             "(3 layers, first split-A)"},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     w = syn.CONFIGS[args.config]
@@ -474,6 +588,8 @@ def main(argv=None):
         w = w.scaled(B=B, N=N, name=f"{w.name}_B{B}_N{N}")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.mlp:
+        return run_mlp(args, w)
     return run_ours(args, w)
 
 
