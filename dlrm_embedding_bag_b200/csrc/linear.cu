@@ -3,19 +3,26 @@
 // linear_bias_relu, linear_bias_sigmoid and the split-A forms), plus the f32 ->
 // bf16 conversion that feeds it. Declared in dlrm_mlp.h.
 //
-// One CTA of 128 threads computes a 128 x BN tile of Y:
-//   - thread 0 streams 64-wide K blocks of A (128 x 64 bf16) and W (BN x 64)
-//     into a 4-stage shared-memory ring with 2-D TMA loads (128-byte swizzle);
-//     K blocks 0..nkb_lo-1 read A_lo, the rest read A_hi, and W's column
-//     offset follows, so the concatenation is never built;
-//   - thread 32 waits for each stage and issues four tcgen05.mma (K = 16 each)
-//     that accumulate the tile in f32 in tensor memory, then commits the
-//     stage back to the producer through an mbarrier;
-//   - after the last MMA all four warps read their 32 accumulator rows with
-//     tcgen05.ld, add the bias, apply the activation and store f32 and/or bf16.
+// Persistent, warp-specialised kernel: CTA c walks the 128 x BN tiles
+// t = c, c + gridDim.x, ... (N tiles fastest, so CTAs running side by side
+// share A rows in L2). Ten warps:
+//   - warp 0 (one thread) streams 64-wide K blocks of A (128 x 64 bf16) and W
+//     (BN x 64) into a 4-stage shared-memory ring with 2-D TMA loads (128-byte
+//     swizzle), running ahead across tiles; K blocks 0..nkb_lo-1 read A_lo,
+//     the rest read A_hi, and W's column offset follows, so the
+//     concatenation is never built;
+//   - warp 1 allocates tensor memory for two f32 accumulators (2 x BN
+//     columns) and one thread issues four tcgen05.mma (K = 16 each) per
+//     stage into the tile's accumulator, committing each stage back to the
+//     producer and each finished accumulator to the epilogue;
+//   - warps 2-9 read the finished accumulator (warp w owns TMEM lanes
+//     32*(w%4)..+31 and half of the columns), add the bias, apply the
+//     activation and store f32 and/or bf16, then hand the accumulator back -
+//     so the epilogue of tile i runs while the MMAs of tile i+1 fill the
+//     other accumulator.
 // Every wait on an mbarrier is bounded; a wait that runs out sets
-// DLRM_FLAG_TIMEOUT in the optional status word and the CTA still frees its
-// tensor memory and exits.
+// DLRM_FLAG_TIMEOUT in the optional status word, ends that role's loop, and
+// the CTA still frees its tensor memory and exits.
 #include <algorithm>
 #include <climits>
 #include <cstdint>
@@ -31,8 +38,12 @@ namespace {
 
 constexpr int kLinBM = 128;    // rows of a tile (tcgen05 M)
 constexpr int kLinBK = 64;     // K per stage: 64 bf16 = one 128-byte swizzle row
-constexpr int kLinStages = 4;  // shared-memory ring depth
-constexpr int kLinThreads = 128;
+#ifndef DLRM_LIN_STAGES
+#define DLRM_LIN_STAGES 4
+#endif
+constexpr int kLinStages = DLRM_LIN_STAGES;  // shared-memory ring depth
+constexpr int kLinEpiWarps = 8;  // two per TMEM lane quarter, each half of the columns
+constexpr int kLinThreads = 64 + 32 * kLinEpiWarps;  // producer warp, MMA warp, epilogue
 constexpr long long kLinWaitLimit = 200000000LL;  // clock cycles, about 0.1 s
 
 template <int BN>
@@ -40,8 +51,11 @@ struct LinSmem {
   static constexpr int kA = kLinBM * kLinBK * 2;
   static constexpr int kB = BN * kLinBK * 2;
   static constexpr int kStage = kA + kB;
-  static constexpr int kBars = kLinStages * kStage;  // full[S], empty[S], done, tmem slot
-  static constexpr int kTotal = kBars + (2 * kLinStages + 1) * 8 + 8 + 1024;  // + alignment
+  // each epilogue warp's slice of the tile's bias, then the barriers:
+  // full[S], empty[S], acc_full[2], acc_empty[2]; then the TMEM slot
+  static constexpr int kBias = kLinStages * kStage;
+  static constexpr int kBars = kBias + kLinEpiWarps * (BN / 2) * 4;
+  static constexpr int kTotal = kBars + (2 * kLinStages + 4) * 8 + 8 + 1024;  // + alignment
 };
 
 struct LinearArgs {
@@ -50,6 +64,7 @@ struct LinearArgs {
   uint16_t* y_bf16;
   int64_t ldy_f32, ldy_bf16;
   int M, N, k_lo, nkb_lo, nkb_hi;
+  int tiles_n, tiles;
   int32_t* status;
 };
 
@@ -69,141 +84,192 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
          (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
 }
 
+// Store 32 consecutive results of one row (columns nb .. nb+31, clipped to N).
+__device__ __forceinline__ void store_chunk32(const LinearArgs& args, int row, int nb,
+                                              const float (&v)[32], bool f32_vec, bool bf_vec) {
+  if (row >= args.M) return;
+  const bool whole = nb + 32 <= args.N;
+  if (args.y_f32 != nullptr) {
+    float* y = args.y_f32 + static_cast<int64_t>(row) * args.ldy_f32 + nb;
+    if (whole && f32_vec) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        reinterpret_cast<float4*>(y)[q] =
+            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (nb + j < args.N) y[j] = v[j];
+    }
+  }
+  if (args.y_bf16 != nullptr) {
+    uint16_t* y = args.y_bf16 + static_cast<int64_t>(row) * args.ldy_bf16 + nb;
+    if (whole && bf_vec) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        reinterpret_cast<uint4*>(y)[q] = make_uint4(
+            pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+            pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (nb + j < args.N) y[j] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
+    }
+  }
+}
+
 template <int BN, int ACT>
 __global__ void __launch_bounds__(kLinThreads, 1)
     linear_bf16_kernel(const __grid_constant__ CUtensorMap map_a_lo,
                        const __grid_constant__ CUtensorMap map_a_hi,
                        const __grid_constant__ CUtensorMap map_w, const LinearArgs args) {
   using L = LinSmem<BN>;
-  constexpr uint32_t kCols = BN < 32 ? 32 : BN;  // TMEM columns: f32 accumulator
+  constexpr uint32_t kCols = 2 * BN;  // two f32 accumulators (a power of two >= 128)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // 1024-byte aligned tiles
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* empty = full + kLinStages;
-  uint64_t* done = empty + kLinStages;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* acc_full = empty + kLinStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(tslot, kCols);
     tmem_relinquish();
   }
-  if (threadIdx.x == 32) {
+  if (threadIdx.x == 0) {
     for (int s = 0; s < kLinStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kLinEpiWarps);  // one arrival per epilogue warp
+    }
     mbar_init_fence();
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tslot;
-
-  const int m0 = blockIdx.x * kLinBM, n0 = blockIdx.y * BN;
   const int nkb = args.nkb_lo + args.nkb_hi;
   bool timed_out = false;
-  if (threadIdx.x == 0) {
-    // TMA producer.
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % kLinStages;
-      if (kb >= kLinStages &&
-          !mbar_wait_bounded(&empty[s], ((kb / kLinStages) - 1) & 1, kLinWaitLimit)) {
-        timed_out = true;
-        break;
-      }
-      uint8_t* sa = smem + s * L::kStage;
-      uint8_t* sb = sa + L::kA;
-      mbar_arrive_expect_tx(&full[s], L::kStage);
-      if (kb < args.nkb_lo) {
-        tma_load_2d(sa, &map_a_lo, &full[s], kb * kLinBK, m0);
-        tma_load_2d(sb, &map_w, &full[s], kb * kLinBK, n0);
-      } else {
-        const int kh = kb - args.nkb_lo;
-        tma_load_2d(sa, &map_a_hi, &full[s], kh * kLinBK, m0);
-        tma_load_2d(sb, &map_w, &full[s], args.k_lo + kh * kLinBK, n0);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // TMA producer: a continuous K-block stream over this CTA's tiles.
+      int g = 0;
+      for (int t = blockIdx.x; t < args.tiles && !timed_out; t += gridDim.x) {
+        const int m0 = (t / args.tiles_n) * kLinBM, n0 = (t % args.tiles_n) * BN;
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = g % kLinStages;
+          if (g >= kLinStages &&
+              !mbar_wait_bounded(&empty[s], ((g / kLinStages) - 1) & 1, kLinWaitLimit)) {
+            timed_out = true;
+            break;
+          }
+          uint8_t* sa = smem + s * L::kStage;
+          uint8_t* sb = sa + L::kA;
+          mbar_arrive_expect_tx(&full[s], L::kStage);
+          if (kb < args.nkb_lo) {
+            tma_load_2d(sa, &map_a_lo, &full[s], kb * kLinBK, m0);
+            tma_load_2d(sb, &map_w, &full[s], kb * kLinBK, n0);
+          } else {
+            const int kh = kb - args.nkb_lo;
+            tma_load_2d(sa, &map_a_hi, &full[s], kh * kLinBK, m0);
+            tma_load_2d(sb, &map_w, &full[s], args.k_lo + kh * kLinBK, n0);
+          }
+        }
       }
     }
-  } else if (threadIdx.x == 32) {
-    // MMA issuer.
-    constexpr uint32_t idesc = idesc_bf16_f32(kLinBM, BN);
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % kLinStages;
-      if (!mbar_wait_bounded(&full[s], (kb / kLinStages) & 1, kLinWaitLimit)) {
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // MMA issuer.
+      constexpr uint32_t idesc = idesc_bf16_f32(kLinBM, BN);
+      int g = 0, j = 0;
+      for (int t = blockIdx.x; t < args.tiles && !timed_out; t += gridDim.x, ++j) {
+        const int b = j & 1;
+        if (j >= 2 && !mbar_wait_bounded(&acc_empty[b], ((j >> 1) - 1) & 1, kLinWaitLimit)) {
+          timed_out = true;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t acc = tmem + static_cast<uint32_t>(b * BN);
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = g % kLinStages;
+          if (!mbar_wait_bounded(&full[s], (g / kLinStages) & 1, kLinWaitLimit)) {
+            timed_out = true;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t sa = smem_u32(smem + s * L::kStage);
+          const uint32_t sb = sa + L::kA;
+#pragma unroll
+          for (int kk = 0; kk < kLinBK / 16; ++kk)
+            tc_mma_bf16(acc, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32), idesc,
+                        (kb | kk) != 0 ? 1u : 0u);
+          tc_commit(&empty[s]);  // the stage is free once these MMAs have read it
+        }
+        tc_commit(&acc_full[b]);  // the accumulator is final once all of them are done
+      }
+    }
+  } else {
+    // Epilogue warps 2..9: warp w reads TMEM lane quarter w % 4 (rows 32*(w%4) ..
+    // +31 of a tile) and column half (w - 2) / 4 of the accumulator, 32 columns
+    // per tcgen05.ld; its slice of the bias is staged in shared memory per tile.
+    constexpr int kColsPerWarp = BN / 2;
+    const int quarter = warp & 3;
+    const int c_begin = ((warp - 2) >> 2) * kColsPerWarp;
+    float* bias_s = reinterpret_cast<float*>(smem + L::kBias) + (warp - 2) * kColsPerWarp;
+    const bool f32_vec = args.y_f32 != nullptr && (args.ldy_f32 % 4) == 0 &&
+                         (reinterpret_cast<uintptr_t>(args.y_f32) % 16) == 0;
+    const bool bf_vec = args.y_bf16 != nullptr && (args.ldy_bf16 % 8) == 0 &&
+                        (reinterpret_cast<uintptr_t>(args.y_bf16) % 16) == 0;
+    int j = 0;
+    for (int t = blockIdx.x; t < args.tiles; t += gridDim.x, ++j) {
+      const int b = j & 1;
+      const int m0 = (t / args.tiles_n) * kLinBM, n0 = (t % args.tiles_n) * BN;
+      for (int c = lane; c < kColsPerWarp; c += 32) {
+        const int n = n0 + c_begin + c;
+        bias_s[c] = (args.bias != nullptr && n < args.N) ? __ldg(args.bias + n) : 0.f;
+      }
+      __syncwarp();
+      const bool ok =
+          __all_sync(0xffffffffu, mbar_wait_bounded(&acc_full[b], (j >> 1) & 1, kLinWaitLimit));
+      if (!ok) {
         timed_out = true;
         break;
       }
       tc_fence_after_sync();
-      const uint32_t sa = smem_u32(smem + s * L::kStage);
-      const uint32_t sb = sa + L::kA;
-#pragma unroll
-      for (int kk = 0; kk < kLinBK / 16; ++kk)
-        tc_mma_bf16(tmem, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32), idesc,
-                    (kb | kk) != 0 ? 1u : 0u);
-      tc_commit(&empty[s]);  // the stage is free once these MMAs have read it
-    }
-    tc_commit(done);
-  }
-  __syncwarp();
-
-  // Epilogue: warp w owns accumulator rows 32w .. 32w+31 (TMEM lanes).
-  const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(done, 0, kLinWaitLimit) ? 1 : 0);
-  tc_fence_after_sync();
-  const int row = m0 + warp * 32 + lane;
-  const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  const bool f32_vec = args.y_f32 != nullptr && (args.ldy_f32 % 4) == 0 &&
-                       (reinterpret_cast<uintptr_t>(args.y_f32) % 16) == 0;
-  const bool bf_vec = args.y_bf16 != nullptr && (args.ldy_bf16 % 8) == 0 &&
-                      (reinterpret_cast<uintptr_t>(args.y_bf16) % 16) == 0;
-  if (ok) {
+      const int row = m0 + quarter * 32 + lane;
+      const uint32_t trow =
+          tmem + static_cast<uint32_t>(b * BN) + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
-    for (int c0 = 0; c0 < BN && n0 + c0 < args.N; c0 += 16) {
-      float v[16];
-      tmem_ld_32x32b_x16(trow + c0, v);
-      const int nb = n0 + c0;
+      for (int c0 = c_begin; c0 < c_begin + kColsPerWarp && n0 + c0 < args.N; c0 += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(trow + c0, v);
+        const float4* bq = reinterpret_cast<const float4*>(bias_s + (c0 - c_begin));
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float b = (args.bias != nullptr && nb + j < args.N) ? __ldg(args.bias + nb + j) : 0.f;
-        v[j] = activate<ACT>(__fadd_rn(v[j], b));
-      }
-      if (row >= args.M) continue;
-      const bool whole = nb + 16 <= args.N;
-      if (args.y_f32 != nullptr) {
-        float* y = args.y_f32 + static_cast<int64_t>(row) * args.ldy_f32 + nb;
-        if (whole && f32_vec) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            reinterpret_cast<float4*>(y)[q] =
-                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (nb + j < args.N) y[j] = v[j];
+        for (int q = 0; q < 8; ++q) {
+          const float4 bb = bq[q];
+          v[4 * q] = activate<ACT>(__fadd_rn(v[4 * q], bb.x));
+          v[4 * q + 1] = activate<ACT>(__fadd_rn(v[4 * q + 1], bb.y));
+          v[4 * q + 2] = activate<ACT>(__fadd_rn(v[4 * q + 2], bb.z));
+          v[4 * q + 3] = activate<ACT>(__fadd_rn(v[4 * q + 3], bb.w));
         }
+        store_chunk32(args, row, n0 + c0, v, f32_vec, bf_vec);
       }
-      if (args.y_bf16 != nullptr) {
-        uint16_t* y = args.y_bf16 + static_cast<int64_t>(row) * args.ldy_bf16 + nb;
-        if (whole && bf_vec) {
-#pragma unroll
-          for (int q = 0; q < 2; ++q)
-            reinterpret_cast<uint4*>(y)[q] =
-                make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                           pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                           pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (nb + j < args.N) y[j] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
-        }
-      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);  // this warp has drained its share
     }
   }
-  if ((timed_out || !ok) && args.status != nullptr) atomicOr(args.status, DLRM_FLAG_TIMEOUT);
+  if (timed_out && args.status != nullptr) atomicOr(args.status, DLRM_FLAG_TIMEOUT);
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kCols);
+  if (warp == 1) tmem_dealloc(tmem, kCols);
 }
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ x, int64_t ldx, int64_t rows,
@@ -235,25 +301,31 @@ cudaError_t encode_bf16_operand(CUtensorMap* map, const void* base, int64_t cols
 
 template <int BN, int ACT>
 cudaError_t run_linear(const CUtensorMap& a_lo, const CUtensorMap& a_hi, const CUtensorMap& w,
-                       const LinearArgs& args, cudaStream_t stream) {
+                       LinearArgs args, int sms, cudaStream_t stream) {
   auto* fn = &linear_bf16_kernel<BN, ACT>;
   constexpr int smem = LinSmem<BN>::kTotal;
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>((args.M + kLinBM - 1) / kLinBM),
-                  static_cast<unsigned>((args.N + BN - 1) / BN));
+  args.tiles_n = (args.N + BN - 1) / BN;
+  const int64_t tiles = static_cast<int64_t>((args.M + kLinBM - 1) / kLinBM) * args.tiles_n;
+  if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+  args.tiles = static_cast<int>(tiles);
+  // one CTA per SM: the shared-memory ring and the 2 x BN TMEM columns size it
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
   fn<<<grid, kLinThreads, smem, stream>>>(a_lo, a_hi, w, args);
   return cudaGetLastError();
 }
 
 template <int BN>
 cudaError_t run_linear_act(int act, const CUtensorMap& a_lo, const CUtensorMap& a_hi,
-                           const CUtensorMap& w, const LinearArgs& args, cudaStream_t stream) {
+                           const CUtensorMap& w, const LinearArgs& args, int sms,
+                           cudaStream_t stream) {
   switch (act) {
-    case DLRM_ACT_RELU: return run_linear<BN, DLRM_ACT_RELU>(a_lo, a_hi, w, args, stream);
-    case DLRM_ACT_SIGMOID: return run_linear<BN, DLRM_ACT_SIGMOID>(a_lo, a_hi, w, args, stream);
-    default: return run_linear<BN, DLRM_ACT_NONE>(a_lo, a_hi, w, args, stream);
+    case DLRM_ACT_RELU: return run_linear<BN, DLRM_ACT_RELU>(a_lo, a_hi, w, args, sms, stream);
+    case DLRM_ACT_SIGMOID:
+      return run_linear<BN, DLRM_ACT_SIGMOID>(a_lo, a_hi, w, args, sms, stream);
+    default: return run_linear<BN, DLRM_ACT_NONE>(a_lo, a_hi, w, args, sms, stream);
   }
 }
 
@@ -267,6 +339,9 @@ int sm_count_current() {
 // Tile width: the widest of 256, 128 whose tile count still covers every SM,
 // else 64 (more, smaller tiles for small layers).
 int choose_bn(int64_t M, int64_t N, int sms) {
+#ifdef DLRM_LIN_FORCE_BN
+  if (N > 64) return DLRM_LIN_FORCE_BN;
+#endif
   const int64_t mt = (M + kLinBM - 1) / kLinBM;
   if (N <= 64) return 64;
   if (mt * ((N + 255) / 256) >= sms) return 256;
@@ -308,7 +383,8 @@ DLRM_API int dlrm_linear_bf16(const uint16_t* a_lo, int64_t lda_lo, int64_t k_lo
       (status_dev != nullptr && !is_aligned(status_dev, 4)))
     return DLRM_ERR_ALIGN;
 
-  const int bn = choose_bn(M, N, sm_count_current());
+  const int sms = sm_count_current();
+  const int bn = choose_bn(M, N, sms);
   CUtensorMap ma_lo, ma_hi, mw;
   cudaError_t e = encode_bf16_operand(&ma_lo, a_lo, k_lo, M, lda_lo, kLinBM);
   if (e == cudaSuccess && k_hi > 0) e = encode_bf16_operand(&ma_hi, a_hi, k_hi, M, lda_hi, kLinBM);
@@ -330,9 +406,9 @@ DLRM_API int dlrm_linear_bf16(const uint16_t* a_lo, int64_t lda_lo, int64_t k_lo
   args.status = status_dev;
   auto* s = reinterpret_cast<cudaStream_t>(stream);
   switch (bn) {
-    case 256: e = run_linear_act<256>(act, ma_lo, ma_hi, mw, args, s); break;
-    case 128: e = run_linear_act<128>(act, ma_lo, ma_hi, mw, args, s); break;
-    default: e = run_linear_act<64>(act, ma_lo, ma_hi, mw, args, s); break;
+    case 256: e = run_linear_act<256>(act, ma_lo, ma_hi, mw, args, sms, s); break;
+    case 128: e = run_linear_act<128>(act, ma_lo, ma_hi, mw, args, sms, s); break;
+    default: e = run_linear_act<64>(act, ma_lo, ma_hi, mw, args, sms, s); break;
   }
   if (e != cudaSuccess) return cuda_fail(e);
   note_launch();
