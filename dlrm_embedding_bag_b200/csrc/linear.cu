@@ -38,24 +38,29 @@ namespace {
 
 constexpr int kLinBM = 128;    // rows of a tile (tcgen05 M)
 constexpr int kLinBK = 64;     // K per stage: 64 bf16 = one 128-byte swizzle row
-#ifndef DLRM_LIN_STAGES
-#define DLRM_LIN_STAGES 4
-#endif
-constexpr int kLinStages = DLRM_LIN_STAGES;  // shared-memory ring depth
+// shared-memory ring depth (3 with 256-column tiles, whose stages are 48 KB)
+template <int BN>
+constexpr int lin_stages() { return BN >= 256 ? 3 : 4; }
 constexpr int kLinEpiWarps = 8;  // two per TMEM lane quarter, each half of the columns
 constexpr int kLinThreads = 64 + 32 * kLinEpiWarps;  // producer warp, MMA warp, epilogue
 constexpr long long kLinWaitLimit = 200000000LL;  // clock cycles, about 0.1 s
 
 template <int BN>
 struct LinSmem {
+  static constexpr int kStages = lin_stages<BN>();
   static constexpr int kA = kLinBM * kLinBK * 2;
   static constexpr int kB = BN * kLinBK * 2;
   static constexpr int kStage = kA + kB;
-  // each epilogue warp's slice of the tile's bias, then the barriers:
-  // full[S], empty[S], acc_full[2], acc_empty[2]; then the TMEM slot
-  static constexpr int kBias = kLinStages * kStage;
+  // After the ring: each epilogue warp's output staging (a 32 x 32 f32 tile in
+  // the 128-byte swizzled layout, then a 32 x 32 bf16 tile in the 64-byte
+  // swizzled layout), its slice of the tile's bias, then the barriers full[S],
+  // empty[S], acc_full[2], acc_empty[2] and the TMEM slot.
+  static constexpr int kStage32 = 32 * 32 * 4;
+  static constexpr int kStage16 = 32 * 32 * 2;
+  static constexpr int kStaging = kStages * kStage;
+  static constexpr int kBias = kStaging + kLinEpiWarps * (kStage32 + kStage16);
   static constexpr int kBars = kBias + kLinEpiWarps * (BN / 2) * 4;
-  static constexpr int kTotal = kBars + (2 * kLinStages + 4) * 8 + 8 + 1024;  // + alignment
+  static constexpr int kTotal = kBars + (2 * kStages + 4) * 8 + 8 + 1024;  // + alignment
 };
 
 struct LinearArgs {
@@ -65,6 +70,7 @@ struct LinearArgs {
   int64_t ldy_f32, ldy_bf16;
   int M, N, k_lo, nkb_lo, nkb_hi;
   int tiles_n, tiles;
+  int tma_f32, tma_bf16;  // write that output through TMA stores (see the launcher)
   int32_t* status;
 };
 
@@ -122,15 +128,17 @@ template <int BN, int ACT>
 __global__ void __launch_bounds__(kLinThreads, 1)
     linear_bf16_kernel(const __grid_constant__ CUtensorMap map_a_lo,
                        const __grid_constant__ CUtensorMap map_a_hi,
-                       const __grid_constant__ CUtensorMap map_w, const LinearArgs args) {
+                       const __grid_constant__ CUtensorMap map_w,
+                       const __grid_constant__ CUtensorMap map_y32,
+                       const __grid_constant__ CUtensorMap map_y16, const LinearArgs args) {
   using L = LinSmem<BN>;
   constexpr uint32_t kCols = 2 * BN;  // two f32 accumulators (a power of two >= 128)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // 1024-byte aligned tiles
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBars);
-  uint64_t* empty = full + kLinStages;
-  uint64_t* acc_full = empty + kLinStages;
+  uint64_t* empty = full + L::kStages;
+  uint64_t* acc_full = empty + L::kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -140,7 +148,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     tmem_relinquish();
   }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kLinStages; ++s) {
+    for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -164,9 +172,9 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       for (int t = blockIdx.x; t < args.tiles && !timed_out; t += gridDim.x) {
         const int m0 = (t / args.tiles_n) * kLinBM, n0 = (t % args.tiles_n) * BN;
         for (int kb = 0; kb < nkb; ++kb, ++g) {
-          const int s = g % kLinStages;
-          if (g >= kLinStages &&
-              !mbar_wait_bounded(&empty[s], ((g / kLinStages) - 1) & 1, kLinWaitLimit)) {
+          const int s = g % L::kStages;
+          if (g >= L::kStages &&
+              !mbar_wait_bounded(&empty[s], ((g / L::kStages) - 1) & 1, kLinWaitLimit)) {
             timed_out = true;
             break;
           }
@@ -198,8 +206,8 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         tc_fence_after_sync();
         const uint32_t acc = tmem + static_cast<uint32_t>(b * BN);
         for (int kb = 0; kb < nkb; ++kb, ++g) {
-          const int s = g % kLinStages;
-          if (!mbar_wait_bounded(&full[s], (g / kLinStages) & 1, kLinWaitLimit)) {
+          const int s = g % L::kStages;
+          if (!mbar_wait_bounded(&full[s], (g / L::kStages) & 1, kLinWaitLimit)) {
             timed_out = true;
             break;
           }
@@ -219,14 +227,23 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     // Epilogue warps 2..9: warp w reads TMEM lane quarter w % 4 (rows 32*(w%4) ..
     // +31 of a tile) and column half (w - 2) / 4 of the accumulator, 32 columns
     // per tcgen05.ld; its slice of the bias is staged in shared memory per tile.
+    // A 32 x 32 result block goes out either through the warp's staging tiles
+    // and one TMA store per output (lane r writes row r; 16-byte chunk q of a row
+    // sits at chunk q ^ (r & 7) of a 128-byte f32 row and q ^ ((r >> 1) & 3) of a
+    // 64-byte bf16 row, the layouts the maps' 128- and 64-byte swizzles read, so
+    // the 32 lanes' 16-byte writes spread over all banks), or with direct stores.
     constexpr int kColsPerWarp = BN / 2;
+    const int ew = warp - 2;
     const int quarter = warp & 3;
-    const int c_begin = ((warp - 2) >> 2) * kColsPerWarp;
-    float* bias_s = reinterpret_cast<float*>(smem + L::kBias) + (warp - 2) * kColsPerWarp;
+    const int c_begin = (ew >> 2) * kColsPerWarp;
+    float* bias_s = reinterpret_cast<float*>(smem + L::kBias) + ew * kColsPerWarp;
+    uint8_t* st32 = smem + L::kStaging + ew * (L::kStage32 + L::kStage16);
+    uint8_t* st16 = st32 + L::kStage32;
     const bool f32_vec = args.y_f32 != nullptr && (args.ldy_f32 % 4) == 0 &&
                          (reinterpret_cast<uintptr_t>(args.y_f32) % 16) == 0;
     const bool bf_vec = args.y_bf16 != nullptr && (args.ldy_bf16 % 8) == 0 &&
                         (reinterpret_cast<uintptr_t>(args.y_bf16) % 16) == 0;
+    const bool tma_out = args.tma_f32 || args.tma_bf16;
     int j = 0;
     for (int t = blockIdx.x; t < args.tiles; t += gridDim.x, ++j) {
       const int b = j & 1;
@@ -243,7 +260,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      const int row = m0 + quarter * 32 + lane;
+      const int row0 = m0 + quarter * 32;
       const uint32_t trow =
           tmem + static_cast<uint32_t>(b * BN) + (static_cast<uint32_t>(quarter * 32) << 16);
 #pragma unroll 1
@@ -259,12 +276,45 @@ __global__ void __launch_bounds__(kLinThreads, 1)
           v[4 * q + 2] = activate<ACT>(__fadd_rn(v[4 * q + 2], bb.z));
           v[4 * q + 3] = activate<ACT>(__fadd_rn(v[4 * q + 3], bb.w));
         }
-        store_chunk32(args, row, n0 + c0, v, f32_vec, bf_vec);
+        if (tma_out) {
+          if (lane == 0) bulk_wait_read_all();  // the previous block has left the staging
+          __syncwarp();
+          if (args.tma_f32) {
+            uint4* rowp = reinterpret_cast<uint4*>(st32 + lane * 128);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              rowp[q ^ (lane & 7)] =
+                  make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                             __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+          }
+          if (args.tma_bf16) {
+            uint4* rowp = reinterpret_cast<uint4*>(st16 + lane * 64);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              rowp[q ^ ((lane >> 1) & 3)] = make_uint4(
+                  pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                  pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (args.tma_f32) tma_store_2d(&map_y32, st32, n0 + c0, row0);
+            if (args.tma_bf16) tma_store_2d(&map_y16, st16, n0 + c0, row0);
+            bulk_commit();
+          }
+        }
+        if (!args.tma_f32 || !args.tma_bf16) {
+          LinearArgs direct = args;  // the outputs not written through TMA
+          if (args.tma_f32) direct.y_f32 = nullptr;
+          if (args.tma_bf16) direct.y_bf16 = nullptr;
+          store_chunk32(direct, row0 + lane, n0 + c0, v, f32_vec, bf_vec);
+        }
       }
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);  // this warp has drained its share
     }
+    if (lane == 0) bulk_wait_all();  // every TMA store of this warp has completed
   }
   if (timed_out && args.status != nullptr) atomicOr(args.status, DLRM_FLAG_TIMEOUT);
   tc_fence_before_sync();
@@ -301,7 +351,8 @@ cudaError_t encode_bf16_operand(CUtensorMap* map, const void* base, int64_t cols
 
 template <int BN, int ACT>
 cudaError_t run_linear(const CUtensorMap& a_lo, const CUtensorMap& a_hi, const CUtensorMap& w,
-                       LinearArgs args, int sms, cudaStream_t stream) {
+                       const CUtensorMap& y32, const CUtensorMap& y16, LinearArgs args, int sms,
+                       cudaStream_t stream) {
   auto* fn = &linear_bf16_kernel<BN, ACT>;
   constexpr int smem = LinSmem<BN>::kTotal;
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
@@ -313,20 +364,36 @@ cudaError_t run_linear(const CUtensorMap& a_lo, const CUtensorMap& a_hi, const C
   args.tiles = static_cast<int>(tiles);
   // one CTA per SM: the shared-memory ring and the 2 x BN TMEM columns size it
   const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
-  fn<<<grid, kLinThreads, smem, stream>>>(a_lo, a_hi, w, args);
+  fn<<<grid, kLinThreads, smem, stream>>>(a_lo, a_hi, w, y32, y16, args);
   return cudaGetLastError();
 }
 
 template <int BN>
 cudaError_t run_linear_act(int act, const CUtensorMap& a_lo, const CUtensorMap& a_hi,
-                           const CUtensorMap& w, const LinearArgs& args, int sms,
-                           cudaStream_t stream) {
+                           const CUtensorMap& w, const CUtensorMap& y32, const CUtensorMap& y16,
+                           const LinearArgs& args, int sms, cudaStream_t stream) {
   switch (act) {
-    case DLRM_ACT_RELU: return run_linear<BN, DLRM_ACT_RELU>(a_lo, a_hi, w, args, sms, stream);
+    case DLRM_ACT_RELU:
+      return run_linear<BN, DLRM_ACT_RELU>(a_lo, a_hi, w, y32, y16, args, sms, stream);
     case DLRM_ACT_SIGMOID:
-      return run_linear<BN, DLRM_ACT_SIGMOID>(a_lo, a_hi, w, args, sms, stream);
-    default: return run_linear<BN, DLRM_ACT_NONE>(a_lo, a_hi, w, args, sms, stream);
+      return run_linear<BN, DLRM_ACT_SIGMOID>(a_lo, a_hi, w, y32, y16, args, sms, stream);
+    default: return run_linear<BN, DLRM_ACT_NONE>(a_lo, a_hi, w, y32, y16, args, sms, stream);
   }
+}
+
+// 2-D output map {N, M} with row pitch ld elements, box {32, 32}, written from a
+// staging tile in the given swizzle layout.
+cudaError_t encode_output(CUtensorMap* map, void* base, CUtensorMapDataType dt, int esz, int64_t N,
+                          int64_t M, int64_t ld, CUtensorMapSwizzle swz) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * esz};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swz, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 int sm_count_current() {
@@ -404,11 +471,25 @@ DLRM_API int dlrm_linear_bf16(const uint16_t* a_lo, int64_t lda_lo, int64_t k_lo
   args.nkb_lo = static_cast<int>((k_lo + kLinBK - 1) / kLinBK);
   args.nkb_hi = static_cast<int>((k_hi + kLinBK - 1) / kLinBK);
   args.status = status_dev;
+  // Outputs whose rows are whole 16-byte units at 16-byte aligned addresses go
+  // out through TMA stores; the others are written directly.
+  CUtensorMap my32, my16;
+  args.tma_f32 = y_f32 != nullptr && ldy_f32 % 4 == 0 && is_aligned(y_f32, 16);
+  args.tma_bf16 = y_bf16 != nullptr && ldy_bf16 % 8 == 0 && is_aligned(y_bf16, 16);
+  if (args.tma_f32)
+    e = encode_output(&my32, y_f32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, M, ldy_f32,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e == cudaSuccess && args.tma_bf16)
+    e = encode_output(&my16, y_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, ldy_bf16,
+                      CU_TENSOR_MAP_SWIZZLE_64B);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (!args.tma_f32) my32 = mw;  // never read
+  if (!args.tma_bf16) my16 = mw;  // never read
   auto* s = reinterpret_cast<cudaStream_t>(stream);
   switch (bn) {
-    case 256: e = run_linear_act<256>(act, ma_lo, ma_hi, mw, args, sms, s); break;
-    case 128: e = run_linear_act<128>(act, ma_lo, ma_hi, mw, args, sms, s); break;
-    default: e = run_linear_act<64>(act, ma_lo, ma_hi, mw, args, sms, s); break;
+    case 256: e = run_linear_act<256>(act, ma_lo, ma_hi, mw, my32, my16, args, sms, s); break;
+    case 128: e = run_linear_act<128>(act, ma_lo, ma_hi, mw, my32, my16, args, sms, s); break;
+    default: e = run_linear_act<64>(act, ma_lo, ma_hi, mw, my32, my16, args, sms, s); break;
   }
   if (e != cudaSuccess) return cuda_fail(e);
   note_launch();
