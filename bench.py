@@ -52,6 +52,8 @@ def parse_args(argv=None):
     ap.add_argument("--batch", type=int, default=None, help="override the batch size")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the fused stage on the 11 x 5 batch x table-count sweep instead")
     ap.add_argument("--mlp", action="store_true",
                     help="time the DLRMv1 MLP layers (tcgen05) and the full forward instead")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -477,6 +479,58 @@ def run_ours(args, w: syn.Workload):
     return 0
 
 
+# ----------------------------------------------------------------------------- sweep
+
+def run_sweep(args):
+    """The fused stage on every cell of the batch x table-count sweep (100000 x 64
+    tables, L=8, uniform indices). One JSON line with one entry per cell."""
+    import torch
+    from dlrm_embedding_bag_b200 import ops
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    cells = list(syn.sweep())
+    Fmax = max(c.F for c in cells)
+    tables = syn.make_weights(cells[0].scaled(F=Fmax), dev)  # table k is the same in every cell
+    out = []
+    for w in cells:
+        idx = torch.from_numpy(syn.make_indices(w)).to(dev)
+        off = torch.from_numpy(syn.make_offsets(w)).to(dev)
+        dense = syn.make_dense(w, dev)
+        inter = torch.empty((w.B, w.P), device=dev)
+        call = ops.SparseInteractCall(tables[:w.F], idx, off, dense, w.L, inter_out=inter)
+        s = torch.cuda.current_stream().cuda_stream
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            call(s)
+        torch.cuda.synchronize()
+        st = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        en = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            st[i].record()
+            call(s)
+            en[i].record()
+        torch.cuda.synchronize()
+        ms = statistics.median([a.elapsed_time(b) for a, b in zip(st, en)])
+        out.append({"B": w.B, "F": w.F, "us": 1e3 * ms,
+                    "lookups_per_s": w.B * w.F * w.L / (ms / 1e3),
+                    "samples_per_s": w.B / (ms / 1e3)})
+    big = max(out, key=lambda c: (c["B"], c["F"]))
+    line = {"metric": METRIC + " over the batch x num_cat sweep", "value": big["lookups_per_s"],
+            "unit": "lookups/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "sweep: B in 1..1024 (11 values) x F in {1,4,8,16,32}, "
+                                   "100000 x 64 f32 tables, L=8 uniform, fixed-stride offsets",
+                       "l2": "flushed before every step", "value_cell": "B=1024, F=32",
+                       "timing": "median of steps per cell"},
+            "cells": out}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- MLP layers
 
 def run_mlp(args, w: syn.Workload):
@@ -553,6 +607,16 @@ def run_mlp(args, w: syn.Workload):
     fwd_launches = ops.launch_count() - n0
     fwd_ms = timeit(lambda: mlp.dlrm_forward(bottom, top, x, weights, idx, off, w.L),
                     args.steps, args.warmup)
+    # the same forward captured once into a CUDA graph and replayed (no launch gaps)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        mlp.dlrm_forward(bottom, top, x, weights, idx, off, w.L)  # allocations outside capture
+        with torch.cuda.graph(graph, stream=side):
+            graph_out = mlp.dlrm_forward(bottom, top, x, weights, idx, off, w.L)  # noqa: F841
+    torch.cuda.current_stream().wait_stream(side)
+    graph_ms = timeit(graph.replay, args.steps, args.warmup)
     big = max(layers, key=lambda r: r["B"] * r["N"] * r["K"])
     peaks = measured_peaks() or {}
     peak = float(peaks.get("bf16_tflops") or 1590.0)
@@ -572,6 +636,7 @@ def run_mlp(args, w: syn.Workload):
         "layers": layers,
         "forward": {"workload": w.name, "B": w.B, "us": 1e3 * fwd_ms,
                     "samples_per_s": w.B / (fwd_ms / 1e3), "gpu_launches": fwd_launches,
+                    "graph_us": 1e3 * graph_ms, "graph_samples_per_s": w.B / (graph_ms / 1e3),
                     "steps": "bottom MLP (3 layers), fused sparse stage, z to bf16, top MLP "
                              "(3 layers, first split-A)"},
     }
@@ -590,6 +655,8 @@ def main(argv=None):
         return run_reference(args, w)
     if args.mlp:
         return run_mlp(args, w)
+    if args.sweep:
+        return run_sweep(args)
     return run_ours(args, w)
 
 
