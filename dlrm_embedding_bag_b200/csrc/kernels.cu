@@ -149,6 +149,9 @@ int64_t interact_smem_per_sample(int F, int D) {
   return FeatLayout::make(F, D).floats_per_sample() * static_cast<int64_t>(sizeof(float));
 }
 
+#ifndef DLRM_FUSED_LQ_MAX
+#define DLRM_FUSED_LQ_MAX 4
+#endif
 // Samples per block and log2 of the lanes per tile for the dot phase.
 static void choose_dot_shape(int F, int D, int B, int samples_wanted, int64_t smem_cap, int& S,
                              int& lq) {
@@ -159,7 +162,7 @@ static void choose_dot_shape(int F, int D, int B, int samples_wanted, int64_t sm
   S = std::min(s, B);
   const int tiles = S * Lf.nT;
   const int qmax = std::max(1, kBlockThreads / tiles);
-  lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), 4});
+  lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), DLRM_FUSED_LQ_MAX});
 }
 
 static cudaError_t counted(cudaError_t e) {
