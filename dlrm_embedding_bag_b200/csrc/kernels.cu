@@ -100,6 +100,18 @@ __global__ void __launch_bounds__(kBlockThreads, 2)
   cp_async_wait<0>();
 }
 
+// The bounded mbarrier wait of the asynchronous kernels, on a barrier that
+// nothing completes (dlrm_probe_bounded_wait).
+__global__ void probe_wait_kernel(long long limit, int32_t* status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, limit)) atomicOr(status, DLRM_FLAG_TIMEOUT);
+}
+
 __global__ void pair_decode_kernel(int64_t p0, int64_t count, int32_t* __restrict__ i_out,
                                    int32_t* __restrict__ j_out) {
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < count;
@@ -434,6 +446,11 @@ cudaError_t launch_interact(const float* dense, const float* emb, int B, int F, 
     e = run_interact<1, 0>(dense, emb, B, F, D, out, smem_limit, sms, stream);
   }
   return counted(e);
+}
+
+cudaError_t launch_probe_wait(int64_t limit, int32_t* status, cudaStream_t stream) {
+  probe_wait_kernel<<<1, 32, 0, stream>>>(static_cast<long long>(limit), status);
+  return counted(cudaGetLastError());
 }
 
 cudaError_t launch_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_t* j_out,

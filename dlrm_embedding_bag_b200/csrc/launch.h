@@ -150,6 +150,8 @@ cudaError_t launch_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_
                                cudaStream_t stream);
 
 int64_t launch_count();
+
+cudaError_t launch_probe_wait(int64_t limit, int32_t* status, cudaStream_t stream);
 // Counts one kernel launch of this library (dlrm_launch_count).
 void note_launch();
 

@@ -57,6 +57,7 @@ SIGNATURES = {
     "dlrm_status_string": (ctypes.c_char_p, [_I]),
     "dlrm_last_cuda_error": (_I, []),
     "dlrm_launch_count": (_I64, []),
+    "dlrm_probe_bounded_wait": (_I, [_I64, _P, _P]),
     # include/dlrm_mlp.h
     "dlrm_linear_bf16": (_I, [_P, _I64, _I64, _P, _I64, _I64, _P, _I64, _P, _I64, _I64, _I, _P,
                               _I64, _P, _I64, _P, _P]),
@@ -495,3 +496,10 @@ def status_from_flags(flags: int) -> int:
 def launch_count() -> int:
     """Kernels the library has launched in this process."""
     return int(_lib.dlrm_launch_count())
+
+
+def probe_bounded_wait(status: torch.Tensor, limit_cycles: int = 1_000_000) -> None:
+    """Run the library's bounded wait on a barrier nothing completes (see the
+    header); DLRM_FLAG_TIMEOUT lands in ``status`` (one int32 on the device)."""
+    _check(_lib.dlrm_probe_bounded_wait(limit_cycles, _dev(status, "status", torch.int32),
+                                        _stream()), "dlrm_probe_bounded_wait")

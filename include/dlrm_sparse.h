@@ -301,6 +301,18 @@ DLRM_API int dlrm_last_cuda_error(void);
 /* Number of kernels this library has launched in this process (all threads). */
 DLRM_API int64_t dlrm_launch_count(void);
 
+/*
+ * dlrm_probe_bounded_wait -- failure-detection check. One thread of one block
+ * waits on a shared-memory mbarrier that nothing ever completes, with the same
+ * bounded wait the asynchronous kernels use (the TMA gather path and the MLP
+ * layers wait that way on their copies and tensor-core work). After about
+ * `limit_cycles` clock cycles (clamped to [1000, 2e8]) the wait gives up, the
+ * kernel ORs DLRM_FLAG_TIMEOUT into *status_dev (dev int32, required) and
+ * returns normally: the CUDA context stays usable. Asynchronous on `stream`.
+ */
+DLRM_API int dlrm_probe_bounded_wait(int64_t limit_cycles, int32_t* status_dev,
+                                     dlrm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -36,7 +36,7 @@ def test_header_declares_the_stage_entry_points():
     names = _declared()
     assert {"embbag_sum_multi", "interact_lower_tri", "dlrm_sparse_interact"} <= names
     assert {"dlrm_linear_bf16", "dlrm_f32_to_bf16"} <= names
-    assert len(names) == 17
+    assert len(names) == 18
 
 
 def test_library_exports_every_declared_symbol(ops):
@@ -183,3 +183,9 @@ def test_linear_host_checks(ops):
     assert lib.dlrm_f32_to_bf16(None, 4, 1, 4, Y, 4, None) == -1
     assert lib.dlrm_f32_to_bf16(A, 3, 1, 4, Y, 4, None) == -2
     assert lib.dlrm_f32_to_bf16(A + 2, 4, 1, 4, Y, 4, None) == -3
+
+
+def test_probe_host_checks(ops):
+    lib = ops._lib
+    assert lib.dlrm_probe_bounded_wait(1000, None, None) == -1
+    assert lib.dlrm_probe_bounded_wait(1000, 0x10002, None) == -3
