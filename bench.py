@@ -51,6 +51,8 @@ def parse_args(argv=None):
                     help="override the rows per table (a smaller case for profiling)")
     ap.add_argument("--batch", type=int, default=None, help="override the batch size")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-depth", type=int, default=4,
+                    help="batches in flight on the end-to-end host pipeline (one stream each)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="time the fused stage on the 11 x 5 batch x table-count sweep instead")
@@ -408,16 +410,18 @@ def run_ours(args, w: syn.Workload):
     e2e = None
     if not args.no_e2e:
         pipe = ops.HostPipeline(weights, w.B, w.L, concat_dense=w.concat_dense, want_pooled=True,
-                                depth=2)
+                                depth=args.e2e_depth)
         batches = []
+        stage0 = pipe.slots[0][0]
         for j in range(E2E_BATCHES):
             ij = syn.make_indices(w, replica=rank * E2E_BATCHES + j) if j else idx_np
-            batches.append((torch.from_numpy(ij.reshape(-1)).pin_memory(),
-                            torch.from_numpy(off_np).pin_memory(), dense.cpu().pin_memory()))
+            # one page-locked block per batch: a single host-to-device copy
+            batches.append(stage0.pack(torch.from_numpy(ij.reshape(-1)), torch.from_numpy(off_np),
+                                       dense.cpu()))
         outs = [torch.empty(tuple(inter.shape), dtype=torch.float32).pin_memory()
-                for _ in range(2)]
+                for _ in range(args.e2e_depth)]
         for i in range(args.warmup):
-            pipe.submit(*batches[i % E2E_BATCHES], outs[i % 2])
+            pipe.submit(*batches[i % E2E_BATCHES], outs[i % args.e2e_depth])
         pipe.drain()
         barrier()
         cur = torch.cuda.current_stream()
@@ -427,7 +431,7 @@ def run_ours(args, w: syn.Workload):
         for _, st, _ in pipe.slots:
             st.wait_event(t0)
         for i in range(args.steps):
-            pipe.submit(*batches[i % E2E_BATCHES], outs[i % 2])
+            pipe.submit(*batches[i % E2E_BATCHES], outs[i % args.e2e_depth])
         for _, st, _ in pipe.slots:
             ev = torch.cuda.Event()
             ev.record(st)
@@ -438,8 +442,8 @@ def run_ours(args, w: syn.Workload):
         e2e = {"value": lookups / (e2e_ms / 1e3), "unit": "lookups/s",
                "h2d_bytes_per_step": pipe.h2d_bytes(), "d2h_bytes_per_step": pipe.d2h_bytes(),
                "ms_per_step": e2e_ms / args.steps,
-               "path": f"dlrm_sparse_interact_host via ops.HostPipeline (2 streams): pinned "
-                       f"indices/offsets/dense in, interaction rows out, {E2E_BATCHES} distinct "
+               "path": f"dlrm_sparse_interact_host via ops.HostPipeline ({args.e2e_depth} streams): one "
+                       f"pinned [indices|offsets|dense] block in, interaction rows out, {E2E_BATCHES} distinct "
                        f"batches in rotation; pooled written to device staging"}
 
     if rank == 0:

@@ -303,16 +303,30 @@ int dlrm_sparse_interact_host(const float* const* weights, const int32_t* indice
   const size_t n_inter = static_cast<size_t>(B) * (concat_dense ? D + P : P) * sizeof(float);
   const size_t n_pooled = static_cast<size_t>(B) * F * D * sizeof(float);
   cudaError_t e;
-  if (n_idx > 0 &&
-      (e = cudaMemcpyAsync(indices_dev, indices_host, n_idx, cudaMemcpyHostToDevice, s)) !=
-          cudaSuccess)
-    return cuda_fail(e);
-  if ((e = cudaMemcpyAsync(offsets_dev, offsets_host, n_off, cudaMemcpyHostToDevice, s)) !=
-      cudaSuccess)
-    return cuda_fail(e);
-  if ((e = cudaMemcpyAsync(dense_dev, dense_host, n_dense, cudaMemcpyHostToDevice, s)) !=
-      cudaSuccess)
-    return cuda_fail(e);
+  // indices, offsets and dense back to back on both sides (no gap): one copy
+  const auto* ih = reinterpret_cast<const char*>(indices_host);
+  auto* id = reinterpret_cast<char*>(indices_dev);
+  const bool packed = n_idx > 0 &&
+                      reinterpret_cast<const char*>(offsets_host) == ih + n_idx &&
+                      reinterpret_cast<const char*>(dense_host) == ih + n_idx + n_off &&
+                      reinterpret_cast<char*>(offsets_dev) == id + n_idx &&
+                      reinterpret_cast<char*>(dense_dev) == id + n_idx + n_off;
+  if (packed) {
+    if ((e = cudaMemcpyAsync(id, ih, n_idx + n_off + n_dense, cudaMemcpyHostToDevice, s)) !=
+        cudaSuccess)
+      return cuda_fail(e);
+  } else {
+    if (n_idx > 0 &&
+        (e = cudaMemcpyAsync(indices_dev, indices_host, n_idx, cudaMemcpyHostToDevice, s)) !=
+            cudaSuccess)
+      return cuda_fail(e);
+    if ((e = cudaMemcpyAsync(offsets_dev, offsets_host, n_off, cudaMemcpyHostToDevice, s)) !=
+        cudaSuccess)
+      return cuda_fail(e);
+    if ((e = cudaMemcpyAsync(dense_dev, dense_host, n_dense, cudaMemcpyHostToDevice, s)) !=
+        cudaSuccess)
+      return cuda_fail(e);
+  }
   int rc = dlrm_sparse_interact(weights, indices_dev, offsets_dev, dense_dev, B, F, L, D,
                                 pooled_dev, inter_dev, concat_dense, stream);
   if (rc != DLRM_OK) return rc;

@@ -390,12 +390,32 @@ class HostStage:
         dev = weights[0].device
         self.P = (self.F + 1) * self.F // 2
         self.row = self.D + self.P if concat_dense else self.P
-        self.idx_dev = torch.empty(self.F * B * L, dtype=torch.int32, device=dev)
-        self.off_dev = torch.empty((self.F, B), dtype=torch.int32, device=dev)
-        self.dense_dev = torch.empty((B, self.D), dtype=torch.float32, device=dev)
+        # one device staging block [indices | offsets | dense], so a packed host
+        # batch (see pack) crosses PCIe in one copy
+        n_idx, n_off, n_dense = self.F * B * L, self.F * B, B * self.D
+        self._staging = torch.empty(n_idx + n_off + n_dense, dtype=torch.int32, device=dev)
+        self.idx_dev = self._staging[:n_idx]
+        self.off_dev = self._staging[n_idx:n_idx + n_off].view(self.F, B)
+        self.dense_dev = self._staging[n_idx + n_off:].view(torch.float32).view(B, self.D)
         self.inter_dev = torch.empty((B, self.row), dtype=torch.float32, device=dev)
         self.pooled_dev = (torch.empty((B, self.F, self.D), dtype=torch.float32, device=dev)
                            if want_pooled else None)
+
+    def pack(self, indices_host: torch.Tensor, offsets_host: torch.Tensor,
+             dense_host: torch.Tensor):
+        """One page-locked host block ``[indices | offsets | dense]`` holding a
+        batch, and the three views into it to pass to a call: the library then
+        moves the batch with a single host-to-device copy."""
+        F, B, L, D = self.F, self.B, self.L, self.D
+        n_idx, n_off = F * B * L, F * B
+        block = torch.empty(n_idx + n_off + B * D, dtype=torch.int32).pin_memory()
+        idx = block[:n_idx]
+        off = block[n_idx:n_idx + n_off].view(F, B)
+        dense = block[n_idx + n_off:].view(torch.float32).view(B, D)
+        idx.copy_(indices_host.reshape(-1))
+        off.copy_(offsets_host.reshape(F, B))
+        dense.copy_(dense_host.reshape(B, D))
+        return idx, off, dense
 
     def h2d_bytes(self) -> int:
         return 4 * (self.F * self.B * self.L + self.F * self.B + self.B * self.D)

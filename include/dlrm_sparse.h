@@ -241,7 +241,9 @@ DLRM_API int dlrm_sparse_interact_pool(const void* const* weights, int table_dty
  * launch dlrm_sparse_interact, copy the interaction rows (and the pooled
  * vectors if pooled_host != NULL) dev -> host. Returns once everything is
  * enqueued; host outputs are valid after the stream has reached this point.
- * Host buffers should be page-locked for the copies to be asynchronous.
+ * Host buffers should be page-locked for the copies to be asynchronous. When
+ * indices, offsets and dense follow each other with no gap both on the host
+ * and in the device staging (indices first), they go over in one copy.
  *   indices_host, offsets_host, dense_host : host, layouts as above.
  *   indices_dev, offsets_dev, dense_dev    : dev staging of the same sizes.
  *   pooled_dev   : dev (B, F, D) or NULL; if given the kernel writes the

@@ -355,6 +355,14 @@ def test_host_stage_matches_device_path(ops):
     assert torch.equal(inter_h.view(torch.int32), fi.cpu().view(torch.int32))
     assert torch.equal(pooled_h.view(torch.int32), fp.cpu().view(torch.int32))
     assert stage.h2d_bytes() == 4 * (w.F * w.B * w.L + w.F * w.B + w.B * w.D)
+    # a packed batch (one host block, one copy) gives the same bits
+    pi, po, pd = stage.pack(ih, oh, dh)
+    inter2 = torch.empty_like(inter_h).pin_memory()
+    pooled2 = torch.empty_like(pooled_h).pin_memory()
+    stage(pi, po, pd, inter2, pooled2)
+    torch.cuda.synchronize()
+    assert torch.equal(inter2.view(torch.int32), inter_h.view(torch.int32))
+    assert torch.equal(pooled2.view(torch.int32), pooled_h.view(torch.int32))
 
 
 def test_repeat_runs_are_bit_identical_and_launch_once(ops):
