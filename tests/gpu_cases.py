@@ -2,7 +2,7 @@
 compare. Pooled sums and every integer result must match bit for bit; a dot
 must satisfy |gpu - oracle| <= 1e-5 * S_ij (S_ij = sum_d |v_i[d] v_j[d]|),
 the relative form of the 1e-5 bound, taken against the magnitudes summed so
-that dots that cancel to near zero are judged on the scale of their terms.
+that dots that cancel to near zero are compared on the scale of their terms.
 """
 from __future__ import annotations
 
