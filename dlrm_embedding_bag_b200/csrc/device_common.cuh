@@ -43,6 +43,7 @@ struct LdF32x4 {  // 128-bit loads of 4 floats
   static constexpr int VEC = 4;
   using Elem = float;
   using Raw = float4;
+  __device__ __forceinline__ static Raw zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
   __device__ __forceinline__ static Raw load(const Elem* p) {
     return __ldg(reinterpret_cast<const float4*>(p));
   }
@@ -55,6 +56,7 @@ struct LdF32x1 {  // scalar fallback
   static constexpr int VEC = 1;
   using Elem = float;
   using Raw = float;
+  __device__ __forceinline__ static Raw zero() { return 0.f; }
   __device__ __forceinline__ static Raw load(const Elem* p) { return __ldg(p); }
   __device__ __forceinline__ static float get(const Raw& r, int) { return r; }
 };
@@ -68,6 +70,7 @@ struct LdBF16x8 {  // 128-bit loads of 8 bf16
   static constexpr int VEC = 8;
   using Elem = uint16_t;
   using Raw = uint4;
+  __device__ __forceinline__ static Raw zero() { return make_uint4(0u, 0u, 0u, 0u); }
   __device__ __forceinline__ static Raw load(const Elem* p) {
     return __ldg(reinterpret_cast<const uint4*>(p));
   }
@@ -81,6 +84,7 @@ struct LdBF16x1 {  // scalar fallback
   static constexpr int VEC = 1;
   using Elem = uint16_t;
   using Raw = unsigned short;
+  __device__ __forceinline__ static Raw zero() { return 0; }
   __device__ __forceinline__ static Raw load(const Elem* p) {
     return __ldg(reinterpret_cast<const unsigned short*>(p));
   }
@@ -193,26 +197,40 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
         const typename LD::Elem* row = W + static_cast<int64_t>(r) * D + col0 + q * VEC;
 #pragma unroll
         for (int m = 0; m < CPL; ++m) {
+          v[u][m] = LD::zero();
           if (ok && colok[m]) v[u][m] = LD::load(row + G * m * VEC);
         }
+        if (POOL == kPoolWeighted) wt[u] = ok ? wt[u] : 0.f;
       }
+      if (POOL != kPoolMax) {
+        // A skipped entry adds +0.0 (weight 0 times 0): the running sum starts
+        // at +0.0 and never becomes -0.0 under round-to-nearest, so adding +0.0
+        // leaves it unchanged, bit for bit, and no branch is needed.
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (use[u]) {
+        for (int u = 0; u < U; ++u) {
 #pragma unroll
           for (int m = 0; m < CPL; ++m)
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
               const float x = LD::get(v[u][m], e);
-              if (POOL == kPoolSum) {
-                acc[m][e] = __fadd_rn(acc[m][e], x);
-              } else if (POOL == kPoolWeighted) {
-                acc[m][e] = __fmaf_rn(wt[u], x, acc[m][e]);
-              } else {
+              acc[m][e] = (POOL == kPoolSum) ? __fadd_rn(acc[m][e], x)
+                                             : __fmaf_rn(wt[u], x, acc[m][e]);
+            }
+          used += use[u] ? 1 : 0;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          if (use[u]) {
+#pragma unroll
+            for (int m = 0; m < CPL; ++m)
+#pragma unroll
+              for (int e = 0; e < VEC; ++e) {
+                const float x = LD::get(v[u][m], e);
                 acc[m][e] = (used == 0) ? x : ((x > acc[m][e]) ? x : acc[m][e]);
               }
-            }
-          ++used;
+            ++used;
+          }
         }
       }
     }
