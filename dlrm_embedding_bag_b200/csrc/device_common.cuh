@@ -161,9 +161,17 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[m][e] = 0.f;
   bool colok[CPL];
+  bool all_cols = true;
 #pragma unroll
-  for (int m = 0; m < CPL; ++m) colok[m] = col0 + (q + G * m) * VEC < D;
-  int used = 0;
+  for (int m = 0; m < CPL; ++m) {
+    colok[m] = col0 + (q + G * m) * VEC < D;
+    all_cols = all_cols && colok[m];
+  }
+  // Batches that every bag of the warp covers entirely, with every column
+  // chunk in range and no index check, take a path with no predicates.
+  const bool plain = POOL != kPoolMax && !check && __all_sync(kFullMask, all_cols);
+  int used = 0;       // entries used; counted only under `check` (else every entry is)
+  bool have = false;  // max pooling: an entry has been combined
 
   for (int c = 0; c < nmax; c += NB) {
     int my_row[IPL];
@@ -179,8 +187,31 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
     for (int cu = 0; cu < NB; cu += U) {
       if (c + cu >= nmax) break;  // warp-uniform
       typename LD::Raw v[U][CPL];
-      bool use[U];
       float wt[U];
+      if (plain && __all_sync(kFullMask, c + cu + U <= n)) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int slot = cu + u;
+          const int r = __shfl_sync(kFullMask, my_row[slot / G], gbase + (slot % G));
+          if (POOL == kPoolWeighted)
+            wt[u] = __shfl_sync(kFullMask, my_w[slot / G], gbase + (slot % G));
+          const typename LD::Elem* row = W + static_cast<int64_t>(r) * D + col0 + q * VEC;
+#pragma unroll
+          for (int m = 0; m < CPL; ++m) v[u][m] = LD::load(row + G * m * VEC);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+          for (int m = 0; m < CPL; ++m)
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+              const float x = LD::get(v[u][m], e);
+              acc[m][e] = (POOL == kPoolSum) ? __fadd_rn(acc[m][e], x)
+                                             : __fmaf_rn(wt[u], x, acc[m][e]);
+            }
+        continue;
+      }
+      bool use[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int slot = cu + u;
@@ -192,6 +223,7 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
           const bool in_range = static_cast<unsigned>(r) < static_cast<unsigned>(rows_k);
           oob |= ok && !in_range;
           ok = ok && in_range;
+          used += ok ? 1 : 0;
         }
         use[u] = ok;
         const typename LD::Elem* row = W + static_cast<int64_t>(r) * D + col0 + q * VEC;
@@ -207,7 +239,7 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
         // at +0.0 and never becomes -0.0 under round-to-nearest, so adding +0.0
         // leaves it unchanged, bit for bit, and no branch is needed.
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
+        for (int u = 0; u < U; ++u)
 #pragma unroll
           for (int m = 0; m < CPL; ++m)
 #pragma unroll
@@ -216,8 +248,6 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
               acc[m][e] = (POOL == kPoolSum) ? __fadd_rn(acc[m][e], x)
                                              : __fmaf_rn(wt[u], x, acc[m][e]);
             }
-          used += use[u] ? 1 : 0;
-        }
       } else {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -227,15 +257,15 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
 #pragma unroll
               for (int e = 0; e < VEC; ++e) {
                 const float x = LD::get(v[u][m], e);
-                acc[m][e] = (used == 0) ? x : ((x > acc[m][e]) ? x : acc[m][e]);
+                acc[m][e] = have ? ((x > acc[m][e]) ? x : acc[m][e]) : x;
               }
-            ++used;
+            have = true;
           }
         }
       }
     }
   }
-  return used;
+  return check ? used : n;
 }
 
 // Mean pooling: one division of the sequential sum by the entries used.
