@@ -54,6 +54,12 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-depth", type=int, default=4,
                     help="batches in flight on the end-to-end host pipeline (one stream each)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tables", choices=["f32", "bf16"], default="f32",
+                    help="table element type (bf16: rows widened exactly, pooled in f32)")
+    ap.add_argument("--pool", choices=["sum", "mean", "max"], default="sum")
+    ap.add_argument("--weighted", action="store_true", help="per-sample weights (sum mode)")
+    ap.add_argument("--ragged", action="store_true",
+                    help="bag lengths drawn uniformly from [0, 2L] (same total entries)")
     ap.add_argument("--sweep", action="store_true",
                     help="time the fused stage on the 11 x 5 batch x table-count sweep instead")
     ap.add_argument("--mlp", action="store_true",
@@ -83,11 +89,13 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
-def algorithmic_bytes(w: syn.Workload, write_pooled: bool = True) -> int:
-    """Bytes the fused step must move once: rows, indices, offsets, dense, outputs."""
+def algorithmic_bytes(w: syn.Workload, write_pooled: bool = True, esz: int = 4,
+                      weighted: bool = False) -> int:
+    """Bytes the fused step must move once: rows (esz bytes per element),
+    indices, per-sample weights, offsets, dense, outputs."""
     B, F, L, D, P = w.B, w.F, w.L, w.D, w.P
-    rows = B * F * L * D * 4
-    idx = B * F * L * 4
+    rows = B * F * L * D * esz
+    idx = B * F * L * 4 * (2 if weighted else 1)
     offs = B * F * 4
     dense = B * D * 4
     pooled = B * F * D * 4 if write_pooled else 0
@@ -313,11 +321,23 @@ def run_reference(args, w: syn.Workload):
     return 0
 
 
-def workload_config(w: syn.Workload, n: int):
-    return {"workload": w.name, "B": w.B, "F": w.F, "N": w.N, "D": w.D, "L": w.L,
+def workload_config(w: syn.Workload, n: int, args=None):
+    tables = getattr(args, "tables", "f32")
+    pool = getattr(args, "pool", "sum")
+    weighted = getattr(args, "weighted", False)
+    ragged = getattr(args, "ragged", False)
+    name = w.name
+    extra = [x for x in (tables if tables != "f32" else "", pool if pool != "sum" else "",
+                         "weighted" if weighted else "", "ragged" if ragged else "") if x]
+    if extra:
+        name = name + "_" + "_".join(extra)
+    return {"workload": name, "B": w.B, "F": w.F, "N": w.N, "D": w.D, "L": w.L,
+            "tables": f"{tables} (rows widened to f32)" if tables != "f32" else "f32",
+            "pooling": pool + (" with per-sample weights" if weighted else ""),
             "index_dist": (f"zipf(alpha={w.alpha}) over rows, rank->row permuted"
                            if w.dist == "zipf" else "uniform"),
-            "offsets": "fixed stride b*L",
+            "offsets": ("ragged: sorted uniform cut points, mean length L" if ragged
+                        else "fixed stride b*L"),
             "outputs": "pooled (B,F,D) f32 + interaction (B,%s) f32" %
                        ("D+P" if w.concat_dense else "P"),
             "l2": "flushed before every step (256 MiB write outside the per-step events)",
@@ -343,19 +363,30 @@ def run_ours(args, w: syn.Workload):
 
     # inputs resident in HBM before timing: tables, this replica's batch, outputs
     weights = syn.make_weights(w, dev)
+    if args.tables == "bf16":
+        weights = [t.to(torch.bfloat16) for t in weights]
+        torch.cuda.empty_cache()
     idx_np = syn.make_indices(w, replica=rank)
-    off_np = syn.make_offsets(w)
+    off_np = syn.make_ragged_offsets(w) if args.ragged else syn.make_offsets(w)
     idx = torch.from_numpy(idx_np).to(dev)
     off = torch.from_numpy(off_np).to(dev)
     dense = syn.make_dense(w, dev)
+    psw = torch.from_numpy(syn.make_sample_weights(w)).to(dev) if args.weighted else None
+    general = args.tables != "f32" or args.pool != "sum" or args.weighted or args.ragged
     pooled = torch.empty((w.B, w.F, w.D), dtype=torch.float32, device=dev)
     inter = torch.empty((w.B, (w.D + w.P) if w.concat_dense else w.P), dtype=torch.float32,
                         device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
 
-    call = ops.SparseInteractCall(weights, idx, off, dense, w.L, concat_dense=w.concat_dense,
-                                  pooled_out=pooled, inter_out=inter)
+    if general:
+        call = ops.PoolInteractCall(weights, idx, off, dense, mode=args.pool,
+                                    per_sample_weights=psw, concat_dense=w.concat_dense,
+                                    pooled_out=pooled, inter_out=inter)
+    else:
+        call = ops.SparseInteractCall(weights, idx, off, dense, w.L,
+                                      concat_dense=w.concat_dense, pooled_out=pooled,
+                                      inter_out=inter)
     stream = torch.cuda.current_stream().cuda_stream
 
     def step():
@@ -408,7 +439,7 @@ def run_ours(args, w: syn.Workload):
     # (tables 8 GB > L2) on a double-buffered two-stream pipeline, so one
     # batch's copies overlap another's kernel; the region is timed with events.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not general:
         pipe = ops.HostPipeline(weights, w.B, w.L, concat_dense=w.concat_dense, want_pooled=True,
                                 depth=args.e2e_depth)
         batches = []
@@ -452,15 +483,17 @@ def run_ours(args, w: syn.Workload):
             peak, peak_src = float(peaks["hbm_gbs"]), "measured"
         else:
             peak, peak_src = FALLBACK_HBM_GBS, "fallback"
-        per_launch = algorithmic_bytes(w)
+        per_launch = algorithmic_bytes(w, esz=2 if args.tables == "bf16" else 4,
+                                       weighted=args.weighted)
         achieved = per_launch / (ms_step / 1e3) / 1e9
-        rows_gbs = w.B * w.F * w.L * w.D * 4 / (ms_step / 1e3) / 1e9
+        rows_gbs = (w.B * w.F * w.L * w.D * (2 if args.tables == "bf16" else 4)
+                    / (ms_step / 1e3) / 1e9)
         clocks = sampler.summary()
         line = {
             "metric": METRIC, "value": value, "unit": "lookups/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic", "config": workload_config(w, world),
+            "data": "synthetic", "config": workload_config(w, world, args),
             "samples_per_s": world * args.steps * w.B / (total_ms / 1e3),
             "gather_row_gbs": rows_gbs,
             "roofline": {"bound": "hbm", "kernel": "fused_kernel (dlrm_sparse_interact)",
@@ -474,7 +507,10 @@ def run_ours(args, w: syn.Workload):
             "step_ms_p50": statistics.median(per), "step_ms_min": min(per),
             "e2e": e2e,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if general:
+            line["e2e"] = None
+            line["e2e_note"] = "end-to-end host path covers the fixed-stride f32 sum stage only"
+        if world == 1 and not args.no_cpu_baseline and not general:
             line["cpu_baseline"] = cpu_baseline(w, weights, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if world > 1:

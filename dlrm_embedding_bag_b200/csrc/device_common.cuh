@@ -168,8 +168,10 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
     all_cols = all_cols && colok[m];
   }
   // Batches that every bag of the warp covers entirely, with every column
-  // chunk in range and no index check, take a path with no predicates.
-  const bool plain = POOL != kPoolMax && !check && __all_sync(kFullMask, all_cols);
+  // chunk in range and no index check, take a path with no predicates (for
+  // max pooling, `have` is the same in every lane of such a batch: all bags of
+  // the warp have had the same number of entries combined so far).
+  const bool plain = !check && __all_sync(kFullMask, all_cols);
   int used = 0;       // entries used; counted only under `check` (else every entry is)
   bool have = false;  // max pooling: an entry has been combined
 
@@ -206,9 +208,15 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
               const float x = LD::get(v[u][m], e);
-              acc[m][e] = (POOL == kPoolSum) ? __fadd_rn(acc[m][e], x)
-                                             : __fmaf_rn(wt[u], x, acc[m][e]);
+              if constexpr (POOL == kPoolMax) {
+                // the bag's first entry starts the maximum (warp-uniform test)
+                acc[m][e] = (u == 0 && !have) ? x : ((x > acc[m][e]) ? x : acc[m][e]);
+              } else {
+                acc[m][e] = (POOL == kPoolSum) ? __fadd_rn(acc[m][e], x)
+                                               : __fmaf_rn(wt[u], x, acc[m][e]);
+              }
             }
+        have = true;
         continue;
       }
       bool use[U];

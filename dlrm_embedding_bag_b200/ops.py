@@ -365,6 +365,42 @@ class SparseInteractCall:
         return self.pooled, self.inter
 
 
+class PoolInteractCall:
+    """A prepared ``dlrm_sparse_interact_pool`` call (general bags, modes, bf16
+    tables) on fixed buffers: checked and marshalled once, one C call each time."""
+
+    def __init__(self, weights: Sequence[torch.Tensor], indices: torch.Tensor,
+                 offsets: torch.Tensor, dense: torch.Tensor, *, mode: str = "sum",
+                 per_sample_weights: Optional[torch.Tensor] = None,
+                 include_last_offset: bool = False, concat_dense: bool = False,
+                 pooled_out=None, inter_out=None, want_pooled: bool = True):
+        arr, dt, rows, bags, F, D, B = _general_args(weights, indices, offsets, mode,
+                                                     per_sample_weights, include_last_offset,
+                                                     False)
+        if tuple(dense.shape) != (B, D):
+            raise ValueError(f"dense must be ({B}, {D})")
+        P = (F + 1) * F // 2
+        dev = weights[0].device
+        if want_pooled and pooled_out is None:
+            pooled_out = torch.empty((B, F, D), dtype=torch.float32, device=dev)
+        if inter_out is None:
+            inter_out = torch.empty((B, D + P if concat_dense else P), dtype=torch.float32,
+                                    device=dev)
+        pp = _dev(pooled_out, "pooled_out", torch.float32) if pooled_out is not None else None
+        self._keep = (list(weights), indices, offsets, dense, per_sample_weights, bags)
+        self.pooled, self.inter = pooled_out, inter_out
+        self._args = (arr, dt, rows, ctypes.byref(bags), _dev(dense, "dense", torch.float32), B,
+                      F, D, pp, _dev(inter_out, "inter_out", torch.float32),
+                      1 if concat_dense else 0, None)
+        self._fn = _lib.dlrm_sparse_interact_pool
+
+    def __call__(self, stream: Optional[int] = None):
+        rc = self._fn(*self._args, _stream() if stream is None else stream)
+        if rc != 0:
+            raise DlrmError(rc, "dlrm_sparse_interact_pool")
+        return self.pooled, self.inter
+
+
 def _host(t: torch.Tensor, name: str, dtype: torch.dtype) -> int:
     if t.device.type != "cpu" or t.dtype != dtype or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous {dtype} CPU tensor")

@@ -200,3 +200,26 @@ def make_dense_features(B: int, device="cpu", seed: int = 5000):
     out = torch.empty((B, 16), dtype=torch.bfloat16, device=device)[:, :DENSE_FEATURES]
     out.copy_(x.to(torch.bfloat16))
     return out
+
+
+def make_ragged_offsets(w: Workload) -> np.ndarray:
+    """``(F, B)`` int32 offsets of ragged bags over the same ``B*L`` entries per
+    table: bag starts are sorted uniform draws on ``[0, B*L]`` with the first at 0
+    (mean length L, lengths from 0 upward), table ``k`` from ``PCG64(6000 + k)``."""
+    T = w.B * w.L
+    off = np.empty((w.F, w.B), dtype=np.int32)
+    for k in range(w.F):
+        rng = np.random.Generator(np.random.PCG64(6000 + k))
+        cuts = np.sort(rng.integers(0, T + 1, size=w.B - 1))
+        off[k, 0] = 0
+        off[k, 1:] = cuts
+    return off
+
+
+def make_sample_weights(w: Workload) -> np.ndarray:
+    """``(F, B*L)`` f32 per-sample weights, uniform on [0, 1), ``PCG64(7000 + k)``."""
+    out = np.empty((w.F, w.B * w.L), dtype=np.float32)
+    for k in range(w.F):
+        out[k] = np.random.Generator(np.random.PCG64(7000 + k)).random(w.B * w.L,
+                                                                        dtype=np.float32)
+    return out
