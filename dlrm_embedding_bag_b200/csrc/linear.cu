@@ -163,11 +163,19 @@ __global__ void __launch_bounds__(kLinThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tslot;
   const int nkb = args.nkb_lo + args.nkb_hi;
+  // A dependent kernel may be scheduled now; it waits for this grid's results
+  // before reading them (griddepcontrol.wait above), and its CTAs only take an
+  // SM once one of these has left it.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   bool timed_out = false;
 
   if (warp == 0) {
     if (lane == 0) {
-      // TMA producer: a continuous K-block stream over this CTA's tiles.
+      // TMA producer: a continuous K-block stream over this CTA's tiles. A may
+      // be the previous kernel's output: with programmatic dependent launch
+      // this kernel can start while that one finishes, so wait for it here
+      // (a no-op without such a dependency).
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       int g = 0;
       for (int t = blockIdx.x; t < args.tiles && !timed_out; t += gridDim.x) {
         const int m0 = (t / args.tiles_n) * kLinBM, n0 = (t % args.tiles_n) * BN;
@@ -364,8 +372,19 @@ cudaError_t run_linear(const CUtensorMap& a_lo, const CUtensorMap& a_hi, const C
   args.tiles = static_cast<int>(tiles);
   // one CTA per SM: the shared-memory ring and the 2 x BN TMEM columns size it
   const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
-  fn<<<grid, kLinThreads, smem, stream>>>(a_lo, a_hi, w, y32, y16, args);
-  return cudaGetLastError();
+  // programmatic dependent launch: the prologue (TMEM allocation, barriers)
+  // overlaps the tail of the kernel before it on the stream
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kLinThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, a_lo, a_hi, w, y32, y16, args);
 }
 
 template <int BN>
