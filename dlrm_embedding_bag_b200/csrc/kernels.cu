@@ -161,6 +161,34 @@ int64_t interact_smem_per_sample(int F, int D) {
   return FeatLayout::make(F, D).floats_per_sample() * static_cast<int64_t>(sizeof(float));
 }
 
+// Samples per block of the fused kernel. A block's S*F bags go to its lane
+// groups in rounds; measured on B200, blocks do best with at least two bags per
+// lane group and little idle time in the last round (B=2048, F=32, D=64: S=1;
+// F=8: S=4; B=65536, F=26, D=128: S=2, 12 % faster than S=1), while blocks too
+// large for four to share an SM lose more than they gain. So: the smallest S
+// up to 4 with >= 2 bags per group, >= 90 % of the rounds' slots used and four
+// blocks' shared memory fitting an SM; else the S with the best product of slot
+// use and resident blocks.
+static int fused_samples_per_block(int F, int D, int B, int groups) {
+  const int64_t per = interact_smem_per_sample(F, D);
+  const int64_t sm_bytes = 228 * 1024;
+  int best_s = 1;
+  double best = -1.0;
+  for (int s = 1; s <= 4 && s <= B; ++s) {
+    const int bags = s * F;
+    const int rounds = (bags + groups - 1) / groups;
+    const double util = static_cast<double>(bags) / (static_cast<double>(rounds) * groups);
+    const int64_t resident = std::min<int64_t>(DLRM_FUSED_MIN_BLOCKS, sm_bytes / (s * per + 1024));
+    if (bags >= 2 * groups && util >= 0.9 && resident >= DLRM_FUSED_MIN_BLOCKS) return s;
+    const double score = util * static_cast<double>(resident) / DLRM_FUSED_MIN_BLOCKS;
+    if (score > best + 1e-9) {
+      best = score;
+      best_s = s;
+    }
+  }
+  return best_s;
+}
+
 #ifndef DLRM_FUSED_LQ_MAX
 #define DLRM_FUSED_LQ_MAX 4
 #endif
@@ -372,11 +400,9 @@ cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_
   a.pooled_out = pooled_out;
   a.inter_out = inter_out;
   a.concat_dense = concat_dense;
-  // enough samples that every lane group has a bag in the gather phase
   const int groups = kBlockThreads / a.g.shape.G;
-  const int want = std::max(1, (groups + g.F - 1) / g.F);
-  choose_dot_shape(g.F, g.D, g.B, std::min(want, 16), std::min<int64_t>(smem_limit, 64 * 1024),
-                   a.S, a.lq);
+  const int want = fused_samples_per_block(g.F, g.D, g.B, groups);
+  choose_dot_shape(g.F, g.D, g.B, want, std::min<int64_t>(smem_limit, 64 * 1024), a.S, a.lq);
   a.smem = a.S * interact_smem_per_sample(g.F, g.D);
   if (a.smem > smem_limit) return cudaErrorInvalidValue;
   switch (g.loader) {

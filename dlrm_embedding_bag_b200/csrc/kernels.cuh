@@ -15,9 +15,6 @@ namespace dlrm {
 #ifndef DLRM_GATHER_MIN_BLOCKS
 #define DLRM_GATHER_MIN_BLOCKS 4
 #endif
-#ifndef DLRM_FUSED_MIN_BLOCKS
-#define DLRM_FUSED_MIN_BLOCKS 4
-#endif
 constexpr int kRowsInFlight = DLRM_ROWS_IN_FLIGHT;
 constexpr int kGatherMinBlocks = DLRM_GATHER_MIN_BLOCKS;
 constexpr int kFusedMinBlocks = DLRM_FUSED_MIN_BLOCKS;

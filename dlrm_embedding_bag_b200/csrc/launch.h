@@ -9,6 +9,11 @@
 
 namespace dlrm {
 
+// Blocks of the fused kernel that the register allocation keeps resident per SM.
+#ifndef DLRM_FUSED_MIN_BLOCKS
+#define DLRM_FUSED_MIN_BLOCKS 4
+#endif
+
 // Which row loader a launch uses.
 enum LoaderKind { kLdF32x4 = 0, kLdF32x1 = 1, kLdBF16x8 = 2, kLdBF16x1 = 3 };
 
