@@ -90,6 +90,7 @@ int prepare(const void* const* weights, int dtype, const int64_t* rows, const dl
   pr->bp.mean = bags->mode == DLRM_POOL_MEAN ? 1 : 0;
   pr->bp.check = rows != nullptr ? 1 : 0;
   pr->bp.status = status_dev;
+  pr->bp.balance = 0;
   pr->pool = bags->per_sample_weights ? dlrm::kPoolWeighted
              : bags->mode == DLRM_POOL_MAX ? dlrm::kPoolMax
                                           : dlrm::kPoolSum;
@@ -160,10 +161,12 @@ int pool_impl(const void* const* weights, int dtype, const int64_t* rows, const 
 int fused_impl(const void* const* weights, int dtype, const int64_t* rows,
                const dlrm_bags_t* bags, const float* dense, int B, int F, int D,
                float* pooled_out, float* inter_out, int concat_dense, int32_t* status_dev,
-               cudaStream_t stream) {
+               bool fixed_stride, cudaStream_t stream) {
   Prepared pr;
   int rc = prepare(weights, dtype, rows, bags, B, F, D, status_dev, &pr);
   if (rc != DLRM_OK) return rc;
+  // bags of any lengths: the fused kernel orders each block's bags by length
+  pr.bp.balance = fixed_stride ? 0 : 1;
   if (dense == nullptr || inter_out == nullptr) return DLRM_ERR_NULL;
   if (!aligned(dense, 4) || !aligned(inter_out, 4) || (pooled_out && !aligned(pooled_out, 4)))
     return DLRM_ERR_ALIGN;
@@ -256,7 +259,7 @@ int dlrm_sparse_interact(const float* const* weights, const int32_t* indices,
   int rc = fixed_stride_bags(indices, offsets, B, L, &bags);
   if (rc != DLRM_OK) return rc;
   return fused_impl(as_void(weights), DLRM_TABLE_F32, nullptr, &bags, dense, B, F, D,
-                    pooled_out, inter_out, concat_dense, nullptr,
+                    pooled_out, inter_out, concat_dense, nullptr, true,
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -270,7 +273,8 @@ int dlrm_sparse_interact_ex(const float* const* weights, const int64_t* rows,
   int rc = fixed_stride_bags(indices, offsets, B, L, &bags);
   if (rc != DLRM_OK) return rc;
   return fused_impl(as_void(weights), DLRM_TABLE_F32, rows, &bags, dense, B, F, D, pooled_out,
-                    inter_out, concat_dense, status_dev, reinterpret_cast<cudaStream_t>(stream));
+                    inter_out, concat_dense, status_dev, true,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dlrm_sparse_interact_pool(const void* const* weights, int table_dtype, const int64_t* rows,
@@ -278,7 +282,7 @@ int dlrm_sparse_interact_pool(const void* const* weights, int table_dtype, const
                               float* pooled_out, float* inter_out, int concat_dense,
                               int32_t* status_dev, dlrm_stream_t stream) {
   return fused_impl(weights, table_dtype, rows, bags, dense, B, F, D, pooled_out, inter_out,
-                    concat_dense, status_dev, reinterpret_cast<cudaStream_t>(stream));
+                    concat_dense, status_dev, false, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dlrm_sparse_interact_host(const float* const* weights, const int32_t* indices_host,

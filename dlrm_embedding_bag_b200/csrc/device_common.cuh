@@ -30,6 +30,7 @@ struct BagParams {
   int mean;                // divide each pooled sum by the bag's entry count
   int check;               // skip (and flag) indices outside [0, rows[k])
   int32_t* status;         // device flags, or null
+  int balance;             // fused kernel: order each block's bags by length
 };
 
 // Pooling combine step, fixed per template instance.
@@ -122,6 +123,27 @@ __device__ __forceinline__ void pair_from_flat_small(int p, int& i_out, int& j_o
 // where the next one starts, or at T for the last bag (include_last_offset=0),
 // or at offsets[k][B] (include_last_offset=1). Invalid bounds give an empty
 // bag and raise *bad.
+// Sort keys of the fused kernel's bag ordering: (length + 1) << 11 | bag.
+constexpr int kSortTaskBits = 11;  // bags per block < 2048
+constexpr int kSortLenMax = (1 << (32 - kSortTaskBits)) - 2;
+
+// Sorts one key per lane across the warp, largest at lane 0: Batcher's
+// bitonic network, log2(32) merge phases of shuffle-exchange steps. In phase
+// k the runs of k lanes alternate direction so that each pair of runs forms a
+// bitonic sequence for the next phase; the last phase runs one direction.
+__device__ __forceinline__ unsigned warp_sort_desc(unsigned key, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const unsigned other = __shfl_xor_sync(kFullMask, key, j);
+      const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+      key = keep_max ? max(key, other) : min(key, other);
+    }
+  }
+  return key;
+}
+
 __device__ __forceinline__ void bag_bounds(const BagParams& bp, int B, int k, int b, int& start,
                                            int& n, bool& bad) {
   const int64_t o = static_cast<int64_t>(k) * (B + bp.ilo) + b;
@@ -188,21 +210,24 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
 #pragma unroll
     for (int cu = 0; cu < NB; cu += U) {
       if (c + cu >= nmax) break;  // warp-uniform
+      // Weights are handed out at combine time (not with the row loads), so
+      // U of them need not stay live across the loads.
       typename LD::Raw v[U][CPL];
-      float wt[U];
       if (plain && __all_sync(kFullMask, c + cu + U <= n)) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
           const int slot = cu + u;
           const int r = __shfl_sync(kFullMask, my_row[slot / G], gbase + (slot % G));
-          if (POOL == kPoolWeighted)
-            wt[u] = __shfl_sync(kFullMask, my_w[slot / G], gbase + (slot % G));
           const typename LD::Elem* row = W + static_cast<int64_t>(r) * D + col0 + q * VEC;
 #pragma unroll
           for (int m = 0; m < CPL; ++m) v[u][m] = LD::load(row + G * m * VEC);
         }
 #pragma unroll
-        for (int u = 0; u < U; ++u)
+        for (int u = 0; u < U; ++u) {
+          const int slot = cu + u;
+          float wt = 0.f;
+          if (POOL == kPoolWeighted)
+            wt = __shfl_sync(kFullMask, my_w[slot / G], gbase + (slot % G));
 #pragma unroll
           for (int m = 0; m < CPL; ++m)
 #pragma unroll
@@ -213,19 +238,18 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
                 acc[m][e] = (u == 0 && !have) ? x : ((x > acc[m][e]) ? x : acc[m][e]);
               } else {
                 acc[m][e] = (POOL == kPoolSum) ? __fadd_rn(acc[m][e], x)
-                                               : __fmaf_rn(wt[u], x, acc[m][e]);
+                                               : __fmaf_rn(wt, x, acc[m][e]);
               }
             }
+        }
         have = true;
         continue;
       }
-      bool use[U];
+      bool use[U];  // entry cu + u is combined
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int slot = cu + u;
         const int r = __shfl_sync(kFullMask, my_row[slot / G], gbase + (slot % G));
-        if (POOL == kPoolWeighted)
-          wt[u] = __shfl_sync(kFullMask, my_w[slot / G], gbase + (slot % G));
         bool ok = (c + slot) < n;
         if (check) {
           const bool in_range = static_cast<unsigned>(r) < static_cast<unsigned>(rows_k);
@@ -240,22 +264,28 @@ __device__ __forceinline__ int pool_bag(const typename LD::Elem* __restrict__ W,
           v[u][m] = LD::zero();
           if (ok && colok[m]) v[u][m] = LD::load(row + G * m * VEC);
         }
-        if (POOL == kPoolWeighted) wt[u] = ok ? wt[u] : 0.f;
       }
       if (POOL != kPoolMax) {
         // A skipped entry adds +0.0 (weight 0 times 0): the running sum starts
         // at +0.0 and never becomes -0.0 under round-to-nearest, so adding +0.0
         // leaves it unchanged, bit for bit, and no branch is needed.
 #pragma unroll
-        for (int u = 0; u < U; ++u)
+        for (int u = 0; u < U; ++u) {
+          const int slot = cu + u;
+          float wt = 0.f;
+          if (POOL == kPoolWeighted) {
+            wt = __shfl_sync(kFullMask, my_w[slot / G], gbase + (slot % G));
+            wt = use[u] ? wt : 0.f;
+          }
 #pragma unroll
           for (int m = 0; m < CPL; ++m)
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
               const float x = LD::get(v[u][m], e);
               acc[m][e] = (POOL == kPoolSum) ? __fadd_rn(acc[m][e], x)
-                                             : __fmaf_rn(wt[u], x, acc[m][e]);
+                                             : __fmaf_rn(wt, x, acc[m][e]);
             }
+        }
       } else {
 #pragma unroll
         for (int u = 0; u < U; ++u) {

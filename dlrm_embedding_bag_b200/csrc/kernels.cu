@@ -169,16 +169,20 @@ int64_t interact_smem_per_sample(int F, int D) {
 // up to 4 with >= 2 bags per group, >= 90 % of the rounds' slots used and four
 // blocks' shared memory fitting an SM; else the S with the best product of slot
 // use and resident blocks.
-static int fused_samples_per_block(int F, int D, int B, int groups) {
+#ifndef DLRM_FUSED_MAX_S
+#define DLRM_FUSED_MAX_S 4
+#endif
+static int fused_samples_per_block(int F, int D, int B, int groups, int64_t extra_per_block) {
   const int64_t per = interact_smem_per_sample(F, D);
   const int64_t sm_bytes = 228 * 1024;
   int best_s = 1;
   double best = -1.0;
-  for (int s = 1; s <= 4 && s <= B; ++s) {
+  for (int s = 1; s <= DLRM_FUSED_MAX_S && s <= B; ++s) {
     const int bags = s * F;
     const int rounds = (bags + groups - 1) / groups;
     const double util = static_cast<double>(bags) / (static_cast<double>(rounds) * groups);
-    const int64_t resident = std::min<int64_t>(DLRM_FUSED_MIN_BLOCKS, sm_bytes / (s * per + 1024));
+    const int64_t resident = std::min<int64_t>(DLRM_FUSED_MIN_BLOCKS,
+                                               sm_bytes / (s * per + extra_per_block + 1024));
     if (bags >= 2 * groups && util >= 0.9 && resident >= DLRM_FUSED_MIN_BLOCKS) return s;
     const double score = util * static_cast<double>(resident) / DLRM_FUSED_MIN_BLOCKS;
     if (score > best + 1e-9) {
@@ -401,9 +405,13 @@ cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_
   a.inter_out = inter_out;
   a.concat_dense = concat_dense;
   const int groups = kBlockThreads / a.g.shape.G;
-  const int want = fused_samples_per_block(g.F, g.D, g.B, groups);
-  choose_dot_shape(g.F, g.D, g.B, want, std::min<int64_t>(smem_limit, 64 * 1024), a.S, a.lq);
-  a.smem = a.S * interact_smem_per_sample(g.F, g.D);
+  // the bag ordering keeps 96 ints per warp after the features
+  const int64_t order_bytes = a.g.bp.balance ? (kBlockThreads / 32) * 96 * sizeof(int) : 0;
+  const int want = fused_samples_per_block(g.F, g.D, g.B, groups, order_bytes);
+  choose_dot_shape(g.F, g.D, g.B, want, std::min<int64_t>(smem_limit, 64 * 1024) - order_bytes,
+                   a.S, a.lq);
+  if (a.S * g.F >= (1 << kSortTaskBits)) a.g.bp.balance = 0;
+  a.smem = a.S * interact_smem_per_sample(g.F, g.D) + (a.g.bp.balance ? order_bytes : 0);
   if (a.smem > smem_limit) return cudaErrorInvalidValue;
   switch (g.loader) {
     case kLdF32x4: return counted(launch_fused_f32x4(a));

@@ -112,15 +112,67 @@ __global__ void __launch_bounds__(kBlockThreads, kFusedMinBlocks)
   bool oob = false, bad_any = false;
   const int ntasks = S_here * F;
   const int rounds = (S * F + kGroups - 1) / kGroups;
+  // Bags of different lengths: a warp runs to its longest bag and the block to
+  // its slowest warp. So the block's bags are taken in runs of 32; a warp
+  // reads the bounds of the run that holds its slots, sorts the run longest
+  // first (key: length, then bag number, so keys are unique; a run of equal
+  // lengths keeps its order), and the rounds walk the sorted runs in
+  // alternating direction: the lane groups of a warp get bags of similar
+  // length, and a warp that drew long bags in one round draws short ones in
+  // the next. Every warp sorts the same runs the same way, so no block-wide
+  // barrier is needed; each warp keeps its sorted run in its own 96 ints of
+  // shared memory after the features (rank r: bag, start, length).
+  const int group = static_cast<int>(threadIdx.x) / G;
   for (int rd = 0; rd < rounds; ++rd) {
-    const int task = rd * kGroups + static_cast<int>(threadIdx.x) / G;
-    const bool active = task < ntasks;
+    const int slot = rd * kGroups + ((bp.balance && (rd & 1)) ? kGroups - 1 - group : group);
+    const bool active = slot < ntasks;
+    int task = slot, start = 0, n = 0;
+    if (bp.balance) {
+      // all slots of a warp in a round lie in one run of 32 (warp-uniform);
+      // the run is (re)sorted when it differs from the previous round's
+      const int g0 = static_cast<int>(threadIdx.x - lane) / G;
+      const auto run_of = [&](int r) { return (r * kGroups + ((r & 1) ? kGroups - 1 - g0 : g0)) >> 5; };
+      const int run = run_of(rd);
+      const int prev = rd == 0 ? -1 : run_of(rd - 1);
+      int* run_sorted = reinterpret_cast<int*>(feat + static_cast<int64_t>(S) * sample_floats) +
+                        (threadIdx.x >> 5) * 96;
+      if (run != prev) {
+        const int t = (run << 5) + lane;
+        int st = 0, len = 0;
+        unsigned key = 0;  // below every real key: empty slots sort last
+        if (t < ntasks) {
+          const int s = t / F;
+          bool bad;
+          bag_bounds(bp, B, t - s * F, static_cast<int>(b0 + s), st, len, bad);
+          bad_any |= bad;
+          key = ((static_cast<unsigned>(min(len, kSortLenMax)) + 1u) << kSortTaskBits) |
+                static_cast<unsigned>(t);
+        }
+        const int len0 = __shfl_sync(kFullMask, len, 0);
+        if (!__all_sync(kFullMask, t >= ntasks || len == len0)) key = warp_sort_desc(key, lane);
+        const int tr = static_cast<int>(key & ((1u << kSortTaskBits) - 1u));
+        const int st_r = __shfl_sync(kFullMask, st, tr & 31);
+        const int len_r = __shfl_sync(kFullMask, len, tr & 31);
+        __syncwarp();  // the previous run's reads are done
+        run_sorted[lane] = tr;
+        run_sorted[32 + lane] = st_r;
+        run_sorted[64 + lane] = len_r;
+        __syncwarp();
+      }
+      if (active) {
+        const int r = slot & 31;
+        task = run_sorted[r];
+        start = run_sorted[32 + r];
+        n = run_sorted[64 + r];
+      }
+    } else if (active) {
+      const int s = task / F;
+      bool bad = false;
+      bag_bounds(bp, B, task - s * F, static_cast<int>(b0 + s), start, n, bad);
+      bad_any |= bad;
+    }
     const int s = active ? task / F : 0;
     const int k = active ? task - s * F : 0;
-    int start = 0, n = 0;
-    bool bad = false;
-    if (active) bag_bounds(bp, B, k, static_cast<int>(b0 + s), start, n, bad);
-    bad_any |= bad;
     const int nmax = __reduce_max_sync(kFullMask, n);
     const Elem* W = static_cast<const Elem*>(tp.w[k]);
     const int32_t* idx_seg = bp.indices + static_cast<int64_t>(k) * bp.T;

@@ -77,6 +77,7 @@ SHAPES = [  # (B, F, N, D, T)
     (11, 3, 25, 7, 40),       # both scalar
     (6, 2, 20, 264, 30),      # two column windows
     (70, 26, 500, 64, 2000),
+    (10, 100, 30, 16, 120),   # fused: 3 samples x 100 bags per block, > 256 bags to order
 ]
 VARIANTS = [("sum", False), ("sum", True), ("mean", False), ("max", False)]
 
@@ -155,6 +156,55 @@ def test_checked_general_pooling_skips_bad_indices(ops, mode):
     ref = oracle.embbag_pool_multi([w.cpu().numpy() for w in weights], new_idx, new_off, B,
                                    mode=mode, include_last_offset=True)
     assert_bits_equal(out, ref, f"checked {mode}")
+
+
+@pytest.mark.parametrize("mode", ["sum", "mean"])
+def test_general_bad_offsets_flagged(ops, mode):
+    """Bags whose bounds break start <= end, start >= 0 or end <= T pool as
+    empty and raise FLAG_OFFSETS, through the gather and the fused entry
+    points; every other bag (and every dot) is exact."""
+    B, F, N, D, T = 40, 5, 60, 64, 300
+    weights, idx, off, _, dense = _case(41, B, F, N, D, T, torch.float32, False, 0.0)
+    off_bad = off.copy()
+    off_bad[1, 7] = off_bad[1, 8] + 1   # bag 7 of table 1: start > end
+    off_bad[3, 0] = -1                  # bag 0 of table 3: start < 0
+    off_bad[4, B - 1] = T + 1           # last bag of table 4: start > T
+    # expected: each valid bag's entries, laid out again back to back
+    idx2 = np.zeros((F, T + 1), np.int32)
+    off2 = np.zeros((F, B + 1), np.int32)
+    bad_bags = []
+    for k in range(F):
+        pos = 0
+        for b in range(B):
+            st = int(off_bad[k, b])
+            en = int(off_bad[k, b + 1]) if b + 1 < B else T
+            off2[k, b] = pos
+            if st < 0 or st > en or en > T:
+                bad_bags.append((b, k))
+                continue
+            idx2[k, pos:pos + en - st] = idx[k, st:en]
+            pos += en - st
+        off2[k, B] = pos
+    assert len(bad_bags) >= 3
+    ws = [_host_bits(w) for w in weights]
+    ref = oracle.embbag_pool_multi(ws, idx2, off2, B, mode=mode, include_last_offset=True)
+    idx_d = torch.from_numpy(idx).to(DEV)
+    off_d = torch.from_numpy(off_bad).to(DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = ops.embbag_pool_multi(weights, idx_d, off_d, mode=mode, checked=True, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == ops.FLAG_OFFSETS
+    assert_bits_equal(out, ref, f"gather, bad offsets, {mode}")
+    status.zero_()
+    fp, fi = ops.sparse_interact_pool(weights, idx_d, off_d, dense, mode=mode, checked=True,
+                                      status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == ops.FLAG_OFFSETS
+    assert_bits_equal(fp, ref, f"fused, bad offsets, {mode}")
+    for b, k in bad_bags:
+        assert torch.count_nonzero(fp[b, k]) == 0
+    ref_i, _, bound = oracle.interact_lower_tri(dense.cpu().numpy(), ref, with_f64=True)
+    assert_dots_close(fi, ref_i, bound, f"fused dots, bad offsets, {mode}")
 
 
 def test_bf16_full_size_sampled(ops):
