@@ -7,7 +7,7 @@
 // t = c, c + gridDim.x, ... (N tiles fastest, so CTAs running side by side
 // share A rows in L2). Ten warps:
 //   - warp 0 (one thread) streams 64-wide K blocks of A (128 x 64 bf16) and W
-//     (BN x 64) into a 4-stage shared-memory ring with 2-D TMA loads (128-byte
+//     (BN x 64) into a 3- or 4-stage shared-memory ring with 2-D TMA loads (128-byte
 //     swizzle), running ahead across tiles; K blocks 0..nkb_lo-1 read A_lo,
 //     the rest read A_hi, and W's column offset follows, so the
 //     concatenation is never built;
@@ -38,24 +38,26 @@ namespace {
 
 constexpr int kLinBM = 128;    // rows of a tile (tcgen05 M)
 constexpr int kLinBK = 64;     // K per stage: 64 bf16 = one 128-byte swizzle row
-// shared-memory ring depth (3 with 256-column tiles, whose stages are 48 KB)
-template <int BN>
-constexpr int lin_stages() { return BN >= 256 ? 3 : 4; }
+// Shared-memory ring depth: 4 stages, except with 256-column tiles (48 KB
+// stages) next to the f32 output staging, where only 3 fit.
+template <int BN, bool F32S>
+constexpr int lin_stages() { return (BN >= 256 && F32S) ? 3 : 4; }
 constexpr int kLinEpiWarps = 8;  // two per TMEM lane quarter, each half of the columns
 constexpr int kLinThreads = 64 + 32 * kLinEpiWarps;  // producer warp, MMA warp, epilogue
 constexpr long long kLinWaitLimit = 200000000LL;  // clock cycles, about 0.1 s
 
-template <int BN>
+template <int BN, bool F32S>
 struct LinSmem {
-  static constexpr int kStages = lin_stages<BN>();
+  static constexpr int kStages = lin_stages<BN, F32S>();
   static constexpr int kA = kLinBM * kLinBK * 2;
   static constexpr int kB = BN * kLinBK * 2;
   static constexpr int kStage = kA + kB;
   // After the ring: each epilogue warp's output staging (a 32 x 32 f32 tile in
-  // the 128-byte swizzled layout, then a 32 x 32 bf16 tile in the 64-byte
-  // swizzled layout), its slice of the tile's bias, then the barriers full[S],
-  // empty[S], acc_full[2], acc_empty[2] and the TMEM slot.
-  static constexpr int kStage32 = 32 * 32 * 4;
+  // the 128-byte swizzled layout when F32S -- the f32 output goes out through
+  // TMA --, then a 32 x 32 bf16 tile in the 64-byte swizzled layout), its slice
+  // of the tile's bias, then the barriers full[S], empty[S], acc_full[2],
+  // acc_empty[2] and the TMEM slot.
+  static constexpr int kStage32 = F32S ? 32 * 32 * 4 : 0;
   static constexpr int kStage16 = 32 * 32 * 2;
   static constexpr int kStaging = kStages * kStage;
   static constexpr int kBias = kStaging + kLinEpiWarps * (kStage32 + kStage16);
@@ -124,14 +126,14 @@ __device__ __forceinline__ void store_chunk32(const LinearArgs& args, int row, i
   }
 }
 
-template <int BN, int ACT>
+template <int BN, int ACT, bool F32S>
 __global__ void __launch_bounds__(kLinThreads, 1)
     linear_bf16_kernel(const __grid_constant__ CUtensorMap map_a_lo,
                        const __grid_constant__ CUtensorMap map_a_hi,
                        const __grid_constant__ CUtensorMap map_w,
                        const __grid_constant__ CUtensorMap map_y32,
                        const __grid_constant__ CUtensorMap map_y16, const LinearArgs args) {
-  using L = LinSmem<BN>;
+  using L = LinSmem<BN, F32S>;
   constexpr uint32_t kCols = 2 * BN;  // two f32 accumulators (a power of two >= 128)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         if (tma_out) {
           if (lane == 0) bulk_wait_read_all();  // the previous block has left the staging
           __syncwarp();
-          if (args.tma_f32) {
+          if (F32S && args.tma_f32) {
             uint4* rowp = reinterpret_cast<uint4*>(st32 + lane * 128);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (args.tma_f32) tma_store_2d(&map_y32, st32, n0 + c0, row0);
+            if (F32S && args.tma_f32) tma_store_2d(&map_y32, st32, n0 + c0, row0);
             if (args.tma_bf16) tma_store_2d(&map_y16, st16, n0 + c0, row0);
             bulk_commit();
           }
@@ -357,12 +359,12 @@ cudaError_t encode_bf16_operand(CUtensorMap* map, const void* base, int64_t cols
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int BN, int ACT>
+template <int BN, int ACT, bool F32S>
 cudaError_t run_linear(const CUtensorMap& a_lo, const CUtensorMap& a_hi, const CUtensorMap& w,
                        const CUtensorMap& y32, const CUtensorMap& y16, LinearArgs args, int sms,
                        cudaStream_t stream) {
-  auto* fn = &linear_bf16_kernel<BN, ACT>;
-  constexpr int smem = LinSmem<BN>::kTotal;
+  auto* fn = &linear_bf16_kernel<BN, ACT, F32S>;
+  constexpr int smem = LinSmem<BN, F32S>::kTotal;
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -387,17 +389,28 @@ cudaError_t run_linear(const CUtensorMap& a_lo, const CUtensorMap& a_hi, const C
   return cudaLaunchKernelEx(&cfg, fn, a_lo, a_hi, w, y32, y16, args);
 }
 
-template <int BN>
+template <int BN, bool F32S>
 cudaError_t run_linear_act(int act, const CUtensorMap& a_lo, const CUtensorMap& a_hi,
                            const CUtensorMap& w, const CUtensorMap& y32, const CUtensorMap& y16,
                            const LinearArgs& args, int sms, cudaStream_t stream) {
   switch (act) {
     case DLRM_ACT_RELU:
-      return run_linear<BN, DLRM_ACT_RELU>(a_lo, a_hi, w, y32, y16, args, sms, stream);
+      return run_linear<BN, DLRM_ACT_RELU, F32S>(a_lo, a_hi, w, y32, y16, args, sms, stream);
     case DLRM_ACT_SIGMOID:
-      return run_linear<BN, DLRM_ACT_SIGMOID>(a_lo, a_hi, w, y32, y16, args, sms, stream);
-    default: return run_linear<BN, DLRM_ACT_NONE>(a_lo, a_hi, w, y32, y16, args, sms, stream);
+      return run_linear<BN, DLRM_ACT_SIGMOID, F32S>(a_lo, a_hi, w, y32, y16, args, sms, stream);
+    default:
+      return run_linear<BN, DLRM_ACT_NONE, F32S>(a_lo, a_hi, w, y32, y16, args, sms, stream);
   }
+}
+
+// The instance with f32 output staging (and, at 256 columns, a 3-stage ring)
+// only when the f32 output goes out through TMA.
+template <int BN>
+cudaError_t run_linear_bn(int act, const CUtensorMap& a_lo, const CUtensorMap& a_hi,
+                          const CUtensorMap& w, const CUtensorMap& y32, const CUtensorMap& y16,
+                          const LinearArgs& args, int sms, cudaStream_t stream) {
+  return args.tma_f32 ? run_linear_act<BN, true>(act, a_lo, a_hi, w, y32, y16, args, sms, stream)
+                      : run_linear_act<BN, false>(act, a_lo, a_hi, w, y32, y16, args, sms, stream);
 }
 
 // 2-D output map {N, M} with row pitch ld elements, box {32, 32}, written from a
@@ -506,9 +519,9 @@ DLRM_API int dlrm_linear_bf16(const uint16_t* a_lo, int64_t lda_lo, int64_t k_lo
   if (!args.tma_bf16) my16 = mw;  // never read
   auto* s = reinterpret_cast<cudaStream_t>(stream);
   switch (bn) {
-    case 256: e = run_linear_act<256>(act, ma_lo, ma_hi, mw, my32, my16, args, sms, s); break;
-    case 128: e = run_linear_act<128>(act, ma_lo, ma_hi, mw, my32, my16, args, sms, s); break;
-    default: e = run_linear_act<64>(act, ma_lo, ma_hi, mw, my32, my16, args, sms, s); break;
+    case 256: e = run_linear_bn<256>(act, ma_lo, ma_hi, mw, my32, my16, args, sms, s); break;
+    case 128: e = run_linear_bn<128>(act, ma_lo, ma_hi, mw, my32, my16, args, sms, s); break;
+    default: e = run_linear_bn<64>(act, ma_lo, ma_hi, mw, my32, my16, args, sms, s); break;
   }
   if (e != cudaSuccess) return cuda_fail(e);
   note_launch();

@@ -105,6 +105,26 @@ def test_linear_wide_tiles_sampled(M, N, K):
     _run(M, N, K, act="relu", seed=11, rows=rows)
 
 
+@pytest.mark.parametrize("M,N,K", [(20000, 512, 592), (10000, 256, 192), (20000, 200, 64),
+                                   (300, 130, 200)])
+def test_linear_bf16_only_outputs(M, N, K):
+    """A layer with only the bf16 output runs the instance without f32 output
+    staging (a deeper operand ring at 256-column tiles); its bits are the RNE
+    of the f32 results of the instance with staging, checked on sampled rows."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(M + N + K)
+    a = _rand_bf16(g, M, K)
+    w = _rand_bf16(g, N, K, K ** -0.5)
+    b = torch.empty(N, device=DEV).normal_(0, 0.5, generator=g)
+    y32, _ = mlp.linear_bf16(a, w, b, "relu")
+    _, y16 = mlp.linear_bf16(a, w, b, "relu", f32=False, bf16=True)
+    torch.cuda.synchronize()
+    rows = torch.from_numpy(np.random.default_rng(K).choice(M, min(M, 96),
+                                                            replace=False)).to(DEV)
+    _check_layer(y32, None, a, w, b, "relu", rows=rows, what=f"M={M} N={N} K={K} f32")
+    assert np.array_equal(_bits(y16), _bits(y32.to(torch.bfloat16)))
+
+
 @pytest.mark.parametrize("k_lo,k_hi", [(64, 528), (128, 351), (24, 40), (8, 8), (64, 0)])
 def test_linear_split_a(k_lo, k_hi):
     g = torch.Generator(device=DEV)
