@@ -436,8 +436,9 @@ def run_ours(args, w: syn.Workload):
     # e2e through the host-buffer entry point: every step copies its batch's
     # indices, offsets and dense rows in from pinned host memory and its
     # interaction rows back out. Steps cycle over E2E_BATCHES distinct batches
-    # (tables 8 GB > L2) on a double-buffered two-stream pipeline, so one
-    # batch's copies overlap another's kernel; the region is timed with events.
+    # (tables 8 GB > L2) on a pipeline of --e2e-depth streams, so one batch's
+    # copies overlap other batches' kernels and copies; the region is timed
+    # with events.
     e2e = None
     if not args.no_e2e and not general:
         pipe = ops.HostPipeline(weights, w.B, w.L, concat_dense=w.concat_dense, want_pooled=True,
