@@ -395,7 +395,8 @@ int64_t dlrm_launch_count(void) { return dlrm::launch_count(); }
 int dlrm_probe_bounded_wait(int64_t limit_cycles, int32_t* status_dev, dlrm_stream_t stream) {
   if (status_dev == nullptr) return DLRM_ERR_NULL;
   if (!aligned(status_dev, 4)) return DLRM_ERR_ALIGN;
-  const int64_t limit = limit_cycles < 1000 ? 1000 : (limit_cycles > 200000000 ? 200000000 : limit_cycles);
+  const int64_t limit =
+      limit_cycles < 1000 ? 1000 : (limit_cycles > 200000000 ? 200000000 : limit_cycles);
   const cudaError_t e =
       dlrm::launch_probe_wait(limit, status_dev, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DLRM_OK : cuda_fail(e);

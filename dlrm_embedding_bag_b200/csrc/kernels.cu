@@ -60,7 +60,8 @@ __global__ void __launch_bounds__(kBlockThreads, 2)
                     int D, int S, int lq, int nbuf, float* __restrict__ out) {
   extern __shared__ __align__(16) float feat[];
   const FeatLayout Lf = FeatLayout::make(F, D);
-  const int64_t bstride = (nbuf > 1) ? S * Lf.floats_per_sample() : 0;  // buffer i at feat + i*bstride
+  // buffer i at feat + i * bstride
+  const int64_t bstride = (nbuf > 1) ? S * Lf.floats_per_sample() : 0;
   const int64_t ngroups = (static_cast<int64_t>(B) + S - 1) / S;
   const int P = Lf.F1 * (Lf.F1 - 1) / 2;
   auto samples = [&](int64_t g) {

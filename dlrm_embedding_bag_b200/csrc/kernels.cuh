@@ -131,7 +131,9 @@ __global__ void __launch_bounds__(kBlockThreads, kFusedMinBlocks)
       // all slots of a warp in a round lie in one run of 32 (warp-uniform);
       // the run is (re)sorted when it differs from the previous round's
       const int g0 = static_cast<int>(threadIdx.x - lane) / G;
-      const auto run_of = [&](int r) { return (r * kGroups + ((r & 1) ? kGroups - 1 - g0 : g0)) >> 5; };
+      const auto run_of = [&](int r) {
+        return (r * kGroups + ((r & 1) ? kGroups - 1 - g0 : g0)) >> 5;
+      };
       const int run = run_of(rd);
       const int prev = rd == 0 ? -1 : run_of(rd - 1);
       int* run_sorted = reinterpret_cast<int*>(feat + static_cast<int64_t>(S) * sample_floats) +

@@ -43,7 +43,8 @@ constexpr int kPipeGatherOnlyThreads = DLRM_PIPE_ONLY_THREADS;
 template <class LD, int G, int CPL, int POOL, bool FUSED>
 struct PipeUnit {
   static constexpr int VEC = LD::VEC;
-  static constexpr int U = CPL == 1 ? DLRM_PIPE_ROWS : DLRM_PIPE_ROWS / 2;  // rows in flight per lane
+  // rows in flight per lane
+  static constexpr int U = CPL == 1 ? DLRM_PIPE_ROWS : DLRM_PIPE_ROWS / 2;
   static constexpr int IPL = (U + G - 1) / G;  // row ids held per lane per batch
   using Raw = typename LD::Raw;
   using Elem = typename LD::Elem;

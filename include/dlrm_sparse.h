@@ -145,8 +145,8 @@ typedef struct {
  * read; the _ex variant also reports it.
  */
 DLRM_API int embbag_sum_multi(const float* const* weights, const int32_t* indices,
-                     const int32_t* offsets, int B, int F, int L, int D, float* out,
-                     dlrm_stream_t stream);
+                              const int32_t* offsets, int B, int F, int L, int D, float* out,
+                              dlrm_stream_t stream);
 
 /*
  * embbag_sum_multi_ex -- embbag_sum_multi with device-side checks.
@@ -158,8 +158,9 @@ DLRM_API int embbag_sum_multi(const float* const* weights, const int32_t* indice
  *                value, once the stream has reached it, to a status.
  */
 DLRM_API int embbag_sum_multi_ex(const float* const* weights, const int64_t* rows,
-                        const int32_t* indices, const int32_t* offsets, int B, int F, int L,
-                        int D, float* out, int32_t* status_dev, dlrm_stream_t stream);
+                                 const int32_t* indices, const int32_t* offsets, int B, int F,
+                                 int L, int D, float* out, int32_t* status_dev,
+                                 dlrm_stream_t stream);
 
 /*
  * embbag_pool_multi -- the general multi-table EmbeddingBag in one launch.
@@ -194,8 +195,8 @@ DLRM_API int embbag_pool_multi(const void* const* weights, int table_dtype, cons
  * sample, at most the device's per-block limit (227 KB on B200); else
  * DLRM_ERR_SHAPE.
  */
-DLRM_API int interact_lower_tri(const float* dense, const float* emb, int B, int F, int D, float* out,
-                       dlrm_stream_t stream);
+DLRM_API int interact_lower_tri(const float* dense, const float* emb, int B, int F, int D,
+                                float* out, dlrm_stream_t stream);
 
 /*
  * dlrm_sparse_interact -- both steps in one launch. Each block gathers its
@@ -213,15 +214,16 @@ DLRM_API int interact_lower_tri(const float* dense, const float* emb, int B, int
  * Shared memory as for interact_lower_tri.
  */
 DLRM_API int dlrm_sparse_interact(const float* const* weights, const int32_t* indices,
-                         const int32_t* offsets, const float* dense, int B, int F, int L, int D,
-                         float* pooled_out, float* inter_out, int concat_dense,
-                         dlrm_stream_t stream);
+                                  const int32_t* offsets, const float* dense, int B, int F, int L,
+                                  int D, float* pooled_out, float* inter_out, int concat_dense,
+                                  dlrm_stream_t stream);
 
 /* dlrm_sparse_interact with the device-side checks of embbag_sum_multi_ex. */
 DLRM_API int dlrm_sparse_interact_ex(const float* const* weights, const int64_t* rows,
-                            const int32_t* indices, const int32_t* offsets, const float* dense,
-                            int B, int F, int L, int D, float* pooled_out, float* inter_out,
-                            int concat_dense, int32_t* status_dev, dlrm_stream_t stream);
+                                     const int32_t* indices, const int32_t* offsets,
+                                     const float* dense, int B, int F, int L, int D,
+                                     float* pooled_out, float* inter_out, int concat_dense,
+                                     int32_t* status_dev, dlrm_stream_t stream);
 
 /*
  * dlrm_sparse_interact_pool -- the fused stage with the general bag
@@ -230,9 +232,9 @@ DLRM_API int dlrm_sparse_interact_ex(const float* const* weights, const int64_t*
  */
 DLRM_API int dlrm_sparse_interact_pool(const void* const* weights, int table_dtype,
                                        const int64_t* rows, const dlrm_bags_t* bags,
-                                       const float* dense, int B, int F, int D,
-                                       float* pooled_out, float* inter_out, int concat_dense,
-                                       int32_t* status_dev, dlrm_stream_t stream);
+                                       const float* dense, int B, int F, int D, float* pooled_out,
+                                       float* inter_out, int concat_dense, int32_t* status_dev,
+                                       dlrm_stream_t stream);
 
 /*
  * dlrm_sparse_interact_host -- the whole stage from host memory, for callers
@@ -252,11 +254,11 @@ DLRM_API int dlrm_sparse_interact_pool(const void* const* weights, int table_dty
  *   pooled_host  : host (B, F, D) or NULL; inter_host : host rows.
  */
 DLRM_API int dlrm_sparse_interact_host(const float* const* weights, const int32_t* indices_host,
-                              const int32_t* offsets_host, const float* dense_host, int B,
-                              int F, int L, int D, int concat_dense, int32_t* indices_dev,
-                              int32_t* offsets_dev, float* dense_dev, float* pooled_dev,
-                              float* inter_dev, float* pooled_host, float* inter_host,
-                              dlrm_stream_t stream);
+                                       const int32_t* offsets_host, const float* dense_host, int B,
+                                       int F, int L, int D, int concat_dense, int32_t* indices_dev,
+                                       int32_t* offsets_dev, float* dense_dev, float* pooled_dev,
+                                       float* inter_dev, float* pooled_host, float* inter_host,
+                                       dlrm_stream_t stream);
 
 /*
  * dlrm_pair_decode -- the kernels' flat-index decoder, exposed so it can be
@@ -268,7 +270,7 @@ DLRM_API int dlrm_sparse_interact_host(const float* const* weights, const int32_
  *                  count >= 0 and p0 + count <= 2^31 (else DLRM_ERR_ARG).
  */
 DLRM_API int dlrm_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_t* j_out,
-                     dlrm_stream_t stream);
+                              dlrm_stream_t stream);
 
 /*
  * dlrm_set_gather_path -- which gather serves later gather and fused calls of
