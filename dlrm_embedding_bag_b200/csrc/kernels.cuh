@@ -71,63 +71,41 @@ __global__ void __launch_bounds__(kBlockThreads, kGatherMinBlocks)
   }
 }
 
-// --------------------------------------------------------------------------
-// Fused: each block owns S consecutive samples. Phase 1 gathers their S*F
-// bags straight into shared memory (and, if asked, to pooled_out) next to the
-// dense rows; phase 2 computes the dots from shared memory. Only pooled_out
-// and inter_out are written to global memory.
-template <class LD, int G, int CPL, int POOL>
-__global__ void __launch_bounds__(kBlockThreads, kFusedMinBlocks)
-    fused_kernel(const __grid_constant__ TableParams tp, const BagParams bp,
-                 const float* __restrict__ dense, int B, int F, int D, int ncolwin, int S, int lq,
-                 float* __restrict__ pooled_out, float* __restrict__ inter_out, int concat_dense) {
+// Phase 1 of the fused kernel: the block's bags (s, k) -> feature row k + 1
+// (and pooled_out); every lane group runs the same number of rounds. ORDER
+// (the general entry point, bags of any lengths) takes the bags in sorted runs
+// as described below; without it (fixed-stride bags) slot j of a round is bag j.
+// Bags of different lengths: a warp runs to its longest bag and the block to
+// its slowest warp. So the block's bags are taken in runs of 32; a warp
+// reads the bounds of the run that holds its slots, sorts the run longest
+// first (key: length, then bag number, so keys are unique; a run of equal
+// lengths keeps its order), and the rounds walk the sorted runs in
+// alternating direction: the lane groups of a warp get bags of similar
+// length, and a warp that drew long bags in one round draws short ones in
+// the next. Every warp sorts the same runs the same way, so no block-wide
+// barrier is needed; each warp keeps its sorted run in its own 96 ints of
+// shared memory after the features (rank r: bag, start, length).
+template <class LD, int G, int CPL, int POOL, bool ORDER>
+__device__ __forceinline__ void fused_gather_rounds(const TableParams& tp, const BagParams& bp,
+                                                    float* feat, const FeatLayout& Lf, int B,
+                                                    int F, int D, int ncolwin, int S, int64_t b0,
+                                                    int ntasks, int rounds,
+                                                    float* __restrict__ pooled_out, bool& oob,
+                                                    bool& bad_any) {
   constexpr int VEC = LD::VEC;
   constexpr int U = CPL == 1 ? kRowsInFlight : kRowsInFlight / 2;
   constexpr int kGroups = kBlockThreads / G;
   using Elem = typename LD::Elem;
-  extern __shared__ __align__(16) float feat[];
-  const FeatLayout Lf = FeatLayout::make(F, D);
-  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * S;
-  const int S_here = (B - b0 < S) ? static_cast<int>(B - b0) : S;
   const int lane = threadIdx.x & 31;
   const int q = lane % G;
   const int gbase = lane - q;
   const int64_t sample_floats = Lf.floats_per_sample();
-
-  // dense rows -> feature row 0 (16-byte loads when the pointer allows)
-  const bool dense_vec = ((D & 3) == 0) && ((reinterpret_cast<uintptr_t>(dense) & 15) == 0);
-  for (int s = 0; s < S_here; ++s) {
-    const float* src = dense + (b0 + s) * D;
-    float* dst = feat + s * sample_floats;
-    if (dense_vec) {
-      for (int c = threadIdx.x; c < (D >> 2); c += blockDim.x)
-        reinterpret_cast<float4*>(dst)[c] = __ldg(reinterpret_cast<const float4*>(src) + c);
-    } else {
-      for (int c = threadIdx.x; c < D; c += blockDim.x) dst[c] = __ldg(src + c);
-    }
-  }
-  zero_feature_padding(feat, Lf, D, S_here, threadIdx.x, blockDim.x);
-
-  // bags (s, k) -> feature row k + 1; every group runs the same number of rounds
-  bool oob = false, bad_any = false;
-  const int ntasks = S_here * F;
-  const int rounds = (S * F + kGroups - 1) / kGroups;
-  // Bags of different lengths: a warp runs to its longest bag and the block to
-  // its slowest warp. So the block's bags are taken in runs of 32; a warp
-  // reads the bounds of the run that holds its slots, sorts the run longest
-  // first (key: length, then bag number, so keys are unique; a run of equal
-  // lengths keeps its order), and the rounds walk the sorted runs in
-  // alternating direction: the lane groups of a warp get bags of similar
-  // length, and a warp that drew long bags in one round draws short ones in
-  // the next. Every warp sorts the same runs the same way, so no block-wide
-  // barrier is needed; each warp keeps its sorted run in its own 96 ints of
-  // shared memory after the features (rank r: bag, start, length).
   const int group = static_cast<int>(threadIdx.x) / G;
   for (int rd = 0; rd < rounds; ++rd) {
-    const int slot = rd * kGroups + ((bp.balance && (rd & 1)) ? kGroups - 1 - group : group);
+    const int slot = rd * kGroups + ((ORDER && (rd & 1)) ? kGroups - 1 - group : group);
     const bool active = slot < ntasks;
     int task = slot, start = 0, n = 0;
-    if (bp.balance) {
+    if constexpr (ORDER) {
       // all slots of a warp in a round lie in one run of 32 (warp-uniform);
       // the run is (re)sorted when it differs from the previous round's
       const int g0 = static_cast<int>(threadIdx.x - lane) / G;
@@ -205,6 +183,45 @@ __global__ void __launch_bounds__(kBlockThreads, kFusedMinBlocks)
       }
     }
   }
+}
+
+// --------------------------------------------------------------------------
+// Fused: each block owns S consecutive samples. Phase 1 gathers their S*F
+// bags straight into shared memory (and, if asked, to pooled_out) next to the
+// dense rows; phase 2 computes the dots from shared memory. Only pooled_out
+// and inter_out are written to global memory.
+template <class LD, int G, int CPL, int POOL, bool ORDER>
+__global__ void __launch_bounds__(kBlockThreads, kFusedMinBlocks)
+    fused_kernel(const __grid_constant__ TableParams tp, const BagParams bp,
+                 const float* __restrict__ dense, int B, int F, int D, int ncolwin, int S, int lq,
+                 float* __restrict__ pooled_out, float* __restrict__ inter_out, int concat_dense) {
+  constexpr int kGroups = kBlockThreads / G;
+  extern __shared__ __align__(16) float feat[];
+  const FeatLayout Lf = FeatLayout::make(F, D);
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * S;
+  const int S_here = (B - b0 < S) ? static_cast<int>(B - b0) : S;
+  const int64_t sample_floats = Lf.floats_per_sample();
+
+  // dense rows -> feature row 0 (16-byte loads when the pointer allows)
+  const bool dense_vec = ((D & 3) == 0) && ((reinterpret_cast<uintptr_t>(dense) & 15) == 0);
+  for (int s = 0; s < S_here; ++s) {
+    const float* src = dense + (b0 + s) * D;
+    float* dst = feat + s * sample_floats;
+    if (dense_vec) {
+      for (int c = threadIdx.x; c < (D >> 2); c += blockDim.x)
+        reinterpret_cast<float4*>(dst)[c] = __ldg(reinterpret_cast<const float4*>(src) + c);
+    } else {
+      for (int c = threadIdx.x; c < D; c += blockDim.x) dst[c] = __ldg(src + c);
+    }
+  }
+  zero_feature_padding(feat, Lf, D, S_here, threadIdx.x, blockDim.x);
+
+  // bags (s, k) -> feature row k + 1; every group runs the same number of rounds
+  bool oob = false, bad_any = false;
+  const int ntasks = S_here * F;
+  const int rounds = (S * F + kGroups - 1) / kGroups;
+  fused_gather_rounds<LD, G, CPL, POOL, ORDER>(tp, bp, feat, Lf, B, F, D, ncolwin, S, b0, ntasks,
+                                                rounds, pooled_out, oob, bad_any);
   if (bp.status != nullptr) {
     const int flags = (oob ? DLRM_FLAG_INDEX_OOB : 0) | (bad_any ? DLRM_FLAG_OFFSETS : 0);
     if (flags) atomicOr(bp.status, flags);
@@ -239,7 +256,9 @@ cudaError_t run_gather(const GatherLaunch& a) {
 
 template <class LD, int G, int CPL, int POOL>
 cudaError_t run_fused(const FusedLaunch& a) {
-  auto* fn = &fused_kernel<LD, G, CPL, POOL>;
+  // bags in length-sorted runs (general entry point) or in order (fixed stride)
+  auto* fn = a.g.bp.balance ? &fused_kernel<LD, G, CPL, POOL, true>
+                            : &fused_kernel<LD, G, CPL, POOL, false>;
   if (a.smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
