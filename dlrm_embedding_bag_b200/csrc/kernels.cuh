@@ -71,10 +71,13 @@ __global__ void __launch_bounds__(kBlockThreads, kGatherMinBlocks)
   }
 }
 
+// How phase 1 of the fused kernel orders the bags: slot j of a round is bag j
+// (fixed-stride bags), the bags are taken in sorted runs as described below
+// (the general entry point, bags of any lengths), or bp.balance chooses.
+enum FusedOrder { kOrderNone = 0, kOrderRuns = 1, kOrderByFlag = 2 };
+
 // Phase 1 of the fused kernel: the block's bags (s, k) -> feature row k + 1
-// (and pooled_out); every lane group runs the same number of rounds. ORDER
-// (the general entry point, bags of any lengths) takes the bags in sorted runs
-// as described below; without it (fixed-stride bags) slot j of a round is bag j.
+// (and pooled_out); every lane group runs the same number of rounds.
 // Bags of different lengths: a warp runs to its longest bag and the block to
 // its slowest warp. So the block's bags are taken in runs of 32; a warp
 // reads the bounds of the run that holds its slots, sorts the run longest
@@ -85,7 +88,7 @@ __global__ void __launch_bounds__(kBlockThreads, kGatherMinBlocks)
 // the next. Every warp sorts the same runs the same way, so no block-wide
 // barrier is needed; each warp keeps its sorted run in its own 96 ints of
 // shared memory after the features (rank r: bag, start, length).
-template <class LD, int G, int CPL, int POOL, bool ORDER>
+template <class LD, int G, int CPL, int POOL, int ORDER>
 __device__ __forceinline__ void fused_gather_rounds(const TableParams& tp, const BagParams& bp,
                                                     float* feat, const FeatLayout& Lf, int B,
                                                     int F, int D, int ncolwin, int S, int64_t b0,
@@ -101,11 +104,12 @@ __device__ __forceinline__ void fused_gather_rounds(const TableParams& tp, const
   const int gbase = lane - q;
   const int64_t sample_floats = Lf.floats_per_sample();
   const int group = static_cast<int>(threadIdx.x) / G;
+  const bool ordered = ORDER == kOrderRuns || (ORDER == kOrderByFlag && bp.balance);
   for (int rd = 0; rd < rounds; ++rd) {
-    const int slot = rd * kGroups + ((ORDER && (rd & 1)) ? kGroups - 1 - group : group);
+    const int slot = rd * kGroups + ((ordered && (rd & 1)) ? kGroups - 1 - group : group);
     const bool active = slot < ntasks;
     int task = slot, start = 0, n = 0;
-    if constexpr (ORDER) {
+    if (ordered) {
       // all slots of a warp in a round lie in one run of 32 (warp-uniform);
       // the run is (re)sorted when it differs from the previous round's
       const int g0 = static_cast<int>(threadIdx.x - lane) / G;
@@ -190,7 +194,7 @@ __device__ __forceinline__ void fused_gather_rounds(const TableParams& tp, const
 // bags straight into shared memory (and, if asked, to pooled_out) next to the
 // dense rows; phase 2 computes the dots from shared memory. Only pooled_out
 // and inter_out are written to global memory.
-template <class LD, int G, int CPL, int POOL, bool ORDER>
+template <class LD, int G, int CPL, int POOL, int ORDER>
 __global__ void __launch_bounds__(kBlockThreads, kFusedMinBlocks)
     fused_kernel(const __grid_constant__ TableParams tp, const BagParams bp,
                  const float* __restrict__ dense, int B, int F, int D, int ncolwin, int S, int lq,
@@ -256,9 +260,19 @@ cudaError_t run_gather(const GatherLaunch& a) {
 
 template <class LD, int G, int CPL, int POOL>
 cudaError_t run_fused(const FusedLaunch& a) {
-  // bags in length-sorted runs (general entry point) or in order (fixed stride)
-  auto* fn = a.g.bp.balance ? &fused_kernel<LD, G, CPL, POOL, true>
-                            : &fused_kernel<LD, G, CPL, POOL, false>;
+  // Bags in length-sorted runs (general entry point) or in order (fixed
+  // stride). Measured on B200: f32 rows run faster with one instance per
+  // order (c3 52.6 -> 51.7 us, c5 1.67 -> 1.61 ms), bf16 rows with the
+  // choice made at run time in one instance (c3 47.1 -> 44.4 us, c5 1.34 ->
+  // 1.30 ms; register allocation at the 64-register cap).
+  void (*fn)(const TableParams, const BagParams, const float*, int, int, int, int, int, int,
+             float*, float*, int);
+  if constexpr (sizeof(typename LD::Elem) == 2) {
+    fn = &fused_kernel<LD, G, CPL, POOL, kOrderByFlag>;
+  } else {
+    fn = a.g.bp.balance ? &fused_kernel<LD, G, CPL, POOL, kOrderRuns>
+                        : &fused_kernel<LD, G, CPL, POOL, kOrderNone>;
+  }
   if (a.smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
