@@ -23,3 +23,40 @@ def test_sampled_oracle_matches_full_oracle():
     assert np.array_equal(sp.view(np.uint32), pooled[samples].view(np.uint32))
     assert np.array_equal(si.view(np.uint32), inter[samples].view(np.uint32))
     assert sb.shape == (4, F * (F + 1) // 2)
+
+
+def test_algorithmic_bytes_model():
+    """The roofline's byte model at the benchmark workload: 294,518,784 bytes per
+    fused step (268.44 MB of rows, 4.19 MB of row ids, 0.26 MB of offsets,
+    0.52 MB of dense rows, 16.78 MB of pooled rows, 4.33 MB of dots)."""
+    import bench
+    from dlrm_embedding_bag_b200 import synthetic as syn
+    w = syn.C3_ZIPF
+    assert bench.algorithmic_bytes(w) == 294_518_784
+    parts = {"rows": 2048 * 32 * 16 * 64 * 4, "ids": 2048 * 32 * 16 * 4, "offsets": 2048 * 32 * 4,
+             "dense": 2048 * 64 * 4, "pooled": 2048 * 32 * 64 * 4, "dots": 2048 * 528 * 4}
+    assert sum(parts.values()) == 294_518_784
+    # without the pooled output, with 2-byte rows, with a 4-byte weight per entry
+    assert bench.algorithmic_bytes(w, write_pooled=False) == 294_518_784 - parts["pooled"]
+    assert bench.algorithmic_bytes(w, esz=2) == 294_518_784 - parts["rows"] // 2
+    assert bench.algorithmic_bytes(w, weighted=True) == 294_518_784 + parts["ids"]
+    # concatenated rows [dense | dots] at c2
+    c2 = syn.C2_CONCAT
+    assert bench.algorithmic_bytes(c2) == (2048 * 8 * 32 * 64 * 4 + 2048 * 8 * 32 * 4
+                                           + 2048 * 8 * 4 + 2048 * 64 * 4
+                                           + 2048 * 8 * 64 * 4 + 2048 * (64 + 36) * 4)
+
+
+def test_recorded_traffic_applies_only_to_unchanged_sources(tmp_path, monkeypatch):
+    """The committed DRAM figure is reported only while the fused kernel's
+    sources still hash to the digest it was captured with."""
+    import json
+    import bench
+    rec = {"w": {"source_digest": bench.source_digest(), "dram_bytes_per_launch": 123}}
+    (tmp_path / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "PROFILES", str(tmp_path))
+    assert bench.recorded_traffic("w") == 123
+    assert bench.recorded_traffic("other") is None
+    rec["w"]["source_digest"] = "0" * 16
+    (tmp_path / "traffic.json").write_text(json.dumps(rec))
+    assert bench.recorded_traffic("w") is None

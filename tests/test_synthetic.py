@@ -61,3 +61,41 @@ def test_weights_and_dense_seeded():
     assert abs(float(t1[0].std()) - 0.1) < 0.01
     d = syn.make_dense(w)
     assert d.shape == (w.B, w.D) and torch.equal(d, syn.make_dense(w))
+
+
+def test_ragged_offsets_cover_the_same_entries():
+    """Ragged bags: sorted cut points on [0, B*L], first bag at 0, mean length L,
+    seeded per table (PCG64(6000 + k))."""
+    w = syn.C3_ZIPF.scaled(B=512)
+    off = syn.make_ragged_offsets(w)
+    T = w.B * w.L
+    assert off.dtype == np.int32 and off.shape == (w.F, w.B)
+    assert np.array_equal(off, syn.make_ragged_offsets(w))
+    assert np.all(off[:, 0] == 0)
+    assert np.all(np.diff(off, axis=1) >= 0) and off.max() <= T
+    lengths = np.diff(np.concatenate([off, np.full((w.F, 1), T)], axis=1), axis=1)
+    assert np.all(lengths.sum(axis=1) == T)          # every entry in exactly one bag
+    assert abs(lengths.mean() - w.L) < 1e-9          # mean length L
+    assert (lengths == 0).any() and lengths.max() > 3 * w.L   # really ragged
+    assert not np.array_equal(off[0], off[1])
+
+
+def test_sample_weights_seeded_in_unit_interval():
+    w = syn.TINY
+    a = syn.make_sample_weights(w)
+    assert a.dtype == np.float32 and a.shape == (w.F, w.B * w.L)
+    assert np.array_equal(a, syn.make_sample_weights(w))
+    assert a.min() >= 0.0 and a.max() < 1.0
+    assert not np.array_equal(a[0], a[1])
+
+
+def test_mlp_layers_shapes_and_dtypes():
+    layers = syn.make_mlp_layers(13, [512, 256, 64], 7, "cpu")
+    assert [tuple(wt.shape) for wt, _, _ in layers] == [(512, 13), (256, 512), (64, 256)]
+    assert all(wt.dtype == torch.bfloat16 and b.dtype == torch.float32 for wt, b, _ in layers)
+    assert [act for _, _, act in layers] == ["relu", "relu", "relu"]
+    top = syn.make_mlp_layers(592, [512, 256, 1], 8, "cpu", last="sigmoid")
+    assert top[-1][2] == "sigmoid" and top[0][2] == "relu"
+    again = syn.make_mlp_layers(13, [512, 256, 64], 7, "cpu")
+    assert all(torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
+               for a, b in zip(layers, again))
