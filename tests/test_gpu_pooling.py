@@ -237,3 +237,57 @@ def test_bf16_full_size_sampled(ops):
     assert_dots_close(inter[sel], ref_i, bound, "bf16 c3 dots (sampled)")
     del weights, pooled, inter
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("weighted", [False, True], ids=["sum", "weighted"])
+def test_ragged_full_size_sampled(ops, weighted):
+    """The c3 workload with ragged bags (the benchmark's ragged input: sorted
+    uniform cut points, mean length L) and optionally per-sample weights,
+    through the fused general entry point; sampled check of pooled rows (bit
+    for bit) and dots."""
+    w = syn.C3_ZIPF
+    torch.cuda.empty_cache()
+    weights = syn.make_weights(w, DEV)
+    idx = syn.make_indices(w)
+    off = syn.make_ragged_offsets(w)
+    psw = syn.make_sample_weights(w) if weighted else None
+    dense = syn.make_dense(w, DEV)
+    pooled, inter = ops.sparse_interact_pool(
+        weights, torch.from_numpy(idx).to(DEV), torch.from_numpy(off).to(DEV), dense,
+        per_sample_weights=torch.from_numpy(psw).to(DEV) if weighted else None)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(11)
+    samples = np.unique(np.concatenate([[0, w.B - 1], rng.integers(0, w.B, 30)]))
+    T = w.B * w.L
+    tables, sub_idx, sub_w = [], [], []
+    sub_off = np.zeros((w.F, len(samples) + 1), np.int32)
+    for k in range(w.F):
+        ends = np.append(off[k, 1:], T)
+        spans = [(int(off[k, s]), int(ends[s])) for s in samples]
+        rows = np.concatenate([idx[k, a:b] for a, b in spans])
+        uniq, inv = np.unique(rows, return_inverse=True)
+        if uniq.size == 0:  # every sampled bag of this table is empty
+            uniq = np.zeros(1, np.int32)
+        t = weights[k].index_select(0, torch.from_numpy(uniq.astype(np.int64)).to(DEV))
+        tables.append(t.cpu().numpy())
+        sub_idx.append(inv.astype(np.int32))
+        if weighted:
+            sub_w.append(np.concatenate([psw[k, a:b] for a, b in spans]))
+        sub_off[k, 1:] = np.cumsum([b - a for a, b in spans])
+    seg = max(1, max(x.size for x in sub_idx))
+    idx_pad = np.zeros((w.F, seg), np.int32)
+    w_pad = np.zeros((w.F, seg), np.float32)
+    for k in range(w.F):
+        idx_pad[k, :sub_idx[k].size] = sub_idx[k]
+        if weighted:
+            w_pad[k, :sub_w[k].size] = sub_w[k]
+    ref = oracle.embbag_pool_multi(tables, idx_pad, sub_off, len(samples),
+                                   per_sample_weights=w_pad if weighted else None,
+                                   include_last_offset=True)
+    sel = torch.from_numpy(samples).to(DEV)
+    what = "ragged c3" + (" weighted" if weighted else "")
+    assert_bits_equal(pooled[sel], ref, what + " pooled (sampled)")
+    ref_i, _, bound = oracle.interact_lower_tri(dense[sel].cpu().numpy(), ref, with_f64=True)
+    assert_dots_close(inter[sel], ref_i, bound, what + " dots (sampled)")
+    del weights, pooled, inter
+    torch.cuda.empty_cache()
