@@ -452,6 +452,19 @@ def pin_mean_and_max_closed_forms(orc):
         assert np.array_equal(z.view(np.uint32), np.zeros_like(z).view(np.uint32)), mode
 
 
+def pin_max_ties_keep_the_earlier_entry(orc):
+    """Max pooling keeps the first entry, then takes x only when x > acc, so a
+    tie keeps the entry seen first: of -0.0 and +0.0 the earlier survives."""
+    tab = np.array([[-0.0, 0.0, 1.0], [0.0, -0.0, 1.0]], np.float32)
+    idx = np.array([[0, 1, 1, 0]], np.int32)      # bag 0: rows 0, 1; bag 1: rows 1, 0
+    off = np.array([[0, 2]], np.int32)
+    mx = orc.embbag_pool_multi([tab], idx, off, 2, mode="max")
+    bits = mx.view(np.uint32)
+    assert bits[0, 0, 0] == 0x80000000 and bits[0, 0, 1] == 0          # -0 then +0 -> -0
+    assert bits[1, 0, 0] == 0 and bits[1, 0, 1] == 0x80000000          # +0 then -0 -> +0
+    assert mx[0, 0, 2] == 1.0 and mx[1, 0, 2] == 1.0
+
+
 def pin_bf16_tables_widen_exactly(orc):
     """bf16 tables pool exactly like their f32 widening (done by torch)."""
     rng = np.random.default_rng(25)

@@ -56,6 +56,10 @@ MUTANTS = {
     "mean_divides_by_count_plus_one": [("acc = acc / (float)(e - s);",
                                         "acc = acc / (float)(e - s + 1);")],
     "max_keeps_the_minimum": [("((x > acc) ? x : acc)", "((x < acc) ? x : acc)")],
+    "max_ties_take_the_later_entry": [("acc = (t == s) ? x : ((x > acc) ? x : acc);",
+                                       "acc = (t == s) ? x : ((x >= acc) ? x : acc);")],
+    "mean_of_empty_bag_divides_by_zero": [("if (mode == ORACLE_POOL_MEAN && e > s) acc",
+                                           "if (mode == ORACLE_POOL_MEAN) acc")],
     "max_starts_from_zero": [("acc = (t == s) ? x : ((x > acc) ? x : acc);",
                               "acc = (x > acc) ? x : acc;")],
     "last_offset_ignored": [("(ilo || b + 1 < B) ? (int64_t)offsets[(int64_t)k * row + b + 1]",
