@@ -291,3 +291,30 @@ def test_ragged_full_size_sampled(ops, weighted):
     assert_dots_close(inter[sel], ref_i, bound, what + " dots (sampled)")
     del weights, pooled, inter
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_max_ties_keep_the_earlier_entry(ops, dtype):
+    """Max pooling keeps the first entry and then takes x only when x > acc, so
+    of two tied entries the earlier survives: -0.0 then +0.0 gives -0.0, +0.0
+    then -0.0 gives +0.0, bit for bit, on every path and in the fused kernel."""
+    B, F, D = 48, 3, 64
+    tab = np.zeros((4, D), np.float32)
+    tab[0] = -0.0
+    tab[2] = -1.0
+    tab[3, ::2] = -0.0
+    pairs = np.array([[0, 1], [1, 0], [2, 0], [0, 2], [3, 1], [1, 3]], np.int32)
+    rng = np.random.default_rng(5)
+    idx = np.stack([pairs[rng.integers(0, len(pairs), B)].reshape(-1) for _ in range(F)])
+    off = np.broadcast_to(np.arange(B, dtype=np.int32) * 2, (F, B)).copy()
+    weights = [torch.from_numpy(tab).to(DEV).to(dtype) for _ in range(F)]
+    ref = oracle.embbag_pool_multi([_host_bits(w) for w in weights], idx, off, B, mode="max")
+    assert (ref.view(np.uint32) == 0x80000000).any() and (ref.view(np.uint32) == 0).any()
+    idx_d = torch.from_numpy(idx).to(DEV)
+    off_d = torch.from_numpy(off).to(DEV)
+    out = ops.embbag_pool_multi(weights, idx_d, off_d, mode="max")
+    dense = torch.zeros((B, D), device=DEV)
+    fp, _ = ops.sparse_interact_pool(weights, idx_d, off_d, dense, mode="max")
+    torch.cuda.synchronize()
+    assert_bits_equal(out, ref, "max ties, embbag_pool_multi")
+    assert_bits_equal(fp, ref, "max ties, fused pooled")
