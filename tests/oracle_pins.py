@@ -428,6 +428,32 @@ def pin_weighted_sum_exact_cases(orc):
             assert all(Fraction(float(o)) == e for o, e in zip(out[b, k], exact)), (b, k)
 
 
+def pin_weighted_sum_rounds_once_per_entry(orc):
+    """Each weighted entry is one fused multiply-add: with w = x = 1 + 2^-12 after a
+    -1, the exact w*x - 1 = 2^-11 + 2^-24 is an f32 and must come out whole (a
+    rounded product first would lose the 2^-24)."""
+    a = 1.0 + 2.0 ** -12
+    tab = np.array([[-1.0], [a]], np.float32)
+    idx = np.array([[0, 1]], np.int32)
+    off = np.zeros((1, 1), np.int32)
+    wts = np.array([[1.0, a]], np.float32)
+    out = orc.embbag_pool_multi([tab], idx, off, 1, per_sample_weights=wts)
+    exact = Fraction(a) * Fraction(a) - 1
+    assert exact == Fraction(2) ** -11 + Fraction(2) ** -24
+    assert Fraction(float(out[0, 0, 0])) == exact
+
+
+def pin_mean_divides_once(orc):
+    """Mean is the f32 sum divided once by the count: entries 2, 2, 1 give the
+    f32 nearest 5/3 (0x3FD55555), not 5 times the f32 nearest 1/3."""
+    tab = np.array([[2.0], [1.0]], np.float32)
+    idx = np.array([[0, 0, 1]], np.int32)
+    off = np.zeros((1, 1), np.int32)
+    out = orc.embbag_pool_multi([tab], idx, off, 1, mode="mean")
+    assert out.view(np.uint32)[0, 0, 0] == 0x3FD55555
+    assert np.float32(5.0) * np.float32(1.0 / 3.0) != out[0, 0, 0]  # the case tells them apart
+
+
 def pin_mean_and_max_closed_forms(orc):
     """Mean of L copies of a dyadic row is the row; max equals numpy's maximum."""
     rng = np.random.default_rng(24)

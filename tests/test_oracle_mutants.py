@@ -51,6 +51,10 @@ MUTANTS = {
     "concat_drops_dense": [("row[d] = dense[(int64_t)b * D + d];", "row[d] = 0.0f;")],
     "bf16_widened_with_wrong_shift": [("((uint32_t)h) << 16", "((uint32_t)h) << 15")],
     "weighted_sum_drops_weight": [("acc = fmaf(wk[t], x, acc);", "acc = acc + x;")],
+    "weighted_sum_rounds_the_product_first": [("acc = fmaf(wk[t], x, acc);",
+                                               "acc = acc + wk[t] * x;")],
+    "mean_multiplies_by_reciprocal": [("acc = acc / (float)(e - s);",
+                                       "acc = acc * (1.0f / (float)(e - s));")],
     "weighted_sum_uses_first_weight": [("acc = fmaf(wk[t], x, acc);",
                                         "acc = fmaf(wk[s], x, acc);")],
     "mean_divides_by_count_plus_one": [("acc = acc / (float)(e - s);",
