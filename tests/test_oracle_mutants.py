@@ -41,6 +41,10 @@ MUTANTS = {
     "dot_wrong_operand": [("(double)a[d] * (double)b[d]", "(double)a[d] * (double)a[d]")],
     "dot_drops_first_term": [("for (int d = 0; d < D; ++d) {\n        double t",
                               "for (int d = 1; d < D; ++d) {\n        double t")],
+    "dot_accumulates_in_float": [("        double t = (double)a[d] * (double)b[d];\n        s += t;",
+                                  "        double t = (double)a[d] * (double)b[d];\n"
+                                  "        s = (double)((float)s + (float)t);")],
+    "dot_bound_loses_the_absolute_value": [("m += (t < 0.0) ? -t : t;", "m += t;")],
     "dot_stores_abs_sum": [("z[p] = (float)s;", "z[p] = (float)m;")],
     "features_in_reverse_table_order": [("emb + ((int64_t)b * F + (i - 1)) * D;",
                                          "emb + ((int64_t)b * F + (F - i)) * D;")],
