@@ -50,6 +50,39 @@ def test_library_exports_every_declared_symbol(ops):
         assert getattr(ops._lib, n) is not None
 
 
+def _declarations():
+    """name -> (return type, [parameter types]) from the headers' DLRM_API lines."""
+    out = {}
+    for h in HEADERS:
+        src = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        for ret, name, params in re.findall(r"DLRM_API\s+([\w\s\*]+?)\b(\w+)\s*\(([^)]*)\)\s*;",
+                                            src):
+            plist = [] if params.strip() in ("", "void") else [p.strip() for p in params.split(",")]
+            types = [re.sub(r"\s*\b\w+$", "", p) if not p.endswith("*") else p for p in plist]
+            out[name] = (" ".join(ret.split()), [" ".join(t.split()) for t in types])
+    return out
+
+
+def _ctype_of(decl):
+    if "*" in decl or decl == "dlrm_stream_t":
+        return ctypes.c_void_p
+    return {"int": ctypes.c_int, "int64_t": ctypes.c_int64, "int32_t": ctypes.c_int32}[decl]
+
+
+def test_binding_signatures_match_the_headers(ops):
+    """Every ctypes signature in the binding has the header's arity and, per
+    argument, the same kind (pointer, int, int32_t or int64_t)."""
+    decls = _declarations()
+    assert set(decls) == set(ops.SIGNATURES)
+    for name, (ret, params) in decls.items():
+        res, args = ops.SIGNATURES[name]
+        assert len(args) == len(params), name
+        for i, (a, p) in enumerate(zip(args, params)):
+            assert a is _ctype_of(p), (name, i, p)
+        want_ret = ctypes.c_char_p if ret == "const char*" else _ctype_of(ret)
+        assert res is want_ret, (name, ret)
+
+
 def _ptrs(*vals):
     return (ctypes.c_void_p * len(vals))(*vals)
 
