@@ -222,3 +222,49 @@ def test_probe_host_checks(ops):
     lib = ops._lib
     assert lib.dlrm_probe_bounded_wait(1000, None, None) == -1
     assert lib.dlrm_probe_bounded_wait(1000, 0x10002, None) == -3
+
+
+def test_header_compiles_as_c_and_matches_the_binding(ops, tmp_path):
+    """The headers are plain C: a probe built with gcc reports the layout of
+    dlrm_bags_t and the constants, which must equal what the binding passes."""
+    from dlrm_embedding_bag_b200 import mlp
+
+    probe = tmp_path / "probe.c"
+    probe.write_text(r"""
+#include <stddef.h>
+#include <stdio.h>
+#include "dlrm_sparse.h"
+#include "dlrm_mlp.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu %zu %zu\n", sizeof(dlrm_bags_t),
+         offsetof(dlrm_bags_t, indices), offsetof(dlrm_bags_t, offsets),
+         offsetof(dlrm_bags_t, per_sample_weights), offsetof(dlrm_bags_t, T),
+         offsetof(dlrm_bags_t, include_last_offset), offsetof(dlrm_bags_t, mode));
+  printf("%d %d %d %d %d %d %d\n", DLRM_MAX_TABLES, DLRM_FLAG_INDEX_OOB, DLRM_FLAG_OFFSETS,
+         DLRM_FLAG_TIMEOUT, DLRM_POOL_SUM, DLRM_POOL_MEAN, DLRM_POOL_MAX);
+  printf("%d %d %d %d %d %d\n", DLRM_TABLE_F32, DLRM_TABLE_BF16, DLRM_PATH_AUTO, DLRM_PATH_LDG,
+         DLRM_PATH_TMA, DLRM_PATH_PIPE);
+  printf("%d %d %d\n", DLRM_ACT_NONE, DLRM_ACT_RELU, DLRM_ACT_SIGMOID);
+  return 0;
+}
+""")
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(probe), "-o", str(exe)], check=True)
+    lines = subprocess.run([str(exe)], capture_output=True, text=True,
+                           check=True).stdout.split("\n")
+    layout = [int(v) for v in lines[0].split()]
+    B = ops.Bags
+    assert layout == [ctypes.sizeof(B), B.indices.offset, B.offsets.offset,
+                      B.per_sample_weights.offset, B.T.offset, B.include_last_offset.offset,
+                      B.mode.offset]
+    consts = [int(v) for v in lines[1].split()]
+    assert consts == [ops.DLRM_MAX_TABLES, ops.FLAG_INDEX_OOB, ops.FLAG_OFFSETS,
+                      ops.FLAG_TIMEOUT, ops.POOL_MODES["sum"], ops.POOL_MODES["mean"],
+                      ops.POOL_MODES["max"]]
+    paths = [int(v) for v in lines[2].split()]
+    import torch
+    assert paths[:2] == [ops.TABLE_DTYPES[torch.float32], ops.TABLE_DTYPES[torch.bfloat16]]
+    assert paths[2:] == [ops.GATHER_PATHS[p] for p in ("auto", "ldg", "tma", "pipe")]
+    assert [int(v) for v in lines[3].split()] == [mlp.ACTS[a] for a in ("none", "relu",
+                                                                        "sigmoid")]
