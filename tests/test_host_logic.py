@@ -60,3 +60,24 @@ def test_recorded_traffic_applies_only_to_unchanged_sources(tmp_path, monkeypatc
     rec["w"]["source_digest"] = "0" * 16
     (tmp_path / "traffic.json").write_text(json.dumps(rec))
     assert bench.recorded_traffic("w") is None
+
+
+def test_oracle_and_cuda_path_share_no_code():
+    """The oracle (test infrastructure) and the product are independent: the
+    package and its CUDA sources never import or include the oracle, and the
+    oracle never imports the package or includes its sources."""
+    import os
+    import re
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "dlrm_embedding_bag_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", src, re.M), f
+                assert "dlrm_oracle" not in src, f
+    for f in os.listdir(os.path.join(root, "oracle")):
+        if f.endswith((".py", ".c", ".h")):
+            src = open(os.path.join(root, "oracle", f)).read()
+            assert not re.search(r"^\s*(import|from)\s+dlrm_embedding_bag_b200\b", src, re.M), f
+            assert not re.search(r"#\s*include\s*[<\"].*(csrc|dlrm_sparse|dlrm_mlp)", src), f
