@@ -81,3 +81,30 @@ def test_oracle_and_cuda_path_share_no_code():
             src = open(os.path.join(root, "oracle", f)).read()
             assert not re.search(r"^\s*(import|from)\s+dlrm_embedding_bag_b200\b", src, re.M), f
             assert not re.search(r"#\s*include\s*[<\"].*(csrc|dlrm_sparse|dlrm_mlp)", src), f
+
+
+def test_fused_bag_rounds_cover_every_bag_once():
+    """The fused kernel's round structure (256 threads, lane groups of G lanes,
+    slot = round * groups + group, mirrored in odd rounds when the bags are
+    ordered): every bag of a block is taken exactly once, and all slots of a
+    warp in a round lie in one run of 32 bags -- the property that lets each
+    warp sort and keep one run at a time without a block-wide barrier."""
+    threads = 256
+    for G in (4, 8, 16, 32):
+        groups = threads // G
+        for S in (1, 2, 3, 4):
+            for F in (1, 2, 3, 5, 8, 26, 32, 33, 100, 256):
+                if S * F >= 2048:
+                    continue
+                rounds = -(-S * F // groups)
+                for ntasks in {S * F, max(1, S * F - F)}:  # full block and a tail block
+                    for ordered in (False, True):
+                        seen = []
+                        for rd in range(rounds):
+                            for warp in range(threads // 32):
+                                gs = range(warp * 32 // G, (warp + 1) * 32 // G)
+                                slots = [rd * groups + ((groups - 1 - g) if ordered and rd & 1
+                                                        else g) for g in gs]
+                                assert len({s >> 5 for s in slots}) == 1, (G, S, F, rd, warp)
+                                seen += [s for s in slots if s < ntasks]
+                        assert sorted(seen) == list(range(ntasks)), (G, S, F, ordered)
