@@ -108,3 +108,36 @@ def test_fused_bag_rounds_cover_every_bag_once():
                                 assert len({s >> 5 for s in slots}) == 1, (G, S, F, rd, warp)
                                 seen += [s for s in slots if s < ntasks]
                         assert sorted(seen) == list(range(ntasks)), (G, S, F, ordered)
+
+
+def test_warp_bitonic_network_sorts_descending():
+    """The 32-lane bitonic network of the fused kernel's bag ordering (phase k,
+    step j: the lane keeps the larger of itself and lane ^ j exactly when bit j
+    and bit k of its index agree) sorts any keys descending; keys are
+    (min(length, 2^21 - 2) + 1) << 11 | bag, so empty slots (key 0) go last and
+    equal lengths keep bag order."""
+    def network(keys):
+        keys = list(keys)
+        k = 2
+        while k <= 32:
+            j = k >> 1
+            while j:
+                other = [keys[lane ^ j] for lane in range(32)]
+                keys = [max(keys[lane], other[lane]) if ((lane & j) == 0) == ((lane & k) == 0)
+                        else min(keys[lane], other[lane]) for lane in range(32)]
+                j >>= 1
+            k <<= 1
+        return keys
+
+    rng = np.random.default_rng(1)
+    for trial in range(300):
+        n = int(rng.integers(0, 33))
+        lengths = rng.integers(0, 40 if trial % 2 else 3, n)
+        keys = [((min(int(ln), (1 << 21) - 2) + 1) << 11) | t for t, ln in enumerate(lengths)]
+        keys += [0] * (32 - n)
+        perm = rng.permutation(32)
+        out = network([keys[p] for p in perm])
+        assert out == sorted(keys, reverse=True)
+        bags = [key & 2047 for key in out[:n]]
+        # longest first; among equal lengths the lower bag number first
+        assert [(-int(lengths[b]), b) for b in bags] == sorted((-int(lengths[b]), b) for b in bags)
