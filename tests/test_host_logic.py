@@ -115,7 +115,7 @@ def test_warp_bitonic_network_sorts_descending():
     step j: the lane keeps the larger of itself and lane ^ j exactly when bit j
     and bit k of its index agree) sorts any keys descending; keys are
     (min(length, 2^21 - 2) + 1) << 11 | bag, so empty slots (key 0) go last and
-    equal lengths keep bag order."""
+    keys are unique (ties in length order by bag number, higher first)."""
     def network(keys):
         keys = list(keys)
         k = 2
@@ -139,5 +139,6 @@ def test_warp_bitonic_network_sorts_descending():
         out = network([keys[p] for p in perm])
         assert out == sorted(keys, reverse=True)
         bags = [key & 2047 for key in out[:n]]
-        # longest first; among equal lengths the lower bag number first
-        assert [(-int(lengths[b]), b) for b in bags] == sorted((-int(lengths[b]), b) for b in bags)
+        # longest first; among equal lengths the higher bag number first
+        assert [(int(lengths[b]), b) for b in bags] == sorted(
+            ((int(lengths[b]), b) for b in bags), reverse=True)
