@@ -28,8 +28,8 @@ STATUS = {
     -5: "DLRM_ERR_INDEX_OOB",
     -6: "DLRM_ERR_OFFSETS",
     -7: "DLRM_ERR_CUDA",
-    -8: "DLRM_ERR_ARG",
-    -9: "DLRM_ERR_TIMEOUT",
+    -8: "DLRM_ERR_TIMEOUT",
+    -9: "DLRM_ERR_ARG",
 }
 GATHER_PATHS = {"auto": 0, "ldg": 1, "tma": 2, "pipe": 3}
 FLAG_INDEX_OOB = 1
@@ -505,9 +505,15 @@ class HostPipeline:
         return self.slots[0][0].d2h_bytes()
 
     def submit(self, indices_host, offsets_host, dense_host, inter_host, pooled_host=None):
+        """Enqueue one batch; returns its completion event. The host inputs
+        must stay unchanged, and the host outputs unread, until that event
+        has completed."""
         stage, stream, done = self.slots[self.n % len(self.slots)]
         self.n += 1
         done.synchronize()  # the slot's previous batch (and its host outputs) is finished
+        # work the caller queued before this call (e.g. writes to the tables)
+        # comes first
+        stream.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(stream):
             stage(indices_host, offsets_host, dense_host, inter_host, pooled_host)
             done.record(stream)

@@ -75,9 +75,9 @@ typedef enum {
                                       or end > B*L */
     DLRM_ERR_CUDA = -7,            /* a CUDA runtime call or launch failed; see
                                       dlrm_last_cuda_error() */
-    DLRM_ERR_ARG = -8,             /* any other invalid argument (e.g. count < 0) */
-    DLRM_ERR_TIMEOUT = -9          /* (device flag) a bounded wait on an asynchronous
+    DLRM_ERR_TIMEOUT = -8,         /* (device flag) a bounded wait on an asynchronous
                                       copy ran out; the results are not valid */
+    DLRM_ERR_ARG = -9              /* any other invalid argument (e.g. count < 0) */
 } dlrm_status_t;
 
 /* Bits that the checked (_ex) entry points OR into *status_dev. */
@@ -265,7 +265,10 @@ DLRM_API int dlrm_sparse_interact_host(const float* const* weights, const int32_
  * checked exhaustively. For p in [p0, p0 + count): (i, j) of the p-th pair of
  * the strict lower triangle, i = floor((1 + sqrt(1 + 8p)) / 2) and
  * j = p - i(i-1)/2, from an f32 square root followed by an exact integer
- * correction (dlrm_interact.rs, stacked-kernel layout comment).
+ * correction (dlrm_interact.rs, stacked-kernel layout comment). For
+ * p < 2^24 this runs the 32-bit decoder that the interaction and fused
+ * kernels apply to their pair-tile index (a tile index is below 2145 at
+ * DLRM_MAX_TABLES); from 2^24 on, a 64-bit form of the same steps.
  *   i_out, j_out : dev int32 arrays of `count` entries. Needs p0 >= 0,
  *                  count >= 0 and p0 + count <= 2^31 (else DLRM_ERR_ARG).
  */

@@ -96,8 +96,8 @@ def test_status_strings_and_flags(ops):
     assert lib.dlrm_status_from_flags(1) == -5
     assert lib.dlrm_status_from_flags(2) == -6
     assert lib.dlrm_status_from_flags(3) == -5
-    assert lib.dlrm_status_from_flags(4) == -9
-    assert lib.dlrm_set_gather_path(7) == -8
+    assert lib.dlrm_status_from_flags(4) == -8
+    assert lib.dlrm_set_gather_path(7) == -9
     assert lib.dlrm_set_gather_path(1) == 0 and lib.dlrm_set_gather_path(0) == 1
     assert lib.dlrm_set_gather_path(3) == 0 and lib.dlrm_set_gather_path(0) == 3
     assert lib.dlrm_launch_count() == 0
@@ -127,7 +127,7 @@ def test_checked_entry_points_need_rows(ops):
     assert rc == -1
     rows = (ctypes.c_int64 * 1)(-5)
     rc = ops._lib.embbag_sum_multi_ex(_ptrs(FAKE), rows, FAKE, FAKE, 4, 1, 2, 8, FAKE, None, None)
-    assert rc == -8
+    assert rc == -9
 
 
 def test_fused_and_interact_host_checks(ops):
@@ -144,9 +144,9 @@ def test_fused_and_interact_host_checks(ops):
     assert lib.interact_lower_tri(FAKE, FAKE + 2, 4, 2, 8, FAKE, None) == -3
     assert lib.dlrm_sparse_interact_host(w, FAKE, FAKE, FAKE, 4, 2, 2, 8, 0, FAKE, FAKE, FAKE,
                                          None, FAKE, FAKE, None, None) == -1
-    assert lib.dlrm_pair_decode(-1, 5, FAKE, FAKE, None) == -8
-    assert lib.dlrm_pair_decode(0, -1, FAKE, FAKE, None) == -8
-    assert lib.dlrm_pair_decode((1 << 31) - 2, 5, FAKE, FAKE, None) == -8
+    assert lib.dlrm_pair_decode(-1, 5, FAKE, FAKE, None) == -9
+    assert lib.dlrm_pair_decode(0, -1, FAKE, FAKE, None) == -9
+    assert lib.dlrm_pair_decode((1 << 31) - 2, 5, FAKE, FAKE, None) == -9
     assert lib.dlrm_pair_decode(0, 5, None, FAKE, None) == -1
     assert lib.dlrm_launch_count() == 0
 
@@ -156,13 +156,13 @@ def test_general_pooling_host_checks(ops):
     w = _ptrs(FAKE, FAKE)
     bags = ops.Bags(FAKE, FAKE, None, 8, 0, 0)
     assert lib.embbag_pool_multi(w, 0, None, None, 4, 2, 8, FAKE, None, None) == -1
-    assert lib.embbag_pool_multi(w, 2, None, ctypes.byref(bags), 4, 2, 8, FAKE, None, None) == -8
+    assert lib.embbag_pool_multi(w, 2, None, ctypes.byref(bags), 4, 2, 8, FAKE, None, None) == -9
     bad_mode = ops.Bags(FAKE, FAKE, None, 8, 0, 7)
     assert lib.embbag_pool_multi(w, 0, None, ctypes.byref(bad_mode), 4, 2, 8, FAKE, None,
-                                 None) == -8
+                                 None) == -9
     psw_mean = ops.Bags(FAKE, FAKE, FAKE, 8, 0, 1)
     assert lib.embbag_pool_multi(w, 0, None, ctypes.byref(psw_mean), 4, 2, 8, FAKE, None,
-                                 None) == -8
+                                 None) == -9
     neg_t = ops.Bags(FAKE, FAKE, None, -1, 0, 0)
     assert lib.embbag_pool_multi(w, 0, None, ctypes.byref(neg_t), 4, 2, 8, FAKE, None,
                                  None) == -2
@@ -177,7 +177,7 @@ def test_general_pooling_host_checks(ops):
                                  None) == -1
     rows = (ctypes.c_int64 * 2)(5, -1)
     assert lib.embbag_pool_multi(w, 0, rows, ctypes.byref(bags), 4, 2, 8, FAKE, None,
-                                 None) == -8
+                                 None) == -9
     assert lib.dlrm_sparse_interact_pool(w, 0, None, ctypes.byref(bags), None, 4, 2, 8, None,
                                          FAKE, 0, None, None) == -1
     assert lib.dlrm_launch_count() == 0
@@ -204,7 +204,7 @@ def test_linear_host_checks(ops):
     assert call(w=None) == -1
     assert call(y32=None) == -1
     assert call(k_hi=8, lda_hi=8, ldw=72) == -1          # a_hi missing
-    assert call(act=3) == -8
+    assert call(act=3) == -9
     assert call(M=0) == -2 and call(N=0) == -2 and call(k_lo=0) == -2
     assert call(lda_lo=56) == -2                          # pitch < k
     assert call(ldw=56) == -2

@@ -15,7 +15,7 @@ def test_bounded_wait_times_out_and_context_survives():
     ops.probe_bounded_wait(status, limit_cycles=2_000_000)  # about a millisecond
     torch.cuda.synchronize()
     assert int(status.item()) == ops.FLAG_TIMEOUT
-    assert ops._lib.dlrm_status_from_flags(int(status.item())) == -9
+    assert ops._lib.dlrm_status_from_flags(int(status.item())) == -8
     # the context is intact: an ordinary call runs and is correct
     w = [torch.arange(12, dtype=torch.float32, device=DEV).reshape(3, 4)]
     idx = torch.tensor([[0, 2]], dtype=torch.int32, device=DEV)
