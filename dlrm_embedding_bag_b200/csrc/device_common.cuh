@@ -109,7 +109,9 @@ __device__ __forceinline__ void pair_from_flat(int64_t p, int& i_out, int& j_out
   j_out = static_cast<int>(p - i * (i - 1) / 2);
 }
 
-// The same decoder for small p (< 2^24, where every int is exact in f32).
+// The same decoder for small p (< 2^24, where every int is exact in f32); the
+// interaction's dot phase decodes its tile index with it.
+constexpr int64_t kPairSmallLimit = int64_t{1} << 24;
 __device__ __forceinline__ void pair_from_flat_small(int p, int& i_out, int& j_out) {
   int i = static_cast<int>((sqrtf(8.0f * static_cast<float>(p) + 1.0f) + 1.0f) * 0.5f);
   if (i < 1) i = 1;

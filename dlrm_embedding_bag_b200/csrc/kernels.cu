@@ -4,7 +4,7 @@
 //   embbag_kernel / fused_kernel : kernels.cuh, instantiated in inst_*.cu
 //   interact_kernel    : strict-lower-triangle pairwise dots
 //                        (dlrm_interact.rs, stacked kernel of the pages)
-//   pair_decode_kernel : the closed-form pair decoder alone, for tests
+//   pair_decode_kernel : the closed-form pair decoders alone, for tests
 #include <algorithm>
 #include <atomic>
 
@@ -113,12 +113,20 @@ __global__ void probe_wait_kernel(long long limit, int32_t* status) {
   if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, limit)) atomicOr(status, DLRM_FLAG_TIMEOUT);
 }
 
+// Below 2^24 it runs pair_from_flat_small, the decoder dots_from_smem runs on
+// the tile index in the interaction and fused kernels; from 2^24 on, the
+// 64-bit pair_from_flat.
 __global__ void pair_decode_kernel(int64_t p0, int64_t count, int32_t* __restrict__ i_out,
                                    int32_t* __restrict__ j_out) {
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < count;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t p = p0 + e;
     int i, j;
-    pair_from_flat(p0 + e, i, j);
+    if (p < kPairSmallLimit) {
+      pair_from_flat_small(static_cast<int>(p), i, j);
+    } else {
+      pair_from_flat(p, i, j);
+    }
     i_out[e] = i;
     j_out[e] = j;
   }
@@ -412,6 +420,10 @@ cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_
   choose_dot_shape(g.F, g.D, g.B, want, std::min<int64_t>(smem_limit, 64 * 1024) - order_bytes,
                    a.S, a.lq);
   if (a.S * g.F >= (1 << kSortTaskBits)) a.g.bp.balance = 0;
+  // bag ordering only changes the order of work: drop it when its shared
+  // memory would not fit next to the features
+  if (a.g.bp.balance && a.S * interact_smem_per_sample(g.F, g.D) + order_bytes > smem_limit)
+    a.g.bp.balance = 0;
   a.smem = a.S * interact_smem_per_sample(g.F, g.D) + (a.g.bp.balance ? order_bytes : 0);
   if (a.smem > smem_limit) return cudaErrorInvalidValue;
   switch (g.loader) {

@@ -309,13 +309,22 @@ def test_checked_entry_points_flag_and_skip(ops):
 # ------------------------------------------------------------------ integer work
 
 def test_pair_decoder_exhaustive(ops):
-    """Every flat index of every triangle up to 4097 features, bit-exact."""
-    nf = 4097
-    pi, pj = oracle.pair_list(nf)
-    gi, gj = ops.pair_decode(0, len(pi))
+    """Every flat index p < 2^24 through pair_from_flat_small, the decoder the
+    interaction and fused kernels run on their pair-tile index (tile indices
+    stay below 2145 at 256 tables), against the oracle's nested-loop
+    enumeration of the triangle of 5794 features, bit-exact."""
+    n = 1 << 24
+    pi, pj = oracle.pair_list(5794)
+    assert len(pi) >= n
+    gi, gj = ops.pair_decode(0, n)
     torch.cuda.synchronize()
-    assert np.array_equal(gi.cpu().numpy(), pi)
-    assert np.array_equal(gj.cpu().numpy(), pj)
+    assert np.array_equal(gi.cpu().numpy(), pi[:n])
+    assert np.array_equal(gj.cpu().numpy(), pj[:n])
+    # across the switch to the 64-bit decoder at 2^24
+    gi, gj = ops.pair_decode(n - 4096, 8192)
+    torch.cuda.synchronize()
+    assert np.array_equal(gi.cpu().numpy(), pi[n - 4096:n + 4096])
+    assert np.array_equal(gj.cpu().numpy(), pj[n - 4096:n + 4096])
 
 
 def test_pair_decoder_near_int32_limit(ops):
