@@ -81,11 +81,12 @@ enum FusedOrder { kOrderNone = 0, kOrderRuns = 1, kOrderByFlag = 2 };
 // Bags of different lengths: a warp runs to its longest bag and the block to
 // its slowest warp. So the block's bags are taken in runs of 32; a warp
 // reads the bounds of the run that holds its slots, sorts the run longest
-// first (key: length, then bag number, so keys are unique; a run of equal
-// lengths keeps its order), and the rounds walk the sorted runs in
-// alternating direction: the lane groups of a warp get bags of similar
-// length, and a warp that drew long bags in one round draws short ones in
-// the next. Every warp sorts the same runs the same way, so no block-wide
+// first (key: length, then bag number, so keys are unique and equal lengths
+// order by bag number, higher first; a run whose bags all have one length is
+// not sorted and keeps ascending bag order), and the rounds walk the sorted
+// runs in alternating direction: the lane groups of a warp get bags of
+// similar length, and a warp that drew long bags in one round draws short
+// ones in the next. Every warp sorts the same runs the same way, so no block-wide
 // barrier is needed; each warp keeps its sorted run in its own 96 ints of
 // shared memory after the features (rank r: bag, start, length).
 template <class LD, int G, int CPL, int POOL, int ORDER>

@@ -318,3 +318,33 @@ def test_max_ties_keep_the_earlier_entry(ops, dtype):
     torch.cuda.synchronize()
     assert_bits_equal(out, ref, "max ties, embbag_pool_multi")
     assert_bits_equal(fp, ref, "max ties, fused pooled")
+
+
+def test_ordering_dropped_when_its_shared_memory_does_not_fit(ops):
+    """A shape whose features fill the block's shared memory to within the
+    768 bytes the bag ordering would add: the general (ragged) entry point
+    still runs, without the ordering, and matches the oracle."""
+    dev = torch.cuda.current_device()
+    limit = torch.cuda.get_device_properties(dev).shared_memory_per_block_optin
+
+    def per_sample(F, D):
+        f1p = 4 * ((F + 1 + 3) // 4)
+        return f1p * (4 * ((D + 3) // 4) + 4) * 4
+
+    shape = next(((F, D) for F in range(200, 257) for D in range(200, 600)
+                  if limit - 768 < per_sample(F, D) <= limit), None)
+    assert shape is not None, limit
+    F, D = shape
+    B, N, T = 3, 20, 12
+    weights, idx, off, psw, dense = _case(5, B, F, N, D, T, torch.float32, False, 0.3)
+    ws = [_host_bits(w) for w in weights]
+    ref = oracle.embbag_pool_multi(ws, idx, off, B)
+    fp, fi = ops.sparse_interact_pool(weights, torch.from_numpy(idx).to(DEV),
+                                      torch.from_numpy(off).to(DEV), dense, concat_dense=True)
+    torch.cuda.synchronize()
+    what = f"F={F} D={D} shared memory {per_sample(F, D)} of {limit}"
+    assert_bits_equal(fp, ref, what + " pooled")
+    ref_i, _, bound = oracle.interact_lower_tri(dense.cpu().numpy(), ref, concat_dense=True,
+                                                with_f64=True)
+    assert_bits_equal(fi[:, :D], ref_i[:, :D], what + " dense part")
+    assert_dots_close(fi[:, D:], ref_i[:, D:], bound, what + " dots")
