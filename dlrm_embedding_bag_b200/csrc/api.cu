@@ -384,6 +384,8 @@ const char* dlrm_status_string(int status) {
     case DLRM_ERR_CUDA: return "a CUDA call or kernel launch failed";
     case DLRM_ERR_ARG: return "invalid argument";
     case DLRM_ERR_TIMEOUT: return "a bounded wait on an asynchronous copy ran out";
+    case DLRM_ERR_SCRATCH:
+      return "the call needs more device staging than the library's fixed array holds";
     default: return "unknown status";
   }
 }

@@ -30,7 +30,10 @@ STATUS = {
     -7: "DLRM_ERR_CUDA",
     -8: "DLRM_ERR_TIMEOUT",
     -9: "DLRM_ERR_ARG",
+    -10: "DLRM_ERR_SCRATCH",
 }
+# Bytes of the library's own device staging (dlrm_sparse_interact_host_static).
+STATIC_SCRATCH_BYTES = 32 << 20
 GATHER_PATHS = {"auto": 0, "ldg": 1, "tma": 2, "pipe": 3}
 FLAG_INDEX_OOB = 1
 FLAG_OFFSETS = 2
@@ -50,6 +53,7 @@ SIGNATURES = {
                                        _P, _P, _P]),
     "embbag_pool_multi": (_I, [_P, _I, _P, _P, _I, _I, _I, _P, _P, _P]),
     "dlrm_sparse_interact_pool": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _P, _P, _I, _P, _P]),
+    "dlrm_sparse_interact_host_static": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "dlrm_pair_decode": (_I, [_I64, _I64, _P, _P, _P]),
     "dlrm_set_gather_path": (_I, [_I]),
     "dlrm_last_gather_path": (_I, []),
@@ -475,6 +479,41 @@ class HostStage:
             _host(pooled_host, "pooled_host", torch.float32) if pooled_host is not None else None,
             _host(inter_host, "inter_host", torch.float32), _stream())
         _check(rc, "dlrm_sparse_interact_host")
+
+
+def sparse_interact_host_static(weights: Sequence[torch.Tensor], indices_host: torch.Tensor,
+                                offsets_host: torch.Tensor, dense_host: torch.Tensor, L: int,
+                                inter_host: torch.Tensor, *, concat_dense: bool = False,
+                                pooled_host: Optional[torch.Tensor] = None) -> None:
+    """The whole stage from host buffers through ``dlrm_sparse_interact_host_static``:
+    the device staging is the library's own fixed array, so nothing is
+    allocated on the device (for callers that cannot allocate device memory).
+
+    Enqueued on the current stream; the host outputs are valid once the
+    stream has reached this point. Calls that overlap on the GPU share the
+    array and race: keep them on one stream. Staging beyond
+    ``STATIC_SCRATCH_BYTES`` raises ``DLRM_ERR_SCRATCH``.
+    """
+    arr, _, F, D = _table_ptrs(weights)
+    if offsets_host.dim() != 2 or offsets_host.shape[0] != F:
+        raise ValueError(f"offsets_host must be (F={F}, B)")
+    B = offsets_host.shape[1]
+    P = (F + 1) * F // 2
+    if indices_host.numel() != F * B * L:
+        raise ValueError(f"indices_host must hold F*B*L = {F * B * L} entries")
+    if tuple(dense_host.shape) != (B, D):
+        raise ValueError(f"dense_host must be ({B}, {D})")
+    if inter_host.numel() != B * (D + P if concat_dense else P):
+        raise ValueError("inter_host has the wrong size")
+    if pooled_host is not None and pooled_host.numel() != B * F * D:
+        raise ValueError("pooled_host must be (B, F, D)")
+    ip = _host(indices_host, "indices_host", torch.int32) if F * B * L else None
+    rc = _lib.dlrm_sparse_interact_host_static(
+        arr, ip, _host(offsets_host, "offsets_host", torch.int32),
+        _host(dense_host, "dense_host", torch.float32), B, F, L, D, 1 if concat_dense else 0,
+        _host(pooled_host, "pooled_host", torch.float32) if pooled_host is not None else None,
+        _host(inter_host, "inter_host", torch.float32), _stream())
+    _check(rc, "dlrm_sparse_interact_host_static")
 
 
 class HostPipeline:

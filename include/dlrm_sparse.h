@@ -77,7 +77,10 @@ typedef enum {
                                       dlrm_last_cuda_error() */
     DLRM_ERR_TIMEOUT = -8,         /* (device flag) a bounded wait on an asynchronous
                                       copy ran out; the results are not valid */
-    DLRM_ERR_ARG = -9              /* any other invalid argument (e.g. count < 0) */
+    DLRM_ERR_ARG = -9,             /* any other invalid argument (e.g. count < 0) */
+    DLRM_ERR_SCRATCH = -10         /* the call needs more device staging than the
+                                      library's fixed array holds
+                                      (dlrm_sparse_interact_host_static) */
 } dlrm_status_t;
 
 /* Bits that the checked (_ex) entry points OR into *status_dev. */
@@ -259,6 +262,52 @@ DLRM_API int dlrm_sparse_interact_host(const float* const* weights, const int32_
                                        int32_t* offsets_dev, float* dense_dev, float* pooled_dev,
                                        float* inter_dev, float* pooled_host, float* inter_host,
                                        dlrm_stream_t stream);
+
+/*
+ * dlrm_sparse_interact_host_static -- dlrm_sparse_interact_host for callers
+ * that cannot allocate device memory: the device staging is a fixed array of
+ * DLRM_STATIC_SCRATCH_BYTES inside this library, so the caller passes only
+ * host buffers and the call makes no cudaMalloc, cudaFree or other
+ * allocation. The paper and pages this library follows have no counterpart;
+ * it is an interface addition. Who needs it: a plugin or callback run by a
+ * host framework that owns the device's memory (a serving runtime, or a
+ * PyTorch process whose caching allocator already holds the free memory, so
+ * a raw cudaMalloc fails or fragments it); code running while a CUDA graph is
+ * being captured elsewhere on the device, where cudaMalloc is not allowed;
+ * and latency-critical loops, where cudaMalloc/cudaFree would synchronise the
+ * device on every batch.
+ *   weights, B, F, L, D, concat_dense : as for dlrm_sparse_interact.
+ *   indices_host, offsets_host, dense_host : host inputs, layouts as above.
+ *   pooled_host  : host (B, F, D) or NULL (then the pooled vectors are not
+ *                  written anywhere).
+ *   inter_host   : host interaction rows, (B, P) or (B, D + P).
+ * On `stream`: the inputs are copied into the array, the fused kernel runs
+ * there, and the interaction rows (and pooled vectors) are copied back. It
+ * returns once that is enqueued; host outputs are valid when the stream has
+ * reached that point. Page-locked host buffers keep the copies asynchronous.
+ * Results are bit-identical to dlrm_sparse_interact_host's.
+ * Limit: the staging of one call, [indices | offsets | dense] then the
+ * interaction rows then the pooled vectors (these two on 256-byte
+ * boundaries), must fit in DLRM_STATIC_SCRATCH_BYTES, else DLRM_ERR_SCRATCH
+ * and nothing is enqueued. Every GPU that loads the library keeps the array
+ * until the process exits.
+ * Sharing: every call on a device uses the same array, and the array keeps
+ * what the last call left there (nothing in it has to start at zero: a call
+ * writes every byte it reads). Calls whose work overlaps on the GPU (two
+ * host threads, or two streams with no ordering between them) race on it and
+ * corrupt each other's results: run them on one stream, or order them.
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current), which may load the
+ * library's code onto the device. Make that first call before any stream
+ * capture on that device.
+ */
+#define DLRM_STATIC_SCRATCH_BYTES (32u << 20)
+DLRM_API int dlrm_sparse_interact_host_static(const float* const* weights,
+                                              const int32_t* indices_host,
+                                              const int32_t* offsets_host,
+                                              const float* dense_host, int B, int F, int L, int D,
+                                              int concat_dense, float* pooled_host,
+                                              float* inter_host, dlrm_stream_t stream);
 
 /*
  * dlrm_pair_decode -- the kernels' flat-index decoder, exposed so it can be

@@ -36,7 +36,7 @@ def test_header_declares_the_stage_entry_points():
     names = _declared()
     assert {"embbag_sum_multi", "interact_lower_tri", "dlrm_sparse_interact"} <= names
     assert {"dlrm_linear_bf16", "dlrm_f32_to_bf16"} <= names
-    assert len(names) == 18
+    assert len(names) == 19
 
 
 def test_library_exports_every_declared_symbol(ops):
@@ -148,6 +148,25 @@ def test_fused_and_interact_host_checks(ops):
     assert lib.dlrm_pair_decode(0, -1, FAKE, FAKE, None) == -9
     assert lib.dlrm_pair_decode((1 << 31) - 2, 5, FAKE, FAKE, None) == -9
     assert lib.dlrm_pair_decode(0, 5, None, FAKE, None) == -1
+    assert lib.dlrm_launch_count() == 0
+
+
+def test_static_staging_host_checks(ops):
+    """The host entry point with library-owned staging rejects missing host
+    buffers and any call whose staging exceeds its fixed array, before any CUDA
+    call."""
+    lib = ops._lib
+    w = _ptrs(FAKE, FAKE)
+    call = lib.dlrm_sparse_interact_host_static
+    assert call(w, FAKE, FAKE, FAKE, 4, 2, 2, 8, 0, None, None, None) == -1
+    assert call(w, None, FAKE, FAKE, 4, 2, 2, 8, 0, None, FAKE, None) == -1
+    assert call(w, FAKE, FAKE, FAKE, 4, 0, 2, 8, 0, None, FAKE, None) == -4
+    # 2 tables, B = 1 << 20, L = 4: 32 MiB of indices alone
+    assert call(w, FAKE, FAKE, FAKE, 1 << 20, 2, 4, 8, 0, None, FAKE, None) == -10
+    # pooled vectors that no longer fit once asked for
+    B, D = 1 << 14, 256  # inputs 16.2 MiB, dots 0.2 MiB, pooled 32 MiB
+    assert call(w, FAKE, FAKE, FAKE, B, 2, 1, D, 0, FAKE, FAKE, None) == -10
+    assert lib.dlrm_status_string(-10).startswith(b"the call needs more device staging")
     assert lib.dlrm_launch_count() == 0
 
 
