@@ -21,6 +21,10 @@ ctypes and marshals numpy arrays. What each function follows on the pages
   (feature 0 = dense vector, features 1..N = pooled embeddings).
 * :meth:`Oracle.pair_list` -- dlrm_interact.rs, pair-table comment: row-major
   over i then j, the torch.tril_indices(F, F, -1) order.
+* :meth:`Oracle.linear_bf16` / :meth:`Oracle.linear_f32a` -- matmul2d.rs:
+  the linear-with-bias layer, its ReLU / sigmoid forms and the split-A form;
+  ``linear_f32a`` is the pages' own arithmetic (f32 activations, f32 or bf16
+  weights), ``linear_bf16`` the bf16-operand variant.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` to facts fixed by
 the pages and by mathematics, not by this code.
@@ -101,6 +105,9 @@ class Oracle:
         lib.oracle_linear_bf16.argtypes = [P, L64, L64, P, L64, L64, P, L64, P, L64, L64, I, P, P,
                                            P]
         lib.oracle_linear_bf16.restype = I
+        lib.oracle_linear_f32a.argtypes = [P, L64, L64, P, L64, L64, P, I, L64, P, L64, L64, I, P,
+                                           P, P]
+        lib.oracle_linear_f32a.restype = I
         self.lib = lib
         self.path = libpath
 
@@ -239,6 +246,40 @@ class Oracle:
         return out, pre, bnd
 
 
+    def linear_f32a(self, a_lo: np.ndarray, w: np.ndarray, bias=None, act: int = 0, *,
+                    a_hi: Optional[np.ndarray] = None, k_lo: Optional[int] = None,
+                    k_hi: Optional[int] = None):
+        """One MLP layer ``act(A W^T + bias)`` with f32 activations, exactly (fp64).
+
+        ``a_lo`` ``(M, >=k_lo)`` and ``a_hi`` ``(M, >=k_hi)`` (optional) are f32;
+        ``w`` ``(N, >=k_lo+k_hi)`` is f32 values or uint16 bf16 bit patterns
+        (the dtype says which); ``bias`` ``(N,)`` f32 or None; ``act`` as for
+        :meth:`linear_bf16`. Returns ``(out, pre, bound)`` like it.
+        """
+        a_lo = _f32(a_lo)
+        w_bf16 = np.asarray(w).dtype == np.uint16
+        w = np.ascontiguousarray(w, dtype=np.uint16) if w_bf16 else _f32(w)
+        M, lda_lo = a_lo.shape
+        N, ldw = w.shape
+        k_lo = lda_lo if k_lo is None else k_lo
+        if a_hi is not None:
+            a_hi = _f32(a_hi)
+            lda_hi = a_hi.shape[1]
+            k_hi = lda_hi if k_hi is None else k_hi
+        else:
+            lda_hi, k_hi = 0, 0
+        b = None if bias is None else _f32(bias)
+        out = np.empty((M, N), dtype=np.float64)
+        pre = np.empty((M, N), dtype=np.float64)
+        bnd = np.empty((M, N), dtype=np.float64)
+        rc = self.lib.oracle_linear_f32a(_ptr(a_lo), lda_lo, k_lo, _ptr(a_hi), lda_hi, k_hi,
+                                         _ptr(w), 1 if w_bf16 else 0, ldw, _ptr(b), M, N, act,
+                                         _ptr(out), _ptr(pre), _ptr(bnd))
+        if rc != OK:
+            raise OracleError(rc, "linear_f32a")
+        return out, pre, bnd
+
+
 _default = None
 
 
@@ -272,3 +313,7 @@ def embbag_pool_multi(*a, **k):
 
 def linear_bf16(*a, **k):
     return default().linear_bf16(*a, **k)
+
+
+def linear_f32a(*a, **k):
+    return default().linear_f32a(*a, **k)

@@ -332,6 +332,25 @@ int oracle_sparse_interact(const float* const* weights, const int64_t* rows,
 }
 
 /*
+ * The end of a linear layer for one output: add the bias to the exact sum s
+ * (and |bias| to the magnitude mag), apply the activation to acc + bias
+ * (0 none, 1 ReLU max(x, 0), 2 sigmoid 1 / (1 + exp(-x))) and store.
+ */
+static void linear_finish(double s, double mag, const float* bias, int64_t n, int act,
+                          int64_t at, double* out, double* pre, double* bound) {
+    if (bias) {
+        s += (double)bias[n];
+        mag += fabs((double)bias[n]);
+    }
+    double y = s;
+    if (act == 1) y = (s > 0.0) ? s : 0.0;
+    if (act == 2) y = 1.0 / (1.0 + exp(-s));
+    out[at] = y;
+    if (pre) pre[at] = s;
+    if (bound) bound[at] = mag;
+}
+
+/*
  * One DLRMv1 MLP layer, y = act(A W^T + bias), the linear-with-bias layer the
  * pages' matmul2d.rs page describes (linear_bias, linear_bias_relu,
  * linear_bias_sigmoid): A is (M, K), W is (N, K) (the nn.Linear weight
@@ -378,16 +397,53 @@ int oracle_linear_bf16(const uint16_t* a_lo, int64_t lda_lo, int64_t k_lo,
                 s += t;
                 mag += (t < 0.0) ? -t : t;
             }
-            if (bias) {
-                s += (double)bias[n];
-                mag += fabs((double)bias[n]);
+            linear_finish(s, mag, bias, n, act, m * N + n, out, pre, bound);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * One DLRMv1 MLP layer with f32 activations: the mixed-precision linear the
+ * pages' matmul2d.rs page describes (A is F32 (M, K), the weights are BF16
+ * or F32 (N, K) by the kernel's weight_dtype, the result F32 (M, N)), with the
+ * bias and activation of oracle_linear_bf16 and the same split form
+ * (columns 0..k_lo-1 of A from a_lo, k_lo..K-1 from a_hi).
+ *   a_lo, a_hi : f32 rows (row pitches lda_lo, lda_hi); a_hi NULL when k_hi == 0
+ *   w          : (N, ldw) rows of f32 values (w_bf16 == 0) or of bf16 bit
+ *                patterns (w_bf16 != 0)
+ *   bias, act, out, pre, bound : as for oracle_linear_bf16
+ * A product of two f32 values has at most 48 significant bits, so it is exact
+ * in fp64; the sum is taken in fp64 in ascending k.
+ */
+static double weight_at(const void* w, int w_bf16, int64_t i) {
+    if (w_bf16) return (double)bf16_bits_to_f32(((const uint16_t*)w)[i]);
+    return (double)((const float*)w)[i];
+}
+
+int oracle_linear_f32a(const float* a_lo, int64_t lda_lo, int64_t k_lo,
+                       const float* a_hi, int64_t lda_hi, int64_t k_hi,
+                       const void* w, int w_bf16, int64_t ldw, const float* bias,
+                       int64_t M, int64_t N, int act, double* out, double* pre,
+                       double* bound) {
+    if (M < 1 || N < 1 || k_lo < 1 || k_hi < 0 || act < 0 || act > 2) return ORACLE_BAD_ARG;
+    if (!a_lo || !w || !out || (k_hi > 0 && !a_hi)) return ORACLE_BAD_ARG;
+    if (lda_lo < k_lo || (k_hi > 0 && lda_hi < k_hi) || ldw < k_lo + k_hi) return ORACLE_BAD_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double s = 0.0, mag = 0.0;
+            for (int64_t k = 0; k < k_lo; ++k) {
+                const double t = (double)a_lo[m * lda_lo + k] * weight_at(w, w_bf16, n * ldw + k);
+                s += t;
+                mag += (t < 0.0) ? -t : t;
             }
-            double y = s;
-            if (act == 1) y = (s > 0.0) ? s : 0.0;
-            if (act == 2) y = 1.0 / (1.0 + exp(-s));
-            out[m * N + n] = y;
-            if (pre) pre[m * N + n] = s;
-            if (bound) bound[m * N + n] = mag;
+            for (int64_t k = 0; k < k_hi; ++k) {
+                const double t =
+                    (double)a_hi[m * lda_hi + k] * weight_at(w, w_bf16, n * ldw + k_lo + k);
+                s += t;
+                mag += (t < 0.0) ? -t : t;
+            }
+            linear_finish(s, mag, bias, n, act, m * N + n, out, pre, bound);
         }
     }
     return ORACLE_OK;

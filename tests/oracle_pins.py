@@ -642,6 +642,135 @@ def pin_linear_rejects(orc):
     _expect_code(lambda: orc.linear_bf16(a, w, None, 0, k_lo=5), BAD_ARG)
 
 
+# ---------------------------------------------------------------------------
+# The MLP layer with f32 activations, the pages' own arithmetic (matmul2d.rs:
+# A F32 (M, K) times weights BF16 or F32 (N, K), result F32).
+
+
+def pin_linear_f32a_exact_integers(orc):
+    """Integer operands of up to 12 bits (exact in f32 and, for the weights,
+    in bf16): the layer is an exact integer matmul, with f32 and bf16 weights."""
+    rng = np.random.default_rng(81)
+    for (M, N, K) in [(1, 1, 1), (3, 5, 7), (17, 9, 40)]:
+        a = rng.integers(-2048, 2049, size=(M, K))
+        w = rng.integers(-128, 129, size=(N, K))
+        b = rng.integers(-500, 501, size=N)
+        want = a.astype(np.int64) @ w.astype(np.int64).T + b
+        wantb = np.abs(a).astype(np.int64) @ np.abs(w).astype(np.int64).T + np.abs(b)
+        for wt in (w.astype(np.float32), _bf16_bits(w)):
+            out, pre, bound = orc.linear_f32a(a.astype(np.float32), wt, b.astype(np.float32))
+            assert np.array_equal(pre, want.astype(np.float64))
+            assert np.array_equal(out, want.astype(np.float64))
+            assert np.array_equal(bound, wantb.astype(np.float64))
+
+
+def pin_linear_f32a_keeps_every_bit_of_a(orc):
+    """Activations with all 24 significant bits enter unrounded, and so do
+    f32 weights: (1 + 2^-23)(1 + 2^-7) = 1 + 2^-7 + 2^-23 + 2^-30 exactly (a
+    bf16 activation would drop the 2^-23 and 2^-30 terms, an f32 product the
+    2^-30 term)."""
+    a = np.array([[1.0 + 2.0 ** -23, 3.0 * (1.0 + 2.0 ** -22)]], np.float32)
+    w = np.array([[1.0 + 2.0 ** -7, 0.0], [0.0, 1.0 + 2.0 ** -20]], np.float32)
+    assert float(a[0, 0]) == 1.0 + 2.0 ** -23
+    _, pre, _ = orc.linear_f32a(a, w)
+    assert pre[0, 0] == 1.0 + 2.0 ** -7 + 2.0 ** -23 + 2.0 ** -30
+    assert pre[0, 1] == 3.0 * (1.0 + 2.0 ** -22) * (1.0 + 2.0 ** -20)
+    # the same with the weights' bf16 bit patterns (1 + 2^-7 is a bf16 value)
+    _, pre16, _ = orc.linear_f32a(a, _bf16_bits(w[:1]))
+    assert pre16[0, 0] == 1.0 + 2.0 ** -7 + 2.0 ** -23 + 2.0 ** -30
+
+
+def pin_linear_f32a_vs_torch_fp64(orc):
+    """Random f32 activations, f32 and bf16 weights, against torch's linear in fp64."""
+    rng = np.random.default_rng(82)
+    for (M, N, K) in [(4, 3, 16), (33, 20, 100)]:
+        a = rng.normal(0, 1, size=(M, K)).astype(np.float32)
+        wf = rng.normal(0, 0.1, size=(N, K)).astype(np.float32)
+        wb = _bf16_bits(wf)
+        b = rng.normal(0, 0.1, size=N).astype(np.float32)
+        ta = torch.from_numpy(a.astype(np.float64))
+        tb = torch.from_numpy(b.astype(np.float64))
+        for w, wvals in ((wf, wf), (wb, _bf16_values(wb))):
+            tw = torch.from_numpy(wvals.astype(np.float64))
+            want = torch.nn.functional.linear(ta, tw, tb).numpy()
+            out, _, bound = orc.linear_f32a(a, w, b, 0)
+            assert np.all(np.abs(out - want) <= 1e-12 * bound + 1e-300)
+            want0 = torch.nn.functional.linear(ta, tw).numpy()
+            out0, _, _ = orc.linear_f32a(a, w, None, 0)
+            assert np.all(np.abs(out0 - want0) <= 1e-12 * bound + 1e-300)
+
+
+def pin_linear_f32a_bf16_weights_are_their_widening(orc):
+    """bf16 weight patterns give the layer of their exact f32 widening, and on
+    bf16-valued activations the layer equals the bf16-operand layer."""
+    rng = np.random.default_rng(83)
+    a16 = _bf16_bits(rng.normal(0, 1, size=(7, 12)))
+    w16 = _bf16_bits(rng.normal(0, 1, size=(5, 12)))
+    b = rng.normal(0, 1, size=5).astype(np.float32)
+    for act in (0, 1, 2):
+        x = orc.linear_f32a(_bf16_values(a16), w16, b, act)
+        y = orc.linear_f32a(_bf16_values(a16), _bf16_values(w16), b, act)
+        z = orc.linear_bf16(a16, w16, b, act)
+        for u, v, t in zip(x, y, z):
+            assert np.array_equal(u, v) and np.array_equal(u, t)
+
+
+def pin_linear_f32a_activations(orc):
+    """ReLU is torch.relu and sigmoid is scipy's expit of the pre-activation."""
+    from scipy.special import expit
+
+    rng = np.random.default_rng(84)
+    a = rng.normal(0, 1, size=(9, 24)).astype(np.float32)
+    w = rng.normal(0, 0.5, size=(7, 24)).astype(np.float32)
+    b = rng.normal(0, 0.5, size=7).astype(np.float32)
+    _, pre, _ = orc.linear_f32a(a, w, b, 0)
+    relu, pre1, _ = orc.linear_f32a(a, w, b, 1)
+    sig, pre2, _ = orc.linear_f32a(a, w, b, 2)
+    assert np.array_equal(pre, pre1) and np.array_equal(pre, pre2)
+    assert (pre < 0).any() and (pre > 0).any()
+    assert np.array_equal(relu, torch.relu(torch.from_numpy(pre)).numpy())
+    assert np.allclose(sig, expit(pre), rtol=1e-15, atol=0)
+
+
+def pin_linear_f32a_split_equals_concat(orc):
+    """Split A equals the layer on the concatenation; weight column k_lo + k
+    multiplies a_hi's column k; only the first k columns of pitched rows count."""
+    rng = np.random.default_rng(85)
+    M, N, k_lo, k_hi = 6, 5, 3, 11
+    a_lo = rng.normal(0, 1, size=(M, k_lo)).astype(np.float32)
+    a_hi = rng.normal(0, 1, size=(M, k_hi)).astype(np.float32)
+    w = rng.normal(0, 1, size=(N, k_lo + k_hi)).astype(np.float32)
+    b = rng.normal(0, 1, size=N).astype(np.float32)
+    cat = np.concatenate([a_lo, a_hi], axis=1)
+    for act in (0, 1, 2):
+        want = orc.linear_f32a(cat, w, b, act)
+        got = orc.linear_f32a(a_lo, w, b, act, a_hi=a_hi)
+        for x, y in zip(want, got):
+            assert np.array_equal(x, y)
+    for k in range(k_hi):
+        e = np.zeros((1, k_hi), np.float32)
+        e[0, k] = 1.0
+        _, pre, _ = orc.linear_f32a(np.zeros((1, k_lo), np.float32), w, None, 0, a_hi=e)
+        assert np.array_equal(pre[0], w[:, k_lo + k].astype(np.float64))
+    junk = np.full((M, 3), 1e30, np.float32)
+    wjunk = np.full((N, 3), -1e30, np.float32)
+    want = orc.linear_f32a(cat, w, None, 0)
+    got = orc.linear_f32a(np.concatenate([cat, junk], 1), np.concatenate([w, wjunk], 1), None, 0,
+                          k_lo=k_lo + k_hi)
+    for x, y in zip(want, got):
+        assert np.array_equal(x, y)
+
+
+def pin_linear_f32a_rejects(orc):
+    from oracle import BAD_ARG
+
+    a = np.zeros((2, 4), np.float32)
+    w = np.zeros((3, 4), np.float32)
+    _expect_code(lambda: orc.linear_f32a(a, w, None, 3), BAD_ARG)
+    _expect_code(lambda: orc.linear_f32a(a, np.zeros((3, 3), np.float32), None, 0), BAD_ARG)
+    _expect_code(lambda: orc.linear_f32a(a, w, None, 0, k_lo=5), BAD_ARG)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 

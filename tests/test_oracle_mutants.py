@@ -81,6 +81,23 @@ MUTANTS = {
     "linear_sigmoid_sign": [("y = 1.0 / (1.0 + exp(-s));", "y = 1.0 / (1.0 + exp(s));")],
     "linear_a_row_pitch_ignored": [("bf16_bits_to_f32(a_lo[m * lda_lo + k])",
                                     "bf16_bits_to_f32(a_lo[m * k_lo + k])")],
+    "linear_f32a_activation_narrowed": [
+        ("const double t = (double)a_lo[m * lda_lo + k] * weight_at(w, w_bf16, n * ldw + k);",
+         "const double t = (double)(float)((double)(int)(a_lo[m * lda_lo + k] * 256.0f) / 256.0)"
+         " * weight_at(w, w_bf16, n * ldw + k);")],
+    "linear_f32a_product_rounded_to_f32": [
+        ("const double t = (double)a_lo[m * lda_lo + k] * weight_at(w, w_bf16, n * ldw + k);",
+         "const double t = (double)(float)((double)a_lo[m * lda_lo + k] *"
+         " weight_at(w, w_bf16, n * ldw + k));")],
+    "linear_f32a_hi_part_reads_lo_weights": [("weight_at(w, w_bf16, n * ldw + k_lo + k)",
+                                               "weight_at(w, w_bf16, n * ldw + k)")],
+    "linear_f32a_weight_transposed": [("weight_at(w, w_bf16, n * ldw + k);",
+                                        "weight_at(w, w_bf16, k * ldw + n);")],
+    "linear_f32a_bf16_weights_read_as_integers": [
+        ("return (double)bf16_bits_to_f32(((const uint16_t*)w)[i]);",
+         "return (double)((const uint16_t*)w)[i];")],
+    "linear_f32a_a_row_pitch_ignored": [("(double)a_lo[m * lda_lo + k]",
+                                         "(double)a_lo[m * k_lo + k]")],
     "general_pooling_table_layout_transposed": [
         ("out[((int64_t)b * F + k) * D + d] = acc;", "out[((int64_t)k * B + b) * D + d] = acc;")],
 }
