@@ -634,11 +634,27 @@ def run_mlp(args, w: syn.Workload):
                 ms = timeit(fn, args.steps, args.warmup)
                 flops = 2.0 * B * N * K
                 layers.append({"mlp": name, "layer": i, "B": B, "K": K, "N": N,
-                               "split_a": bool(split and i == 0), "act": act, "us": 1e3 * ms,
-                               "tflops": flops / (ms / 1e3) / 1e12})
+                               "split_a": bool(split and i == 0), "act": act, "mode": "bf16",
+                               "us": 1e3 * ms, "tflops": flops / (ms / 1e3) / 1e12})
+                # the same layer with f32 activations (three exact bf16 planes per
+                # value: three times the tensor work of the bf16 layer)
+                p_lo = mlp.split_bf16x3(a_lo.float())
+                p_hi = mlp.split_bf16x3(a_hi.float()) if a_hi is not None else None
+                yp = None if last_layer else mlp.planes_empty(B, N, dev)
+
+                def fn32(p_lo=p_lo, p_hi=p_hi, wt=wt, b=b, act=act, y32=y32, yp=yp):
+                    mlp.linear_f32a(p_lo, wt, b, act, a_hi=p_hi, out_f32=y32, out_planes=yp,
+                                    f32=y32 is not None, planes=yp is not None)
+
+                ms32 = timeit(fn32, args.steps, args.warmup)
+                layers.append({"mlp": name, "layer": i, "B": B, "K": K, "N": N,
+                               "split_a": bool(split and i == 0), "act": act, "mode": "f32",
+                               "us": 1e3 * ms32, "tflops": flops / (ms32 / 1e3) / 1e12,
+                               "tensor_tflops": 3 * flops / (ms32 / 1e3) / 1e12})
     # the full forward at the workload's batch
-    bottom = mlp.MLP(syn.make_mlp_layers(bottom_w[0], bottom_w[1:], 7, dev))
-    top = mlp.MLP(syn.make_mlp_layers(top_w[0], top_w[1:], 8, dev, last="sigmoid"))
+    bottom = mlp.MLP(syn.make_mlp_layers(bottom_w[0], bottom_w[1:], 7, dev), mode="bf16")
+    top = mlp.MLP(syn.make_mlp_layers(top_w[0], top_w[1:], 8, dev, last="sigmoid"),
+                  mode="bf16")
     weights = syn.make_weights(w, dev)
     idx = torch.from_numpy(syn.make_indices(w)).to(dev)
     off = torch.from_numpy(syn.make_offsets(w)).to(dev)
@@ -658,11 +674,31 @@ def run_mlp(args, w: syn.Workload):
             graph_out = mlp.dlrm_forward(bottom, top, x, weights, idx, off, w.L)  # noqa: F841
     torch.cuda.current_stream().wait_stream(side)
     graph_ms = timeit(graph.replay, args.steps, args.warmup)
-    big = max(layers, key=lambda r: r["B"] * r["N"] * r["K"])
+    # the same forward with f32 activations throughout (the pages' arithmetic)
+    bottom32 = mlp.MLP(bottom.layers, mode="f32")
+    top32 = mlp.MLP(top.layers, mode="f32")
+    x32 = x.float().contiguous()
+    n0 = ops.launch_count()
+    mlp.dlrm_forward(bottom32, top32, x32, weights, idx, off, w.L)
+    fwd32_launches = ops.launch_count() - n0
+    fwd32_ms = timeit(lambda: mlp.dlrm_forward(bottom32, top32, x32, weights, idx, off, w.L),
+                      args.steps, args.warmup)
+    side32 = torch.cuda.Stream()
+    side32.wait_stream(torch.cuda.current_stream())
+    graph32 = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side32):
+        mlp.dlrm_forward(bottom32, top32, x32, weights, idx, off, w.L)
+        with torch.cuda.graph(graph32, stream=side32):
+            graph32_out = mlp.dlrm_forward(bottom32, top32, x32, weights, idx, off, w.L)  # noqa: F841
+    torch.cuda.current_stream().wait_stream(side32)
+    graph32_ms = timeit(graph32.replay, args.steps, args.warmup)
+    big = max((r for r in layers if r["mode"] == "bf16"), key=lambda r: r["B"] * r["N"] * r["K"])
+    big32 = max((r for r in layers if r["mode"] == "f32"), key=lambda r: r["B"] * r["N"] * r["K"])
     peaks = measured_peaks() or {}
     peak = float(peaks.get("bf16_tflops") or 1590.0)
     line = {
-        "metric": "DLRMv1 MLP layer TFLOP/s (bf16 tcgen05, f32 accumulate, fused bias+act)",
+        "metric": "DLRMv1 MLP layer TFLOP/s (tcgen05, f32 accumulate, fused bias+act; bf16 "
+                  "activations, and f32 activations as three exact bf16 planes)",
         "value": big["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16",
         "data": "synthetic",
@@ -680,6 +716,16 @@ def run_mlp(args, w: syn.Workload):
                     "graph_us": 1e3 * graph_ms, "graph_samples_per_s": w.B / (graph_ms / 1e3),
                     "steps": "bottom MLP (3 layers), fused sparse stage, z to bf16, top MLP "
                              "(3 layers, first split-A)"},
+        "forward_f32": {"workload": w.name, "B": w.B, "us": 1e3 * fwd32_ms,
+                        "samples_per_s": w.B / (fwd32_ms / 1e3), "gpu_launches": fwd32_launches,
+                        "graph_us": 1e3 * graph32_ms,
+                        "graph_samples_per_s": w.B / (graph32_ms / 1e3),
+                        "steps": "features split into planes, bottom MLP (3 f32-activation "
+                                 "layers), fused sparse stage, z split into planes, top MLP"},
+        "f32_layer": {"kernel": f"linear_f32a B={big32['B']} K={big32['K']} N={big32['N']}",
+                      "us": big32["us"], "tflops": big32["tflops"],
+                      "tensor_tflops": big32["tensor_tflops"],
+                      "tensor_frac": big32["tensor_tflops"] / peak},
     }
     print(json.dumps(line), flush=True)
     return 0

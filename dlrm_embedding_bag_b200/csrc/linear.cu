@@ -26,6 +26,7 @@
 #include <algorithm>
 #include <climits>
 #include <cstdint>
+#include <cstring>
 
 #include <cuda_bf16.h>
 
@@ -65,12 +66,36 @@ struct LinSmem {
   static constexpr int kTotal = kBars + (2 * kStages + 4) * 8 + 8 + 1024;  // + alignment
 };
 
+// Tensor maps of one launch: the A operand's parts (up to two, lo and hi)
+// times their bf16 planes (up to three), the weight planes (up to three), and
+// the two TMA-stored outputs.
+constexpr int kLinMaxAMaps = 6;
+constexpr int kLinMaxWMaps = 3;
+constexpr int kLinMaxSegs = 12;
+struct alignas(64) LinMaps {
+  CUtensorMap a[kLinMaxAMaps];
+  CUtensorMap w[kLinMaxWMaps];
+  CUtensorMap y32, y16;
+};
+
+// The K blocks of a tile, in order, are the concatenation of segments: nkb
+// blocks of A map `a` from column a_k0 times W map `w` from column w_k0. A
+// plain layer is one segment, the split form two (A_lo, then A_hi against W's
+// columns k_lo..), and an f32-activation layer one per (A plane, W plane)
+// product it sums.
+struct LinSeg {
+  int a, w, a_k0, w_k0, nkb;
+};
+
 struct LinearArgs {
   const float* bias;
   float* y_f32;
   uint16_t* y_bf16;
-  int64_t ldy_f32, ldy_bf16;
-  int M, N, k_lo, nkb_lo, nkb_hi;
+  uint16_t* y_planes;  // three bf16 planes of the f32 result (exact split), or null
+  int64_t ldy_f32, ldy_bf16, ldy_planes, splane_y;
+  int M, N;
+  LinSeg seg[kLinMaxSegs];
+  int nseg, nkb;
   int tiles_n, tiles;
   int tma_f32, tma_bf16;  // write that output through TMA stores (see the launcher)
   int32_t* status;
@@ -92,13 +117,39 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
          (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
 }
 
+// Exact split of an f32 value into three bf16 values, x = p0 + p1 + p2: p0 is x
+// with the low 16 bits of its encoding cleared (its top 8 significant bits),
+// p1 the same of the remainder x - p0, and p2 = x - p0 - p1, whose at most 8
+// significant bits fit a bf16 exactly. Both subtractions are exact.
+__device__ __forceinline__ void split_bf16x3(float x, uint16_t& p0, uint16_t& p1, uint16_t& p2) {
+  const uint32_t u = __float_as_uint(x);
+  const float h0 = __uint_as_float(u & 0xffff0000u);
+  const float r = __fsub_rn(x, h0);
+  const uint32_t v = __float_as_uint(r);
+  const float h1 = __uint_as_float(v & 0xffff0000u);
+  const float t = __fsub_rn(r, h1);
+  p0 = static_cast<uint16_t>(u >> 16);
+  p1 = static_cast<uint16_t>(v >> 16);
+  p2 = static_cast<uint16_t>(__float_as_uint(t) >> 16);
+}
+
+// Where the epilogue's direct stores go (outputs not written through TMA).
+struct LinOut {
+  float* y_f32;
+  uint16_t* y_bf16;
+  uint16_t* y_planes;
+  int64_t ldy_f32, ldy_bf16, ldy_planes, splane_y;
+  int M, N;
+};
+
 // Store 32 consecutive results of one row (columns nb .. nb+31, clipped to N).
-__device__ __forceinline__ void store_chunk32(const LinearArgs& args, int row, int nb,
-                                              const float (&v)[32], bool f32_vec, bool bf_vec) {
-  if (row >= args.M) return;
-  const bool whole = nb + 32 <= args.N;
-  if (args.y_f32 != nullptr) {
-    float* y = args.y_f32 + static_cast<int64_t>(row) * args.ldy_f32 + nb;
+__device__ __forceinline__ void store_chunk32(const LinOut& o, int row, int nb,
+                                              const float (&v)[32], bool f32_vec, bool bf_vec,
+                                              bool planes_vec) {
+  if (row >= o.M) return;
+  const bool whole = nb + 32 <= o.N;
+  if (o.y_f32 != nullptr) {
+    float* y = o.y_f32 + static_cast<int64_t>(row) * o.ldy_f32 + nb;
     if (whole && f32_vec) {
 #pragma unroll
       for (int q = 0; q < 8; ++q)
@@ -107,11 +158,38 @@ __device__ __forceinline__ void store_chunk32(const LinearArgs& args, int row, i
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (nb + j < args.N) y[j] = v[j];
+        if (nb + j < o.N) y[j] = v[j];
     }
   }
-  if (args.y_bf16 != nullptr) {
-    uint16_t* y = args.y_bf16 + static_cast<int64_t>(row) * args.ldy_bf16 + nb;
+  if (o.y_planes != nullptr) {
+    uint16_t* y0 = o.y_planes + static_cast<int64_t>(row) * o.ldy_planes + nb;
+    uint16_t* y1 = y0 + o.splane_y;
+    uint16_t* y2 = y1 + o.splane_y;
+    if (whole && planes_vec) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t a[4], b[4], c[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint16_t a0, a1, b0, b1, c0, c1;
+          split_bf16x3(v[8 * q + 2 * e], a0, b0, c0);
+          split_bf16x3(v[8 * q + 2 * e + 1], a1, b1, c1);
+          a[e] = a0 | (static_cast<uint32_t>(a1) << 16);
+          b[e] = b0 | (static_cast<uint32_t>(b1) << 16);
+          c[e] = c0 | (static_cast<uint32_t>(c1) << 16);
+        }
+        reinterpret_cast<uint4*>(y0)[q] = make_uint4(a[0], a[1], a[2], a[3]);
+        reinterpret_cast<uint4*>(y1)[q] = make_uint4(b[0], b[1], b[2], b[3]);
+        reinterpret_cast<uint4*>(y2)[q] = make_uint4(c[0], c[1], c[2], c[3]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (nb + j < o.N) split_bf16x3(v[j], y0[j], y1[j], y2[j]);
+    }
+  }
+  if (o.y_bf16 != nullptr) {
+    uint16_t* y = o.y_bf16 + static_cast<int64_t>(row) * o.ldy_bf16 + nb;
     if (whole && bf_vec) {
 #pragma unroll
       for (int q = 0; q < 4; ++q)
@@ -121,18 +199,14 @@ __device__ __forceinline__ void store_chunk32(const LinearArgs& args, int row, i
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (nb + j < args.N) y[j] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
+        if (nb + j < o.N) y[j] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
     }
   }
 }
 
 template <int BN, int ACT, bool F32S>
 __global__ void __launch_bounds__(kLinThreads, 1)
-    linear_bf16_kernel(const __grid_constant__ CUtensorMap map_a_lo,
-                       const __grid_constant__ CUtensorMap map_a_hi,
-                       const __grid_constant__ CUtensorMap map_w,
-                       const __grid_constant__ CUtensorMap map_y32,
-                       const __grid_constant__ CUtensorMap map_y16, const LinearArgs args) {
+    linear_bf16_kernel(const __grid_constant__ LinMaps maps, const __grid_constant__ LinearArgs args) {
   using L = LinSmem<BN, F32S>;
   constexpr uint32_t kCols = 2 * BN;  // two f32 accumulators (a power of two >= 128)
   extern __shared__ uint8_t smem_raw[];
@@ -164,7 +238,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tslot;
-  const int nkb = args.nkb_lo + args.nkb_hi;
+  const int nkb = args.nkb;
   // A dependent kernel may be scheduled now; it waits for this grid's results
   // before reading them (griddepcontrol.wait above), and its CTAs only take an
   // SM once one of these has left it.
@@ -181,6 +255,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       int g = 0;
       for (int t = blockIdx.x; t < args.tiles && !timed_out; t += gridDim.x) {
         const int m0 = (t / args.tiles_n) * kLinBM, n0 = (t % args.tiles_n) * BN;
+        int si = 0, sb0 = 0;  // current segment and its first K block
         for (int kb = 0; kb < nkb; ++kb, ++g) {
           const int s = g % L::kStages;
           if (g >= L::kStages &&
@@ -188,17 +263,14 @@ __global__ void __launch_bounds__(kLinThreads, 1)
             timed_out = true;
             break;
           }
+          while (kb - sb0 >= args.seg[si].nkb) sb0 += args.seg[si++].nkb;
+          const LinSeg& sg = args.seg[si];
+          const int kk = (kb - sb0) * kLinBK;
           uint8_t* sa = smem + s * L::kStage;
           uint8_t* sb = sa + L::kA;
           mbar_arrive_expect_tx(&full[s], L::kStage);
-          if (kb < args.nkb_lo) {
-            tma_load_2d(sa, &map_a_lo, &full[s], kb * kLinBK, m0);
-            tma_load_2d(sb, &map_w, &full[s], kb * kLinBK, n0);
-          } else {
-            const int kh = kb - args.nkb_lo;
-            tma_load_2d(sa, &map_a_hi, &full[s], kh * kLinBK, m0);
-            tma_load_2d(sb, &map_w, &full[s], args.k_lo + kh * kLinBK, n0);
-          }
+          tma_load_2d(sa, &maps.a[sg.a], &full[s], sg.a_k0 + kk, m0);
+          tma_load_2d(sb, &maps.w[sg.w], &full[s], sg.w_k0 + kk, n0);
         }
       }
     }
@@ -253,7 +325,23 @@ __global__ void __launch_bounds__(kLinThreads, 1)
                          (reinterpret_cast<uintptr_t>(args.y_f32) % 16) == 0;
     const bool bf_vec = args.y_bf16 != nullptr && (args.ldy_bf16 % 8) == 0 &&
                         (reinterpret_cast<uintptr_t>(args.y_bf16) % 16) == 0;
+    const bool planes_vec = args.y_planes != nullptr && (args.ldy_planes % 8) == 0 &&
+                            (args.splane_y % 8) == 0 &&
+                            (reinterpret_cast<uintptr_t>(args.y_planes) % 16) == 0;
     const bool tma_out = args.tma_f32 || args.tma_bf16;
+    // the outputs not written through TMA
+    LinOut direct;
+    direct.y_f32 = args.tma_f32 ? nullptr : args.y_f32;
+    direct.y_bf16 = args.tma_bf16 ? nullptr : args.y_bf16;
+    direct.y_planes = args.y_planes;
+    direct.ldy_f32 = args.ldy_f32;
+    direct.ldy_bf16 = args.ldy_bf16;
+    direct.ldy_planes = args.ldy_planes;
+    direct.splane_y = args.splane_y;
+    direct.M = args.M;
+    direct.N = args.N;
+    const bool any_direct =
+        direct.y_f32 != nullptr || direct.y_bf16 != nullptr || direct.y_planes != nullptr;
     int j = 0;
     for (int t = blockIdx.x; t < args.tiles; t += gridDim.x, ++j) {
       const int b = j & 1;
@@ -308,17 +396,12 @@ __global__ void __launch_bounds__(kLinThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (F32S && args.tma_f32) tma_store_2d(&map_y32, st32, n0 + c0, row0);
-            if (args.tma_bf16) tma_store_2d(&map_y16, st16, n0 + c0, row0);
+            if (F32S && args.tma_f32) tma_store_2d(&maps.y32, st32, n0 + c0, row0);
+            if (args.tma_bf16) tma_store_2d(&maps.y16, st16, n0 + c0, row0);
             bulk_commit();
           }
         }
-        if (!args.tma_f32 || !args.tma_bf16) {
-          LinearArgs direct = args;  // the outputs not written through TMA
-          if (args.tma_f32) direct.y_f32 = nullptr;
-          if (args.tma_bf16) direct.y_bf16 = nullptr;
-          store_chunk32(direct, row0 + lane, n0 + c0, v, f32_vec, bf_vec);
-        }
+        if (any_direct) store_chunk32(direct, row0 + lane, n0 + c0, v, f32_vec, bf_vec, planes_vec);
       }
       tc_fence_before_sync();
       __syncwarp();
@@ -360,9 +443,7 @@ cudaError_t encode_bf16_operand(CUtensorMap* map, const void* base, int64_t cols
 }
 
 template <int BN, int ACT, bool F32S>
-cudaError_t run_linear(const CUtensorMap& a_lo, const CUtensorMap& a_hi, const CUtensorMap& w,
-                       const CUtensorMap& y32, const CUtensorMap& y16, LinearArgs args, int sms,
-                       cudaStream_t stream) {
+cudaError_t run_linear(const LinMaps& maps, LinearArgs args, int sms, cudaStream_t stream) {
   auto* fn = &linear_bf16_kernel<BN, ACT, F32S>;
   constexpr int smem = LinSmem<BN, F32S>::kTotal;
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
@@ -386,31 +467,26 @@ cudaError_t run_linear(const CUtensorMap& a_lo, const CUtensorMap& a_hi, const C
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fn, a_lo, a_hi, w, y32, y16, args);
+  return cudaLaunchKernelEx(&cfg, fn, maps, args);
 }
 
 template <int BN, bool F32S>
-cudaError_t run_linear_act(int act, const CUtensorMap& a_lo, const CUtensorMap& a_hi,
-                           const CUtensorMap& w, const CUtensorMap& y32, const CUtensorMap& y16,
-                           const LinearArgs& args, int sms, cudaStream_t stream) {
+cudaError_t run_linear_act(int act, const LinMaps& maps, const LinearArgs& args, int sms,
+                           cudaStream_t stream) {
   switch (act) {
-    case DLRM_ACT_RELU:
-      return run_linear<BN, DLRM_ACT_RELU, F32S>(a_lo, a_hi, w, y32, y16, args, sms, stream);
-    case DLRM_ACT_SIGMOID:
-      return run_linear<BN, DLRM_ACT_SIGMOID, F32S>(a_lo, a_hi, w, y32, y16, args, sms, stream);
-    default:
-      return run_linear<BN, DLRM_ACT_NONE, F32S>(a_lo, a_hi, w, y32, y16, args, sms, stream);
+    case DLRM_ACT_RELU: return run_linear<BN, DLRM_ACT_RELU, F32S>(maps, args, sms, stream);
+    case DLRM_ACT_SIGMOID: return run_linear<BN, DLRM_ACT_SIGMOID, F32S>(maps, args, sms, stream);
+    default: return run_linear<BN, DLRM_ACT_NONE, F32S>(maps, args, sms, stream);
   }
 }
 
 // The instance with f32 output staging (and, at 256 columns, a 3-stage ring)
 // only when the f32 output goes out through TMA.
 template <int BN>
-cudaError_t run_linear_bn(int act, const CUtensorMap& a_lo, const CUtensorMap& a_hi,
-                          const CUtensorMap& w, const CUtensorMap& y32, const CUtensorMap& y16,
-                          const LinearArgs& args, int sms, cudaStream_t stream) {
-  return args.tma_f32 ? run_linear_act<BN, true>(act, a_lo, a_hi, w, y32, y16, args, sms, stream)
-                      : run_linear_act<BN, false>(act, a_lo, a_hi, w, y32, y16, args, sms, stream);
+cudaError_t run_linear_bn(int act, const LinMaps& maps, const LinearArgs& args, int sms,
+                          cudaStream_t stream) {
+  return args.tma_f32 ? run_linear_act<BN, true>(act, maps, args, sms, stream)
+                      : run_linear_act<BN, false>(act, maps, args, sms, stream);
 }
 
 // 2-D output map {N, M} with row pitch ld elements, box {32, 32}, written from a
@@ -450,6 +526,130 @@ int choose_bn(int64_t M, int64_t N, int sms) {
 
 bool is_aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+
+// One layer: the checks shared by both entry points are done; `parts` lists
+// the A parts (1 or 2) as (base, pitch, plane stride, k) with `a_planes`
+// planes each, W has `w_planes` planes. Builds the maps and the segment table
+// and launches.
+struct APart {
+  const uint16_t* base;
+  int64_t ld, splane, k;
+};
+
+int launch_layer(const APart* parts, int nparts, int a_planes, const uint16_t* w, int64_t ldw,
+                 int64_t splane_w, int w_planes, const float* bias, int64_t M, int64_t N,
+                 int act, float* y_f32, int64_t ldy_f32, uint16_t* y_bf16, int64_t ldy_bf16,
+                 uint16_t* y_planes, int64_t ldy_planes, int64_t splane_y, int32_t* status_dev,
+                 cudaStream_t stream) {
+  const int64_t K = parts[0].k + (nparts > 1 ? parts[1].k : 0);
+  const int sms = sm_count_current();
+  const int bn = choose_bn(M, N, sms);
+  LinMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  cudaError_t e = cudaSuccess;
+  for (int p = 0; p < nparts && e == cudaSuccess; ++p)
+    for (int i = 0; i < a_planes && e == cudaSuccess; ++i)
+      e = encode_bf16_operand(&maps.a[p * 3 + i], parts[p].base + i * parts[p].splane,
+                              parts[p].k, M, parts[p].ld, kLinBM);
+  for (int j = 0; j < w_planes && e == cudaSuccess; ++j)
+    e = encode_bf16_operand(&maps.w[j], w + j * splane_w, K, N, ldw, bn);
+  if (e != cudaSuccess) return cuda_fail(e);
+
+  LinearArgs args;
+  std::memset(&args, 0, sizeof(args));
+  args.bias = bias;
+  args.y_f32 = y_f32;
+  args.y_bf16 = y_bf16;
+  args.y_planes = y_planes;
+  args.ldy_f32 = ldy_f32;
+  args.ldy_bf16 = ldy_bf16;
+  args.ldy_planes = ldy_planes;
+  args.splane_y = splane_y;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.status = status_dev;
+  // Products summed: A plane i times W plane j for i + j < 3 (all three A
+  // planes against a single weight plane; against three weight planes the six
+  // products whose planes' leading bits lie within 2^-16 of the value's).
+  int w_off = 0;
+  for (int p = 0; p < nparts; ++p) {
+    const int nkb = static_cast<int>((parts[p].k + kLinBK - 1) / kLinBK);
+    for (int i = 0; i < a_planes; ++i)
+      for (int j = 0; j < w_planes; ++j) {
+        if (i + j >= 3) continue;
+        LinSeg& sg = args.seg[args.nseg++];
+        sg.a = p * 3 + i;
+        sg.w = j;
+        sg.a_k0 = 0;
+        sg.w_k0 = w_off;
+        sg.nkb = nkb;
+        args.nkb += nkb;
+      }
+    w_off += static_cast<int>(parts[p].k);
+  }
+  // Outputs whose rows are whole 16-byte units at 16-byte aligned addresses go
+  // out through TMA stores; the others are written directly.
+  args.tma_f32 = y_f32 != nullptr && ldy_f32 % 4 == 0 && is_aligned(y_f32, 16);
+  args.tma_bf16 = y_bf16 != nullptr && ldy_bf16 % 8 == 0 && is_aligned(y_bf16, 16);
+  if (args.tma_f32)
+    e = encode_output(&maps.y32, y_f32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, M, ldy_f32,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e == cudaSuccess && args.tma_bf16)
+    e = encode_output(&maps.y16, y_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, ldy_bf16,
+                      CU_TENSOR_MAP_SWIZZLE_64B);
+  if (e != cudaSuccess) return cuda_fail(e);
+  switch (bn) {
+    case 256: e = run_linear_bn<256>(act, maps, args, sms, stream); break;
+    case 128: e = run_linear_bn<128>(act, maps, args, sms, stream); break;
+    default: e = run_linear_bn<64>(act, maps, args, sms, stream); break;
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+  note_launch();
+  return DLRM_OK;
+}
+
+// Shape and alignment checks of one layer (see dlrm_mlp.h).
+int check_layer(const APart* parts, int nparts, const uint16_t* w, int64_t ldw,
+                const float* bias, int64_t M, int64_t N, int act, const float* y_f32,
+                int64_t ldy_f32, const uint16_t* y_bf16, int64_t ldy_bf16,
+                const uint16_t* y_planes, int64_t ldy_planes, const int32_t* status_dev) {
+  if (parts[0].base == nullptr || w == nullptr) return DLRM_ERR_NULL;
+  if (y_f32 == nullptr && y_bf16 == nullptr && y_planes == nullptr) return DLRM_ERR_NULL;
+  if (nparts > 1 && parts[1].base == nullptr) return DLRM_ERR_NULL;
+  if (act < DLRM_ACT_NONE || act > DLRM_ACT_SIGMOID) return DLRM_ERR_ARG;
+  if (M < 1 || N < 1 || parts[0].k < 1 || (nparts > 1 && parts[1].k < 1)) return DLRM_ERR_SHAPE;
+  const int64_t K = parts[0].k + (nparts > 1 ? parts[1].k : 0);
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return DLRM_ERR_SHAPE;
+  for (int p = 0; p < nparts; ++p)
+    if (parts[p].ld < parts[p].k) return DLRM_ERR_SHAPE;
+  if (ldw < K) return DLRM_ERR_SHAPE;
+  if ((y_f32 != nullptr && ldy_f32 < N) || (y_bf16 != nullptr && ldy_bf16 < N) ||
+      (y_planes != nullptr && ldy_planes < N))
+    return DLRM_ERR_SHAPE;
+  if ((N + 63) / 64 > 65535) return DLRM_ERR_SHAPE;
+  for (int p = 0; p < nparts; ++p)
+    if (parts[p].ld % 8 != 0 || !is_aligned(parts[p].base, 16)) return DLRM_ERR_ALIGN;
+  if (ldw % 8 != 0 || !is_aligned(w, 16)) return DLRM_ERR_ALIGN;
+  if (nparts > 1 && parts[0].k % 8 != 0) return DLRM_ERR_ALIGN;
+  if ((bias != nullptr && !is_aligned(bias, 4)) || (y_f32 != nullptr && !is_aligned(y_f32, 4)) ||
+      (y_bf16 != nullptr && !is_aligned(y_bf16, 2)) ||
+      (y_planes != nullptr && !is_aligned(y_planes, 2)) ||
+      (status_dev != nullptr && !is_aligned(status_dev, 4)))
+    return DLRM_ERR_ALIGN;
+  return DLRM_OK;
+}
+
+__global__ void split_bf16x3_kernel(const float* __restrict__ x, int64_t ldx, int64_t rows,
+                                    int64_t cols, uint16_t* __restrict__ y, int64_t ldy,
+                                    int64_t splane) {
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const float* xr = x + r * ldx;
+    uint16_t* yr = y + r * ldy;
+    for (int64_t c = threadIdx.x; c < cols; c += blockDim.x)
+      split_bf16x3(__ldg(xr + c), yr[c], yr[c + splane], yr[c + 2 * splane]);
+  }
+}
+
 }  // namespace
 }  // namespace dlrm
 
@@ -462,67 +662,59 @@ DLRM_API int dlrm_linear_bf16(const uint16_t* a_lo, int64_t lda_lo, int64_t k_lo
                               uint16_t* y_bf16, int64_t ldy_bf16, int32_t* status_dev,
                               dlrm_stream_t stream) {
   using namespace dlrm;
-  if (a_lo == nullptr || w == nullptr) return DLRM_ERR_NULL;
-  if (y_f32 == nullptr && y_bf16 == nullptr) return DLRM_ERR_NULL;
-  if (k_hi > 0 && a_hi == nullptr) return DLRM_ERR_NULL;
-  if (act < DLRM_ACT_NONE || act > DLRM_ACT_SIGMOID) return DLRM_ERR_ARG;
-  if (M < 1 || N < 1 || k_lo < 1 || k_hi < 0) return DLRM_ERR_SHAPE;
-  const int64_t K = k_lo + k_hi;
-  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return DLRM_ERR_SHAPE;
-  if (lda_lo < k_lo || (k_hi > 0 && lda_hi < k_hi) || ldw < K) return DLRM_ERR_SHAPE;
-  if ((y_f32 != nullptr && ldy_f32 < N) || (y_bf16 != nullptr && ldy_bf16 < N))
+  if (k_hi < 0) return DLRM_ERR_SHAPE;
+  const APart parts[2] = {{a_lo, lda_lo, 0, k_lo}, {a_hi, lda_hi, 0, k_hi}};
+  const int nparts = k_hi > 0 ? 2 : 1;
+  int rc = check_layer(parts, nparts, w, ldw, bias, M, N, act, y_f32, ldy_f32, y_bf16, ldy_bf16,
+                       nullptr, 0, status_dev);
+  if (rc != DLRM_OK) return rc;
+  return launch_layer(parts, nparts, 1, w, ldw, 0, 1, bias, M, N, act, y_f32, ldy_f32, y_bf16,
+                      ldy_bf16, nullptr, 0, 0, status_dev,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+DLRM_API int dlrm_linear_f32a(const uint16_t* a_lo, int64_t lda_lo, int64_t splane_lo,
+                              int64_t k_lo, const uint16_t* a_hi, int64_t lda_hi,
+                              int64_t splane_hi, int64_t k_hi, const uint16_t* w, int64_t ldw,
+                              int64_t splane_w, int w_planes, const float* bias, int64_t M,
+                              int64_t N, int act, float* y_f32, int64_t ldy_f32,
+                              uint16_t* y_planes, int64_t ldy_planes, int64_t splane_y,
+                              int32_t* status_dev, dlrm_stream_t stream) {
+  using namespace dlrm;
+  if (k_hi < 0) return DLRM_ERR_SHAPE;
+  if (w_planes != 1 && w_planes != 3) return DLRM_ERR_ARG;
+  const APart parts[2] = {{a_lo, lda_lo, splane_lo, k_lo}, {a_hi, lda_hi, splane_hi, k_hi}};
+  const int nparts = k_hi > 0 ? 2 : 1;
+  int rc = check_layer(parts, nparts, w, ldw, bias, M, N, act, y_f32, ldy_f32, nullptr, 0,
+                       y_planes, ldy_planes, status_dev);
+  if (rc != DLRM_OK) return rc;
+  // plane strides: whole 16-byte rows apart, and the planes must not overlap
+  for (int p = 0; p < nparts; ++p)
+    if (parts[p].splane % 8 != 0) return DLRM_ERR_ALIGN;
+  if (w_planes == 3 && splane_w % 8 != 0) return DLRM_ERR_ALIGN;
+  if (splane_lo < (M - 1) * lda_lo + k_lo || (k_hi > 0 && splane_hi < (M - 1) * lda_hi + k_hi) ||
+      (w_planes == 3 && splane_w < (N - 1) * ldw + k_lo + k_hi) ||
+      (y_planes != nullptr && splane_y < (M - 1) * ldy_planes + N))
     return DLRM_ERR_SHAPE;
-  if ((N + 63) / 64 > 65535) return DLRM_ERR_SHAPE;  // grid.y
-  if (lda_lo % 8 != 0 || (k_hi > 0 && lda_hi % 8 != 0) || ldw % 8 != 0) return DLRM_ERR_ALIGN;
-  if (k_hi > 0 && k_lo % 8 != 0) return DLRM_ERR_ALIGN;
-  if (!is_aligned(a_lo, 16) || (k_hi > 0 && !is_aligned(a_hi, 16)) || !is_aligned(w, 16))
-    return DLRM_ERR_ALIGN;
-  if ((bias != nullptr && !is_aligned(bias, 4)) || (y_f32 != nullptr && !is_aligned(y_f32, 4)) ||
-      (y_bf16 != nullptr && !is_aligned(y_bf16, 2)) ||
-      (status_dev != nullptr && !is_aligned(status_dev, 4)))
-    return DLRM_ERR_ALIGN;
+  return launch_layer(parts, nparts, 3, w, ldw, splane_w, w_planes, bias, M, N, act, y_f32,
+                      ldy_f32, nullptr, 0, y_planes, ldy_planes, splane_y, status_dev,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
 
-  const int sms = sm_count_current();
-  const int bn = choose_bn(M, N, sms);
-  CUtensorMap ma_lo, ma_hi, mw;
-  cudaError_t e = encode_bf16_operand(&ma_lo, a_lo, k_lo, M, lda_lo, kLinBM);
-  if (e == cudaSuccess && k_hi > 0) e = encode_bf16_operand(&ma_hi, a_hi, k_hi, M, lda_hi, kLinBM);
-  if (e == cudaSuccess) e = encode_bf16_operand(&mw, w, K, N, ldw, bn);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (k_hi == 0) ma_hi = ma_lo;  // never read
-
-  LinearArgs args;
-  args.bias = bias;
-  args.y_f32 = y_f32;
-  args.y_bf16 = y_bf16;
-  args.ldy_f32 = ldy_f32;
-  args.ldy_bf16 = ldy_bf16;
-  args.M = static_cast<int>(M);
-  args.N = static_cast<int>(N);
-  args.k_lo = static_cast<int>(k_lo);
-  args.nkb_lo = static_cast<int>((k_lo + kLinBK - 1) / kLinBK);
-  args.nkb_hi = static_cast<int>((k_hi + kLinBK - 1) / kLinBK);
-  args.status = status_dev;
-  // Outputs whose rows are whole 16-byte units at 16-byte aligned addresses go
-  // out through TMA stores; the others are written directly.
-  CUtensorMap my32, my16;
-  args.tma_f32 = y_f32 != nullptr && ldy_f32 % 4 == 0 && is_aligned(y_f32, 16);
-  args.tma_bf16 = y_bf16 != nullptr && ldy_bf16 % 8 == 0 && is_aligned(y_bf16, 16);
-  if (args.tma_f32)
-    e = encode_output(&my32, y_f32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, N, M, ldy_f32,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
-  if (e == cudaSuccess && args.tma_bf16)
-    e = encode_output(&my16, y_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, ldy_bf16,
-                      CU_TENSOR_MAP_SWIZZLE_64B);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (!args.tma_f32) my32 = mw;  // never read
-  if (!args.tma_bf16) my16 = mw;  // never read
-  auto* s = reinterpret_cast<cudaStream_t>(stream);
-  switch (bn) {
-    case 256: e = run_linear_bn<256>(act, ma_lo, ma_hi, mw, my32, my16, args, sms, s); break;
-    case 128: e = run_linear_bn<128>(act, ma_lo, ma_hi, mw, my32, my16, args, sms, s); break;
-    default: e = run_linear_bn<64>(act, ma_lo, ma_hi, mw, my32, my16, args, sms, s); break;
-  }
+DLRM_API int dlrm_split_f32_bf16x3(const float* x, int64_t ldx, int64_t rows, int64_t cols,
+                                   uint16_t* y, int64_t ldy, int64_t splane,
+                                   dlrm_stream_t stream) {
+  using namespace dlrm;
+  if (x == nullptr || y == nullptr) return DLRM_ERR_NULL;
+  if (rows < 1 || cols < 1 || ldx < cols || ldy < cols) return DLRM_ERR_SHAPE;
+  if (splane < (rows - 1) * ldy + cols) return DLRM_ERR_SHAPE;
+  if (!is_aligned(x, 4) || !is_aligned(y, 2)) return DLRM_ERR_ALIGN;
+  const int64_t blocks = std::min<int64_t>(rows, 148 * 32);
+  const int threads = cols >= 256 ? 256 : static_cast<int>(((cols + 31) / 32) * 32);
+  split_bf16x3_kernel<<<static_cast<unsigned>(blocks), threads, 0,
+                        reinterpret_cast<cudaStream_t>(stream)>>>(x, ldx, rows, cols, y, ldy,
+                                                                 splane);
+  const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   note_launch();
   return DLRM_OK;

@@ -65,6 +65,9 @@ SIGNATURES = {
     # include/dlrm_mlp.h
     "dlrm_linear_bf16": (_I, [_P, _I64, _I64, _P, _I64, _I64, _P, _I64, _P, _I64, _I64, _I, _P,
                               _I64, _P, _I64, _P, _P]),
+    "dlrm_linear_f32a": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I64, _I64, _P, _I64, _I64, _I,
+                              _P, _I64, _I64, _I, _P, _I64, _P, _I64, _I64, _P, _P]),
+    "dlrm_split_f32_bf16x3": (_I, [_P, _I64, _I64, _I64, _P, _I64, _I64, _P]),
     "dlrm_f32_to_bf16": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P]),
 }
 

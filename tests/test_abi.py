@@ -36,7 +36,7 @@ def test_header_declares_the_stage_entry_points():
     names = _declared()
     assert {"embbag_sum_multi", "interact_lower_tri", "dlrm_sparse_interact"} <= names
     assert {"dlrm_linear_bf16", "dlrm_f32_to_bf16"} <= names
-    assert len(names) == 19
+    assert len(names) == 21
 
 
 def test_library_exports_every_declared_symbol(ops):

@@ -162,9 +162,10 @@ def test_f32_to_bf16_matches_torch_rne():
 def _dlrm_case(seed, B, F, N, D, L, dense_in=13, bot=(64, 32), top=(64, 32)):
     g = torch.Generator(device=DEV)
     g.manual_seed(seed)
-    bottom = mlp.MLP(syn.make_mlp_layers(dense_in, list(bot) + [D], seed, DEV))
+    bottom = mlp.MLP(syn.make_mlp_layers(dense_in, list(bot) + [D], seed, DEV), mode="bf16")
     P = (F + 1) * F // 2
-    top_m = mlp.MLP(syn.make_mlp_layers(D + P, list(top) + [1], seed + 1, DEV, last="sigmoid"))
+    top_m = mlp.MLP(syn.make_mlp_layers(D + P, list(top) + [1], seed + 1, DEV, last="sigmoid"),
+                    mode="bf16")
     w = syn.Workload("t", B=B, F=F, N=N, D=D, L=L)
     weights = syn.make_weights(w, DEV)
     idx = torch.from_numpy(syn.make_indices(w)).to(DEV)
@@ -242,3 +243,180 @@ def test_linear_graph_capture_and_launch_count():
     torch.cuda.synchronize()
     assert torch.equal(y, ref)
     assert int(status.item()) == 0
+
+
+# ---------------------------------------------------------------------------
+# f32 activations (dlrm_linear_f32a): the pages' own arithmetic. Each
+# activation is three exact bf16 planes and every product is exact, so the
+# only error is the f32 accumulation of the 3K (bf16 weights) or 6K (f32
+# weights, whose dropped plane products are below 2^-20 |a w|) products.
+
+
+def _rand_f32(g, rows, cols, std=1.0):
+    return torch.empty((rows, cols), device=DEV).normal_(0, std, generator=g)
+
+
+def _f32a_tol(bound, out, K, act, w_planes):
+    slope = 0.25 if act == "sigmoid" else 1.0
+    n = (3 if w_planes == 1 else 6) * K + 2
+    rep = 0.0 if w_planes == 1 else 2.0 ** -20
+    return slope * (n * 2.0 ** -23 * 1.02 + rep) * bound + 8 * 2.0 ** -24 * np.abs(out) + 1e-30
+
+
+def _check_f32a(y32, a_lo, w, bias, act, a_hi=None, rows=None, w_planes=1, what=""):
+    """a_lo/a_hi: the f32 activations; w: bf16 (N, K) or f32 (N, K) weights."""
+    a = a_lo if rows is None else a_lo[rows]
+    h = None if a_hi is None else (a_hi if rows is None else a_hi[rows])
+    wn = _bits(w) if w.dtype == torch.bfloat16 else w.cpu().numpy()
+    out, pre, bound = oracle.linear_f32a(a.cpu().numpy(), wn,
+                                         None if bias is None else bias.cpu().numpy(),
+                                         ACT_CODE[act],
+                                         a_hi=None if h is None else h.cpu().numpy())
+    K = w.shape[1]
+    tol = _f32a_tol(bound, out, K, act, w_planes)
+    got = (y32 if rows is None else y32[rows]).double().cpu().numpy()
+    err = np.abs(got - out)
+    bad = err > tol
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside the bound; worst "
+                           f"err {err.max():.3e}, tol there {tol.flat[err.argmax()]:.3e}")
+    return err, bound
+
+
+def test_split_bf16x3_is_exact():
+    """The three planes are bf16 values that sum to the f32 value exactly,
+    p0 holds the value's top 8 significant bits and p1 the next 8."""
+    rng = np.random.default_rng(19)
+    bits = rng.integers(0, 2 ** 32, size=(41, 133), dtype=np.uint64).astype(np.uint32)
+    x = bits.view(np.float32).copy()
+    x[~np.isfinite(x)] = 1.0
+    x[np.abs(x) < 1e-30] = 0.5  # away from subnormal planes
+    x[0, :6] = [0.0, -0.0, 1.0, -3.0, 1.0 + 2 ** -23, -(1.0 + 2 ** -9 + 2 ** -17 + 2 ** -23)]
+    xt = torch.from_numpy(x).to(DEV)
+    p = mlp.split_bf16x3(xt)
+    torch.cuda.synchronize()
+    planes = [(_bits(p[i]).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+              for i in range(3)]
+    assert np.array_equal(planes[0] + planes[1] + planes[2], x.astype(np.float64))
+    assert np.array_equal(_bits(p[0]), (x.view(np.uint32) >> 16).astype(np.uint16))
+    r = x.astype(np.float64) - planes[0]
+    assert np.array_equal(planes[1], (r.astype(np.float32).view(np.uint32) & 0xffff0000)
+                          .view(np.float32).astype(np.float64))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 8), (5, 3, 16), (128, 64, 64), (200, 96, 72),
+                                   (300, 130, 200), (129, 257, 136), (1000, 512, 592),
+                                   (64, 40, 13)])
+@pytest.mark.parametrize("wdt", ["bf16", "f32"])
+def test_linear_f32a_shapes(M, N, K, wdt):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(M + N + K)
+    a = _rand_f32(g, M, K)
+    b = torch.empty(N, device=DEV).normal_(0, 0.5, generator=g)
+    if wdt == "bf16":
+        w = _rand_bf16(g, N, K, K ** -0.5)
+        wk = w
+    else:
+        w = _rand_f32(g, N, K, K ** -0.5)
+        wk = mlp.split_bf16x3(w)
+    y32, planes = mlp.linear_f32a(mlp.split_bf16x3(a), wk, b, "none", planes=True)
+    torch.cuda.synchronize()
+    err, bound = _check_f32a(y32, a, w, b, "none", w_planes=1 if wdt == "bf16" else 3,
+                             what=f"M={M} N={N} K={K} {wdt} weights")
+    # the planes written for the next layer are the exact split of the f32 result
+    p = [(_bits(planes[i]).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+         for i in range(3)]
+    assert np.array_equal(p[0] + p[1] + p[2], y32.double().cpu().numpy())
+    if wdt == "bf16" and K >= 64:
+        # the f32 activations are honoured: the bf16-activation layer is far off
+        y16, _ = mlp.linear_bf16(mlp.to_bf16(a), w, b, "none")
+        torch.cuda.synchronize()
+        e16 = np.abs(y16.double().cpu().numpy() - y32.double().cpu().numpy())
+        assert e16.max() > 100 * max(err.max(), 1e-30)
+
+
+@pytest.mark.parametrize("act", ["none", "relu", "sigmoid"])
+def test_linear_f32a_activations(act):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(77)
+    a = _rand_f32(g, 333, 96)
+    w = _rand_bf16(g, 200, 96, 96 ** -0.5)
+    b = torch.empty(200, device=DEV).normal_(0, 0.5, generator=g)
+    y32, _ = mlp.linear_f32a(mlp.split_bf16x3(a), w, b, act)
+    torch.cuda.synchronize()
+    _check_f32a(y32, a, w, b, act, what=f"f32a {act}")
+
+
+@pytest.mark.parametrize("k_lo,k_hi", [(64, 528), (128, 351), (24, 40), (8, 8)])
+def test_linear_f32a_split_a(k_lo, k_hi):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(k_lo * 7 + k_hi)
+    M, N = 260, 192
+    a_lo = _rand_f32(g, M, k_lo)
+    a_hi = _rand_f32(g, M, k_hi)
+    w = _rand_bf16(g, N, k_lo + k_hi, (k_lo + k_hi) ** -0.5)
+    b = torch.empty(N, device=DEV).normal_(0, 0.5, generator=g)
+    y32, _ = mlp.linear_f32a(mlp.split_bf16x3(a_lo), w, b, "relu",
+                             a_hi=mlp.split_bf16x3(a_hi))
+    torch.cuda.synchronize()
+    _check_f32a(y32, a_lo, w, b, "relu", a_hi=a_hi, what=f"f32a split {k_lo}+{k_hi}")
+
+
+@pytest.mark.parametrize("M,N,K", [(20000, 512, 592), (10000, 256, 192)])
+def test_linear_f32a_wide_tiles_sampled(M, N, K):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(M + K)
+    a = _rand_f32(g, M, K)
+    w = _rand_bf16(g, N, K, K ** -0.5)
+    b = torch.empty(N, device=DEV).normal_(0, 0.5, generator=g)
+    y32, _ = mlp.linear_f32a(mlp.split_bf16x3(a), w, b, "relu")
+    torch.cuda.synchronize()
+    rows = torch.from_numpy(np.random.default_rng(M).choice(M, 96, replace=False)).to(DEV)
+    _check_f32a(y32, a, w, b, "relu", rows=rows, what=f"f32a M={M} N={N} K={K}")
+
+
+def test_dlrm_forward_f32_chain():
+    """The f32-activation forward, each stage against the oracle on the
+    kernel's own f32 inputs: bottom layers, sparse stage, split top layer 0,
+    CTR head."""
+    B, F, N, D, L = 256, 8, 1000, 64, 4
+    g = torch.Generator(device=DEV)
+    g.manual_seed(33)
+    seed = 41
+    bottom = mlp.MLP(syn.make_mlp_layers(13, [64, 32, D], seed, DEV), mode="f32")
+    P = (F + 1) * F // 2
+    top = mlp.MLP(syn.make_mlp_layers(D + P, [64, 32, 1], seed + 1, DEV, last="sigmoid"),
+                  mode="f32")
+    w = syn.Workload("t", B=B, F=F, N=N, D=D, L=L)
+    weights = syn.make_weights(w, DEV)
+    idx = torch.from_numpy(syn.make_indices(w)).to(DEV)
+    off = torch.from_numpy(syn.make_offsets(w)).to(DEV)
+    x = _rand_f32(g, B, 13).abs()
+    ctr, t = mlp.dlrm_forward(bottom, top, x, weights, idx, off, L, keep=True)
+    torch.cuda.synchronize()
+    assert ctr.shape == (B, 1) and ((ctr > 0) & (ctr < 1)).all()
+
+    def f32_of(planes):
+        return sum((_bits(planes[i]).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+                   for i in range(3))
+
+    # the dense features enter as their exact planes
+    a_in = torch.from_numpy(f32_of(mlp.split_bf16x3(x)).astype(np.float32)).to(DEV)
+    assert torch.equal(a_in, x)
+    # the dense vector handed to the top MLP is exactly the f32 one the interaction used
+    assert np.array_equal(f32_of(t["dense16"]), t["dense32"].double().cpu().numpy())
+    wn = [w_.cpu().numpy() for w_ in weights]
+    pooled, inter, bound = oracle.sparse_interact(wn, idx.cpu().numpy(), off.cpu().numpy(),
+                                                  t["dense32"].cpu().numpy(), B, L,
+                                                  with_bound=True)
+    assert np.array_equal(t["pooled"].cpu().numpy().view(np.uint32), pooled.view(np.uint32))
+    assert np.all(np.abs(t["z"].cpu().numpy().astype(np.float64) - inter) <= 1e-5 * bound + 1e-30)
+    assert np.array_equal(f32_of(t["z16"]), t["z"].double().cpu().numpy())
+    (a0, h0) = t["top_inputs"][0]
+    w0, b0, act0 = top.layers[0]
+    r32, _ = mlp.linear_f32a(a0, w0, b0, act0, a_hi=h0)
+    torch.cuda.synchronize()
+    _check_f32a(r32, t["dense32"], w0, b0, act0, a_hi=t["z"], what="f32 top layer 0")
+    (a_last, _) = t["top_inputs"][-1]
+    wl, bl, actl = top.layers[-1]
+    a_last32 = torch.from_numpy(f32_of(a_last).astype(np.float32)).to(DEV)
+    _check_f32a(ctr, a_last32, wl, bl, actl, what="f32 CTR head")
