@@ -64,6 +64,11 @@ def parse_args(argv=None):
                     help="time the fused stage on the 11 x 5 batch x table-count sweep instead")
     ap.add_argument("--mlp", action="store_true",
                     help="time the DLRMv1 MLP layers (tcgen05) and the full forward instead")
+    ap.add_argument("--kernel", choices=["fused", "gather", "interact"], default="fused",
+                    help="time the fused stage (default), the gather alone (embbag_sum_multi / "
+                         "embbag_pool_multi) or the interaction alone (interact_lower_tri)")
+    ap.add_argument("--path", choices=["auto", "ldg"], default="auto",
+                    help="gather path of the library (auto = the measured fastest)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU time budget of the oracle baseline sample")
     args = ap.parse_args(argv)
@@ -275,19 +280,74 @@ def time_oracle(orc, tables, idx, off, dense, S, L, concat, budget_s, min_calls=
     return times
 
 
+def host_cpu():
+    """Host core count and CPU model (``nproc`` / ``lscpu``)."""
+    import subprocess
+
+    cores = os.cpu_count() or 1
+    model = ""
+    try:
+        cores = int(subprocess.run(["nproc"], capture_output=True, text=True,
+                                   check=True).stdout.strip())
+        for line in subprocess.run(["lscpu"], capture_output=True, text=True,
+                                   check=True).stdout.splitlines():
+            if line.startswith("Model name:"):
+                model = line.split(":", 1)[1].strip()
+    except (OSError, subprocess.SubprocessError, ValueError):
+        pass
+    return cores, model
+
+
 def cpu_baseline(w: syn.Workload, source, budget_s: float):
+    """The oracle timed on one core and on all host cores.
+
+    All cores: the whole batch is cut into one contiguous chunk of samples per
+    core, and one thread per core calls the oracle's C code on its chunk
+    (ctypes releases the interpreter lock for the call), so every core runs
+    the same per-sample loops in parallel over samples."""
+    import concurrent.futures as cf
+
     import oracle  # test infrastructure: this leg times the oracle as it stands
 
+    orc = oracle.default()
     S = min(w.B, 512)
     tables, idx, off, dense = oracle_sample(w, S, source=source)
-    orc = oracle.default()
     orc.sparse_interact(tables, idx, off, dense, S, w.L, concat_dense=w.concat_dense)  # warm
-    times = time_oracle(orc, tables, idx, off, dense, S, w.L, w.concat_dense, budget_s)
-    t = statistics.median(times)
-    return {"value": S * w.F * w.L / t, "unit": "lookups/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {S} of {w.B} samples of {w.name} (all {w.F} tables, L={w.L}), "
-                      f"full-size host tables holding the referenced rows; median of "
-                      f"{len(times)} single-thread oracle calls"}
+    times = time_oracle(orc, tables, idx, off, dense, S, w.L, w.concat_dense, budget_s / 2)
+    single = S * w.F * w.L / statistics.median(times)
+
+    cores, model = host_cpu()
+    SB = w.B
+    tables_b, idx_b, _, dense_b = oracle_sample(w, SB, source=source)
+    n = max(1, min(cores, SB))
+    bounds = [(SB * c // n, SB * (c + 1) // n) for c in range(n)]
+    chunks = []
+    for s0, s1 in bounds:
+        sub = w.scaled(B=s1 - s0)
+        chunks.append((np.ascontiguousarray(idx_b[:, s0 * w.L:s1 * w.L]), syn.make_offsets(sub),
+                       np.ascontiguousarray(dense_b[s0:s1]), s1 - s0))
+
+    def one(ch):
+        ci, co, cd, cb = ch
+        orc.sparse_interact(tables_b, ci, co, cd, cb, w.L, concat_dense=w.concat_dense)
+
+    with cf.ThreadPoolExecutor(max_workers=n) as ex:
+        list(ex.map(one, chunks))  # warm
+        par = []
+        t_end = time.perf_counter() + budget_s / 2
+        while len(par) < 3 or time.perf_counter() < t_end:
+            t0 = time.perf_counter()
+            list(ex.map(one, chunks))
+            par.append(time.perf_counter() - t0)
+    allc = SB * w.F * w.L / statistics.median(par)
+    return {"value": allc, "unit": "lookups/s", "cores": n, "kind": "oracle",
+            "cpu": model, "nproc": cores,
+            "sample": f"all {SB} samples of {w.name} (all {w.F} tables, L={w.L}) cut into {n} "
+                      f"chunks, one thread per core calling the oracle on its chunk; full-size "
+                      f"host tables holding the referenced rows; median of {len(par)} passes",
+            "single_core": {"value": single, "unit": "lookups/s", "cores": 1,
+                            "sample": f"first {S} samples, median of {len(times)} "
+                                      f"single-thread oracle calls"}}
 
 
 def run_reference(args, w: syn.Workload):
@@ -361,6 +421,7 @@ def run_ours(args, w: syn.Workload):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     from dlrm_embedding_bag_b200 import ops
 
+    ops.set_gather_path(args.path)
     # inputs resident in HBM before timing: tables, this replica's batch, outputs
     weights = syn.make_weights(w, dev)
     if args.tables == "bf16":
@@ -379,7 +440,21 @@ def run_ours(args, w: syn.Workload):
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
 
-    if general:
+    if args.kernel == "gather":
+        def call(_stream):
+            if general:
+                ops.embbag_pool_multi(weights, idx, off, mode=args.pool, per_sample_weights=psw,
+                                      out=pooled)
+            else:
+                ops.embbag_sum_multi(weights, idx, off, w.L, out=pooled)
+    elif args.kernel == "interact":
+        # the pooled vectors the interaction reads, made once outside the timing
+        ops.embbag_sum_multi(weights, idx, off, w.L, out=pooled)
+        inter = torch.empty((w.B, w.P), dtype=torch.float32, device=dev)
+
+        def call(_stream):
+            ops.interact_lower_tri(dense, pooled, out=inter)
+    elif general:
         call = ops.PoolInteractCall(weights, idx, off, dense, mode=args.pool,
                                     per_sample_weights=psw, concat_dense=w.concat_dense,
                                     pooled_out=pooled, inter_out=inter)
@@ -433,6 +508,53 @@ def run_ours(args, w: syn.Workload):
     value = lookups / (total_ms / 1e3)
     ms_step = total_ms / args.steps
 
+    extras = {}
+    if world == 1 and args.kernel == "fused" and not general:
+        # warm-L2 timing, the pages' harness protocol: 5 rounds of 20 back-to-back
+        # steps (no flush between them), median of the round medians
+        rounds = []
+        for _ in range(5):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(21)]
+            torch.cuda.synchronize()
+            ev[0].record()
+            for i in range(20):
+                step()
+                ev[i + 1].record()
+            torch.cuda.synchronize()
+            rounds.append(statistics.median(ev[i].elapsed_time(ev[i + 1]) for i in range(20)))
+        warm_ms = statistics.median(rounds)
+        extras["warm_l2"] = {"ms_per_step": warm_ms, "value": w.B * w.F * w.L / (warm_ms / 1e3),
+                             "unit": "lookups/s",
+                             "protocol": "5 rounds x 20 steps without L2 flush, median of round "
+                                         "medians"}
+        if w.dist == "zipf":
+            # the same shapes with uniform indices: every row from HBM, the pure
+            # bandwidth check of the gather (tables shared with the run above)
+            wu = w.scaled(name=w.name.replace("zipf" + str(w.alpha), "uniform"),
+                          dist="uniform", alpha=0.0)
+            idx_u = torch.from_numpy(syn.make_indices(wu, replica=rank)).to(dev)
+            call_u = ops.SparseInteractCall(weights, idx_u, off, dense, w.L,
+                                            concat_dense=w.concat_dense, pooled_out=pooled,
+                                            inter_out=inter)
+            for _ in range(args.warmup):
+                flush.fill_(1)
+                call_u(stream)
+            ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+            ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+            for i in range(args.steps):
+                flush.fill_(i & 0xFF)
+                ev_s[i].record()
+                call_u(stream)
+                ev_e[i].record()
+            torch.cuda.synchronize()
+            u_ms = sum(a.elapsed_time(b) for a, b in zip(ev_s, ev_e)) / args.steps
+            extras["hbm_check"] = {"workload": wu.name, "ms_per_step": u_ms,
+                                   "value": w.B * w.F * w.L / (u_ms / 1e3),
+                                   "unit": "lookups/s",
+                                   "achieved_gbs": algorithmic_bytes(wu) / (u_ms / 1e3) / 1e9,
+                                   "algorithmic_bytes_per_launch": algorithmic_bytes(wu)}
+            del idx_u, call_u
+
     # e2e through the host-buffer entry point: every step copies its batch's
     # indices, offsets and dense rows in from pinned host memory and its
     # interaction rows back out. Steps cycle over E2E_BATCHES distinct batches
@@ -440,7 +562,7 @@ def run_ours(args, w: syn.Workload):
     # copies overlap other batches' kernels and copies; the region is timed
     # with events.
     e2e = None
-    if not args.no_e2e and not general:
+    if not args.no_e2e and not general and args.kernel == "fused":
         pipe = ops.HostPipeline(weights, w.B, w.L, concat_dense=w.concat_dense, want_pooled=True,
                                 depth=args.e2e_depth)
         batches = []
@@ -471,9 +593,52 @@ def run_ours(args, w: syn.Workload):
         t1.record(cur)
         barrier()
         e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+
+        # the same with the batch in three separate page-locked buffers (a
+        # caller that does not pack): three host-to-device copies per step
+        loose = []
+        for j in range(E2E_BATCHES):
+            ij, oj, dj = batches[j]
+            loose.append((ij.clone().pin_memory(), oj.clone().pin_memory(),
+                          dj.clone().pin_memory()))
+        for i in range(args.warmup):
+            pipe.submit(*loose[i % E2E_BATCHES], outs[i % args.e2e_depth])
+        pipe.drain()
+        barrier()
+        u0 = torch.cuda.Event(enable_timing=True)
+        u1 = torch.cuda.Event(enable_timing=True)
+        u0.record(cur)
+        for _, st, _ in pipe.slots:
+            st.wait_event(u0)
+        for i in range(args.steps):
+            pipe.submit(*loose[i % E2E_BATCHES], outs[i % args.e2e_depth])
+        for _, st, _ in pipe.slots:
+            ev = torch.cuda.Event()
+            ev.record(st)
+            cur.wait_event(ev)
+        u1.record(cur)
+        barrier()
+        loose_ms = max_over_ranks(u0.elapsed_time(u1), world, dev)
+        # what packing one batch into a reused page-locked block costs on the
+        # host (outside the timed region above; batch 0 is rewritten with its
+        # own values)
+        pipe.drain()
+        idx_t, off_t, dense_t = (torch.from_numpy(idx_np.reshape(-1)), torch.from_numpy(off_np),
+                                 dense.cpu())
+        bi, bo, bd = batches[0]
+        p0 = time.perf_counter()
+        for _ in range(5):
+            bi.copy_(idx_t)
+            bo.copy_(off_t)
+            bd.copy_(dense_t)
+        pack_ms = (time.perf_counter() - p0) / 5 * 1e3
         e2e = {"value": lookups / (e2e_ms / 1e3), "unit": "lookups/s",
                "h2d_bytes_per_step": pipe.h2d_bytes(), "d2h_bytes_per_step": pipe.d2h_bytes(),
                "ms_per_step": e2e_ms / args.steps,
+               "unpacked": {"value": lookups / (loose_ms / 1e3), "ms_per_step": loose_ms / args.steps,
+                            "note": "indices, offsets and dense in three separate pinned "
+                                    "buffers: three host-to-device copies per step"},
+               "host_pack_ms_per_batch": pack_ms,
                "path": f"dlrm_sparse_interact_host via ops.HostPipeline ({args.e2e_depth} streams): one "
                        f"pinned [indices|offsets|dense] block in, interaction rows out, {E2E_BATCHES} distinct "
                        f"batches in rotation; pooled written to device staging"}
@@ -486,6 +651,15 @@ def run_ours(args, w: syn.Workload):
             peak, peak_src = FALLBACK_HBM_GBS, "fallback"
         per_launch = algorithmic_bytes(w, esz=2 if args.tables == "bf16" else 4,
                                        weighted=args.weighted)
+        kernel_name = "fused_kernel (dlrm_sparse_interact)"
+        if args.kernel == "gather":
+            per_launch = algorithmic_bytes(w, esz=2 if args.tables == "bf16" else 4,
+                                           weighted=args.weighted) - 4 * w.B * w.D \
+                - 4 * w.B * ((w.D + w.P) if w.concat_dense else w.P)
+            kernel_name = "gather (embbag_sum_multi)"
+        elif args.kernel == "interact":
+            per_launch = 4 * w.B * w.D + 4 * w.B * w.F * w.D + 4 * w.B * w.P
+            kernel_name = "interact_kernel (interact_lower_tri)"
         achieved = per_launch / (ms_step / 1e3) / 1e9
         rows_gbs = (w.B * w.F * w.L * w.D * (2 if args.tables == "bf16" else 4)
                     / (ms_step / 1e3) / 1e9)
@@ -497,21 +671,37 @@ def run_ours(args, w: syn.Workload):
             "data": "synthetic", "config": workload_config(w, world, args),
             "samples_per_s": world * args.steps * w.B / (total_ms / 1e3),
             "gather_row_gbs": rows_gbs,
-            "roofline": {"bound": "hbm", "kernel": "fused_kernel (dlrm_sparse_interact)",
+            "roofline": {"bound": "hbm", "kernel": kernel_name,
                          "achieved": achieved, "peak": peak, "peak_source": peak_src,
                          "unit": "GB/s", "frac": achieved / peak,
                          "algorithmic_bytes_per_launch": per_launch,
                          "traffic": recorded_traffic(w.name)},
+            "gather_path": ops.last_gather_path(),
             "clocks": clocks, "remeasured": remeasured,
             "gpu_launches": launches,
             "region_wall_ms": 1e3 * wall,
             "step_ms_p50": statistics.median(per), "step_ms_min": min(per),
             "e2e": e2e,
         }
+        line.update(extras)
+        if "hbm_check" in line:
+            line["hbm_check"]["peak"] = peak
+            line["hbm_check"]["frac"] = line["hbm_check"]["achieved_gbs"] / peak
         if general:
             line["e2e"] = None
             line["e2e_note"] = "end-to-end host path covers the fixed-stride f32 sum stage only"
-        if world == 1 and not args.no_cpu_baseline and not general:
+        if args.kernel != "fused":
+            line["metric"] = (METRIC.replace("fused EmbeddingBag-sum + lower-triangle "
+                                             "interaction", "EmbeddingBag gather alone")
+                              if args.kernel == "gather"
+                              else "interaction samples/s (lower-triangle dots alone)")
+            if args.kernel == "interact":
+                line["value"] = line["samples_per_s"]
+                line["unit"] = "samples/s"
+            line["roofline"]["traffic"] = None
+            line["e2e"] = None
+            line["e2e_note"] = "end-to-end host path covers the fused stage only"
+        if world == 1 and not args.no_cpu_baseline and not general and args.kernel == "fused":
             line["cpu_baseline"] = cpu_baseline(w, weights, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -113,20 +113,7 @@ int clear_status(int32_t* status_dev, cudaStream_t stream) {
   return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
 }
 
-// The TMA path needs whole 16-byte row chunks of 64..512 bytes, 16-byte
-// aligned tables, tensor maps for every table and at least one row per table.
-bool tma_eligible(const Prepared& pr, const int64_t* rows, int F, int D) {
-  const int row_bytes = D * pr.elem_size;
-  if (row_bytes % 16 != 0 || row_bytes < 64 || row_bytes > 512) return false;
-  if (!pr.tables_aligned16 || F > dlrm::kTmaMaxTables) return false;
-  if (rows != nullptr)
-    for (int k = 0; k < F; ++k)
-      if (rows[k] < 1) return false;
-  return true;
-}
-
-dlrm::GatherPlan make_plan(const Prepared& pr, const int64_t* rows, int B, int F, int D,
-                           int loader, bool tma_ok) {
+dlrm::GatherPlan make_plan(const Prepared& pr, int B, int F, int D, int loader) {
   dlrm::GatherPlan g;
   g.tp = &pr.tp;
   g.bp = pr.bp;
@@ -136,8 +123,6 @@ dlrm::GatherPlan make_plan(const Prepared& pr, const int64_t* rows, int B, int F
   g.pool = pr.pool;
   g.loader = loader;
   g.esz = pr.elem_size;
-  g.tma_ok = tma_ok;
-  g.rows = rows;
   return g;
 }
 
@@ -152,8 +137,7 @@ int pool_impl(const void* const* weights, int dtype, const int64_t* rows, const 
   if (!aligned(out, 4)) return DLRM_ERR_ALIGN;
   const bool out16 = aligned(out, 16);
   const int loader = pick_loader(dtype, D, pr.tables_aligned16 && out16);
-  const dlrm::GatherPlan g =
-      make_plan(pr, rows, B, F, D, loader, out16 && tma_eligible(pr, rows, F, D));
+  const dlrm::GatherPlan g = make_plan(pr, B, F, D, loader);
   if ((rc = clear_status(status_dev, stream)) != DLRM_OK) return rc;
   return launch_status(dlrm::launch_embbag(g, out, stream));
 }
@@ -176,8 +160,7 @@ int fused_impl(const void* const* weights, int dtype, const int64_t* rows,
   if (dlrm::interact_smem_per_sample(F, D) > limit) return DLRM_ERR_SHAPE;
   const bool pooled16 = pooled_out == nullptr || aligned(pooled_out, 16);
   const int loader = pick_loader(dtype, D, pr.tables_aligned16 && pooled16);
-  const dlrm::GatherPlan g =
-      make_plan(pr, rows, B, F, D, loader, pooled16 && tma_eligible(pr, rows, F, D));
+  const dlrm::GatherPlan g = make_plan(pr, B, F, D, loader);
   if ((rc = clear_status(status_dev, stream)) != DLRM_OK) return rc;
   return launch_status(dlrm::launch_fused(g, dense, pooled_out, inter_out, concat_dense ? 1 : 0,
                                           limit, stream));
@@ -355,9 +338,7 @@ int dlrm_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_t* j_out,
 }
 
 int dlrm_set_gather_path(int path) {
-  if (path != DLRM_PATH_AUTO && path != DLRM_PATH_LDG && path != DLRM_PATH_TMA &&
-      path != DLRM_PATH_PIPE)
-    return DLRM_ERR_ARG;
+  if (path != DLRM_PATH_AUTO && path != DLRM_PATH_LDG) return DLRM_ERR_ARG;
   const int prev = dlrm::gather_path();
   dlrm::set_gather_path(path);
   return prev;

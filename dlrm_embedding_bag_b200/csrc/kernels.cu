@@ -10,8 +10,7 @@
 
 #include "interact_common.cuh"
 #include "launch.h"
-#include "pipe_kernels.cuh"
-#include "tma_kernels.cuh"
+#include "tma_common.cuh"
 
 namespace dlrm {
 
@@ -224,7 +223,7 @@ static cudaError_t counted(cudaError_t e) {
 }
 
 // --------------------------------------------------------------------------
-// Path choice and the TMA path's tensor maps.
+// Path choice and the tensor-map encoder.
 
 static std::atomic<int> g_path{DLRM_PATH_AUTO};
 static thread_local int t_last_path = 0;
@@ -246,33 +245,6 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// One map per table: a 2-D tensor {D, rows} with row pitch D*esz, box {D, 1},
-// out-of-range rows read as zeros.
-static cudaError_t make_tma_params(const GatherPlan& g, TmaParams* tp) {
-  const EncodeTiledFn enc = encode_tiled();
-  if (enc == nullptr) return cudaErrorNotSupported;
-  const int row_bytes = g.D * g.esz;
-  const CUtensorMapL2promotion promo = row_bytes >= 256   ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
-                                       : row_bytes >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
-                                                          : CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
-  for (int k = 0; k < g.F; ++k) {
-    const int64_t rows = g.rows ? g.rows[k] : INT32_MAX;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(g.D), static_cast<cuuint64_t>(rows)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(g.D), 1};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r =
-        enc(&tp->map[k], g.esz == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-            2, const_cast<void*>(g.tp->w[k]), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, promo,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    tp->rows[k] = g.tp->rows[k];
-  }
-  return cudaSuccess;
-}
-
 static int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -281,49 +253,10 @@ static int sm_count() {
 }
 
 
-// DLRM_PATH_AUTO takes the per-block register-load kernels: on B200 they are
-// faster than the TMA path on the measured workloads (L1 serves the hot rows
-// of skewed index streams, which TMA loads bypass) and than the pipelined
-// path (whose fused kernel has fewer warps to hide latency with).
+// One path serves every call: the per-block register-load kernels
+// (DLRM_PATH_AUTO = DLRM_PATH_LDG).
 cudaError_t launch_embbag(const GatherPlan& g, float* out, cudaStream_t stream) {
-  const int path = gather_path();
-  if (g.tma_ok && path == DLRM_PATH_TMA) {
-    t_last_path = DLRM_PATH_TMA;
-    TmaParams tp;
-    cudaError_t e = make_tma_params(g, &tp);
-    if (e != cudaSuccess) return e;
-    TmaLaunch a{};
-    a.tp = &tp;
-    a.bp = g.bp;
-    a.B = g.B;
-    a.F = g.F;
-    a.D = g.D;
-    a.G = tma_unit_lanes(g.D * g.esz);
-    a.cpl = tma_chunks_per_lane(g.D * g.esz);
-    a.pool = g.pool;
-    a.out = out;
-    a.sms = sm_count();
-    a.stream = stream;
-    return counted(g.esz == 4 ? launch_tma_gather_f32(a) : launch_tma_gather_bf16(a));
-  }
   const GatherShape sh = choose_gather_shape(g.D, g.loader);
-  const bool pipe_ok = (g.loader == kLdF32x4 || g.loader == kLdBF16x8) && sh.ncolwin == 1;
-  if (pipe_ok && path == DLRM_PATH_PIPE) {
-    t_last_path = DLRM_PATH_PIPE;
-    PipeLaunch a{};
-    a.tp = g.tp;
-    a.bp = g.bp;
-    a.B = g.B;
-    a.F = g.F;
-    a.D = g.D;
-    a.G = sh.G;
-    a.cpl = sh.cpl;
-    a.pool = g.pool;
-    a.out = out;
-    a.sms = sm_count();
-    a.stream = stream;
-    return counted(g.esz == 4 ? launch_pipe_gather_f32(a) : launch_pipe_gather_bf16(a));
-  }
   t_last_path = DLRM_PATH_LDG;
   GatherLaunch a{g.tp, g.bp, g.B, g.F, g.D, out, g.pool, sh, stream};
   switch (g.loader) {
@@ -338,77 +271,10 @@ cudaError_t launch_embbag(const GatherPlan& g, float* out, cudaStream_t stream) 
 cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_out,
                          float* inter_out, int concat_dense, int64_t smem_limit,
                          cudaStream_t stream) {
-  const int path = gather_path();
-  const FeatLayout Lf = FeatLayout::make(g.F, g.D);
-  bool tma_ok = g.tma_ok && (reinterpret_cast<uintptr_t>(dense) % 16 == 0);
-  TmaLaunch t{};
-  if (tma_ok) {
-    t.G = tma_unit_lanes(g.D * g.esz);
-    t.cpl = tma_chunks_per_lane(g.D * g.esz);
-    const int units = kTmaGatherWarps * (32 / t.G);
-    // about two bags per unit per tile; the dot warps take (S * nT) << lq tasks
-    t.S = std::max(1, std::min(16, (2 * units + g.F - 1) / g.F));
-    t.S = std::min(t.S, g.B);
-    const int64_t per = Lf.floats_per_sample() * 4;
-    while (t.S > 1 && TmaSmem::make(t.G, g.D * g.esz, 2 * t.S * per).total > smem_limit) --t.S;
-    tma_ok = TmaSmem::make(t.G, g.D * g.esz, 2 * t.S * per).total <= smem_limit;
-    const int qmax = std::max(1, kTmaDotWarps * 32 / (t.S * Lf.nT));
-    t.lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), 4});
-  }
-  if (tma_ok && path == DLRM_PATH_TMA) {
-    t_last_path = DLRM_PATH_TMA;
-    TmaParams tp;
-    cudaError_t e = make_tma_params(g, &tp);
-    if (e != cudaSuccess) return e;
-    t.tp = &tp;
-    t.bp = g.bp;
-    t.B = g.B;
-    t.F = g.F;
-    t.D = g.D;
-    t.pool = g.pool;
-    t.dense = dense;
-    t.pooled_out = pooled_out;
-    t.inter_out = inter_out;
-    t.concat_dense = concat_dense;
-    t.smem_limit = smem_limit;
-    t.sms = sm_count();
-    t.stream = stream;
-    return counted(g.esz == 4 ? launch_tma_fused_f32(t) : launch_tma_fused_bf16(t));
-  }
-  const GatherShape sh = choose_gather_shape(g.D, g.loader);
-  const bool pipe_ok = (g.loader == kLdF32x4 || g.loader == kLdBF16x8) && sh.ncolwin == 1;
-  if (pipe_ok && path == DLRM_PATH_PIPE) {
-    PipeLaunch a{};
-    const int units = kPipeGatherWarps * 32 / sh.G;
-    // about two bags per unit per tile, two tiles of features in shared memory
-    a.S = std::max(1, std::min({16, (2 * units + g.F - 1) / g.F, g.B}));
-    const int64_t per = Lf.floats_per_sample() * 4;
-    while (a.S > 1 && 2 * a.S * per > smem_limit) --a.S;
-    a.smem = 2 * a.S * per;
-    if (a.smem <= smem_limit) {
-      t_last_path = DLRM_PATH_PIPE;
-      const int qmax = std::max(1, kPipeDotWarps * 32 / (a.S * Lf.nT));
-      a.lq = std::min({log2_floor(qmax), log2_floor(std::max(1, Lf.D4)), 4});
-      a.tp = g.tp;
-      a.bp = g.bp;
-      a.B = g.B;
-      a.F = g.F;
-      a.D = g.D;
-      a.G = sh.G;
-      a.cpl = sh.cpl;
-      a.pool = g.pool;
-      a.dense = dense;
-      a.pooled_out = pooled_out;
-      a.inter_out = inter_out;
-      a.concat_dense = concat_dense;
-      a.sms = sm_count();
-      a.stream = stream;
-      return counted(g.esz == 4 ? launch_pipe_fused_f32(a) : launch_pipe_fused_bf16(a));
-    }
-  }
   t_last_path = DLRM_PATH_LDG;
   FusedLaunch a;
-  a.g = GatherLaunch{g.tp, g.bp, g.B, g.F, g.D, nullptr, g.pool, sh, stream};
+  a.g = GatherLaunch{g.tp, g.bp, g.B, g.F, g.D, nullptr, g.pool,
+                     choose_gather_shape(g.D, g.loader), stream};
   a.dense = dense;
   a.pooled_out = pooled_out;
   a.inter_out = inter_out;

@@ -45,7 +45,8 @@ struct FusedLaunch {
 };
 
 // cuTensorMapEncodeTiled, looked up once through the runtime's driver entry
-// point (null if the driver does not provide it).
+// point (null if the driver does not provide it); the MLP layers' TMA loads
+// use it.
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -54,61 +55,6 @@ EncodeTiledFn encode_tiled();
 
 // Records a failed CUDA call for dlrm_last_cuda_error() and returns DLRM_ERR_CUDA.
 int cuda_fail(cudaError_t e);
-
-// Tensor maps of the TMA gather path: one 2-D map per table ({D, rows},
-// box {D, 1}), passed by value in the kernel's parameter block.
-constexpr int kTmaMaxTables = 64;
-struct alignas(64) TmaParams {
-  CUtensorMap map[kTmaMaxTables];
-  int32_t rows[kTmaMaxTables];
-};
-
-struct TmaLaunch {
-  const TmaParams* tp;
-  BagParams bp;
-  int B, F, D;
-  int G;     // lanes per unit (8 or 16)
-  int cpl;   // 16-byte row chunks per lane (1 or 2)
-  int pool;  // PoolKind
-  float* out;  // gather-only output
-  // fused
-  const float* dense;
-  float* pooled_out;
-  float* inter_out;
-  int concat_dense;
-  int S, lq;
-  int64_t smem_limit;
-  int sms;
-  cudaStream_t stream;
-};
-
-// The persistent pipelined register-load path.
-struct PipeLaunch {
-  const TableParams* tp;
-  BagParams bp;
-  int B, F, D;
-  int G, cpl;  // lanes per unit, 16-byte chunks per lane
-  int pool;
-  float* out;  // gather-only output
-  const float* dense;
-  float* pooled_out;
-  float* inter_out;
-  int concat_dense;
-  int S, lq;
-  int64_t smem;
-  int sms;
-  cudaStream_t stream;
-};
-
-cudaError_t launch_pipe_gather_f32(const PipeLaunch& a);
-cudaError_t launch_pipe_gather_bf16(const PipeLaunch& a);
-cudaError_t launch_pipe_fused_f32(const PipeLaunch& a);
-cudaError_t launch_pipe_fused_bf16(const PipeLaunch& a);
-
-cudaError_t launch_tma_gather_f32(const TmaLaunch& a);
-cudaError_t launch_tma_gather_bf16(const TmaLaunch& a);
-cudaError_t launch_tma_fused_f32(const TmaLaunch& a);
-cudaError_t launch_tma_fused_bf16(const TmaLaunch& a);
 
 // One pair of launchers per loader (inst_*.cu).
 cudaError_t launch_gather_f32x4(const GatherLaunch& a);
@@ -128,20 +74,18 @@ struct GatherPlan {
   const TableParams* tp;
   BagParams bp;
   int B, F, D;
-  int pool;             // PoolKind
-  int loader;           // LoaderKind of the register (LDG) path
-  int esz;              // table element bytes (4 or 2)
-  bool tma_ok;          // tables and shape qualify for the TMA gather path
-  const int64_t* rows;  // host row counts, or null (then the maps span INT32_MAX rows)
+  int pool;    // PoolKind
+  int loader;  // LoaderKind
+  int esz;     // table element bytes (4 or 2)
 };
 
 // Process-wide choice of gather path (dlrm_set_gather_path).
 int gather_path();
 void set_gather_path(int path);
-// The path (DLRM_PATH_LDG / DLRM_PATH_TMA) of this thread's last gather launch.
+// The path (DLRM_PATH_LDG) of this thread's last gather launch.
 int last_path();
 
-// Picks the path and shape, then launches.
+// Picks the shape, then launches.
 cudaError_t launch_embbag(const GatherPlan& g, float* out, cudaStream_t stream);
 
 cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_out,

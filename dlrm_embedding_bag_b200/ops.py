@@ -34,7 +34,7 @@ STATUS = {
 }
 # Bytes of the library's own device staging (dlrm_sparse_interact_host_static).
 STATIC_SCRATCH_BYTES = 32 << 20
-GATHER_PATHS = {"auto": 0, "ldg": 1, "tma": 2, "pipe": 3}
+GATHER_PATHS = {"auto": 0, "ldg": 1}
 FLAG_INDEX_OOB = 1
 FLAG_OFFSETS = 2
 FLAG_TIMEOUT = 4
@@ -581,7 +581,7 @@ def pair_decode(p0: int, count: int, device="cuda"):
 
 
 def set_gather_path(path: str) -> str:
-    """Choose the gather path for later calls ("auto", "ldg", "tma", "pipe"); returns the old one."""
+    """Choose the gather path for later calls ("auto" or "ldg"); returns the old one."""
     prev = _lib.dlrm_set_gather_path(GATHER_PATHS[path])
     if prev < 0:
         raise DlrmError(prev, "dlrm_set_gather_path")
@@ -590,7 +590,7 @@ def set_gather_path(path: str) -> str:
 
 def last_gather_path() -> str:
     """The path that served this thread's last gather or fused launch."""
-    return {0: "none", 1: "ldg", 2: "tma", 3: "pipe"}[_lib.dlrm_last_gather_path()]
+    return {0: "none", 1: "ldg"}[_lib.dlrm_last_gather_path()]
 
 
 def status_from_flags(flags: int) -> int:

@@ -88,16 +88,13 @@ typedef enum {
 #define DLRM_FLAG_OFFSETS 2
 #define DLRM_FLAG_TIMEOUT 4
 
-/* Gather paths (dlrm_set_gather_path). */
+/* Gather paths (dlrm_set_gather_path). Earlier builds also offered a TMA
+ * tile::gather4 path (2), a persistent pipelined register-load path (3) and a
+ * persistent shared-memory ring path; each lost to DLRM_PATH_LDG on every
+ * measured workload and was removed. Those values are now rejected. */
 #define DLRM_PATH_AUTO 0 /* the path measured fastest on B200: DLRM_PATH_LDG */
 #define DLRM_PATH_LDG 1  /* one block per batch of bags (fused: of samples), register
                             (128-bit ld.global.nc) loads; serves every call */
-#define DLRM_PATH_TMA 2  /* the TMA tile::gather4 gather for the calls that qualify
-                            (see dlrm_set_gather_path), DLRM_PATH_LDG for the rest */
-#define DLRM_PATH_PIPE 3 /* persistent register-load units that prefetch the next bag's
-                            ids and bounds; rows of whole 16-byte chunks (f32: D % 4 == 0,
-                            D <= 256; bf16: D % 8 == 0, D <= 512) and 16-byte aligned
-                            tables and outputs, DLRM_PATH_LDG for the rest */
 
 /* Pooling of a bag's rows (torch.nn.EmbeddingBag modes). The pages implement
  * only SUM and name the others as what a later model would need (movement.rs,
@@ -326,23 +323,13 @@ DLRM_API int dlrm_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_t
 
 /*
  * dlrm_set_gather_path -- which gather serves later gather and fused calls of
- * this process (all threads): DLRM_PATH_AUTO (default), DLRM_PATH_LDG,
- * DLRM_PATH_TMA or DLRM_PATH_PIPE. Returns the previous setting, or DLRM_ERR_ARG for an unknown
- * value. Both paths give bit-identical pooled results; the choice exists for
- * testing and tuning.
- *
- * The TMA path serves a call when each table row is 64..512 bytes and a
- * multiple of 16 bytes (f32: D in 16..128, D % 4 == 0; bf16: D in 32..256,
- * D % 8 == 0), every table, the pooled output and the dense rows are 16-byte
- * aligned, F <= 64, and (fused) two tiles of features fit in shared memory.
- * It builds one tensor map per table on the host for every call. When row
- * counts are given (the calls that take `rows`), an index outside its table
- * reads zeros on this path instead of other memory.
+ * this process (all threads): DLRM_PATH_AUTO (default) or DLRM_PATH_LDG.
+ * Returns the previous setting, or DLRM_ERR_ARG for any other value.
  */
 DLRM_API int dlrm_set_gather_path(int path);
 
-/* The path (DLRM_PATH_LDG, _TMA or _PIPE) that served the calling thread's
- * last gather or fused launch; 0 before the first one. */
+/* The path (DLRM_PATH_LDG) that served the calling thread's last gather or
+ * fused launch; 0 before the first one. */
 DLRM_API int dlrm_last_gather_path(void);
 
 /* Status of a *status_dev value written by an _ex call (DLRM_OK if 0). */
@@ -360,8 +347,8 @@ DLRM_API int64_t dlrm_launch_count(void);
 /*
  * dlrm_probe_bounded_wait -- failure-detection check. One thread of one block
  * waits on a shared-memory mbarrier that nothing ever completes, with the same
- * bounded wait the asynchronous kernels use (the TMA gather path and the MLP
- * layers wait that way on their copies and tensor-core work). After about
+ * bounded wait the asynchronous kernels use (the MLP layers wait that way on
+ * their TMA copies and tensor-core work). After about
  * `limit_cycles` clock cycles (clamped to [1000, 2e8]) the wait gives up, the
  * kernel ORs DLRM_FLAG_TIMEOUT into *status_dev (dev int32, required) and
  * returns normally: the CUDA context stays usable. Asynchronous on `stream`.

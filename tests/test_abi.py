@@ -99,7 +99,8 @@ def test_status_strings_and_flags(ops):
     assert lib.dlrm_status_from_flags(4) == -8
     assert lib.dlrm_set_gather_path(7) == -9
     assert lib.dlrm_set_gather_path(1) == 0 and lib.dlrm_set_gather_path(0) == 1
-    assert lib.dlrm_set_gather_path(3) == 0 and lib.dlrm_set_gather_path(0) == 3
+    for retired in (2, 3, 4):
+        assert lib.dlrm_set_gather_path(retired) == -9
     assert lib.dlrm_launch_count() == 0
 
 
@@ -261,8 +262,7 @@ int main(void) {
          offsetof(dlrm_bags_t, include_last_offset), offsetof(dlrm_bags_t, mode));
   printf("%d %d %d %d %d %d %d\n", DLRM_MAX_TABLES, DLRM_FLAG_INDEX_OOB, DLRM_FLAG_OFFSETS,
          DLRM_FLAG_TIMEOUT, DLRM_POOL_SUM, DLRM_POOL_MEAN, DLRM_POOL_MAX);
-  printf("%d %d %d %d %d %d\n", DLRM_TABLE_F32, DLRM_TABLE_BF16, DLRM_PATH_AUTO, DLRM_PATH_LDG,
-         DLRM_PATH_TMA, DLRM_PATH_PIPE);
+  printf("%d %d %d %d\n", DLRM_TABLE_F32, DLRM_TABLE_BF16, DLRM_PATH_AUTO, DLRM_PATH_LDG);
   printf("%d %d %d\n", DLRM_ACT_NONE, DLRM_ACT_RELU, DLRM_ACT_SIGMOID);
   return 0;
 }
@@ -284,6 +284,6 @@ int main(void) {
     paths = [int(v) for v in lines[2].split()]
     import torch
     assert paths[:2] == [ops.TABLE_DTYPES[torch.float32], ops.TABLE_DTYPES[torch.bfloat16]]
-    assert paths[2:] == [ops.GATHER_PATHS[p] for p in ("auto", "ldg", "tma", "pipe")]
+    assert paths[2:] == [ops.GATHER_PATHS[p] for p in ("auto", "ldg")]
     assert [int(v) for v in lines[3].split()] == [mlp.ACTS[a] for a in ("none", "relu",
                                                                         "sigmoid")]

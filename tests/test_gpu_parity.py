@@ -28,16 +28,6 @@ def ops():
     return _ops
 
 
-@pytest.fixture(params=["pipe", "tma", "ldg"], autouse=True)
-def gather_path(request, ops):
-    """Every test runs on the pipelined path and on the TMA gather path (each
-    where the call qualifies; the per-block register loads serve the rest) and
-    on the per-block register-load path."""
-    prev = ops.set_gather_path(request.param)
-    yield request.param
-    ops.set_gather_path(prev)
-
-
 def _inputs(w: syn.Workload):
     weights = syn.make_weights(w, DEV)
     idx = syn.make_indices(w)
@@ -374,6 +364,68 @@ def test_host_stage_matches_device_path(ops):
     assert torch.equal(pooled2.view(torch.int32), pooled_h.view(torch.int32))
 
 
+def test_host_stage_matches_the_oracle(ops):
+    """The host-buffer entry point against the oracle directly (not only
+    against the device entry point)."""
+    w = syn.C2_CONCAT.scaled(B=300)
+    weights, idx, off, dense = _inputs(w)
+    stage = ops.HostStage(weights, w.B, w.L, concat_dense=True, want_pooled=True)
+    inter_h = torch.empty((w.B, w.D + w.P)).pin_memory()
+    pooled_h = torch.empty((w.B, w.F, w.D)).pin_memory()
+    stage(torch.from_numpy(idx.reshape(-1)).pin_memory(), torch.from_numpy(off).pin_memory(),
+          dense.cpu().pin_memory(), inter_h, pooled_h)
+    torch.cuda.synchronize()
+    ref_p, ref_i, bound = oracle_stage(host_tables(weights), idx, off, dense.cpu().numpy(), w.B,
+                                       w.L, True)
+    assert_bits_equal(pooled_h, ref_p, "host stage pooled")
+    check_inter(inter_h, ref_i, bound, w.D, True, "host stage")
+
+
+def test_one_hot_tables_are_exact(ops):
+    """Tables W_k[r, :] = e_(r mod D): every pooled value is an entry count and
+    every dot an integer, so both sides agree bit for bit, dots included."""
+    B, F, N, D, L = 67, 6, 200, 64, 9
+    w = syn.Workload("one_hot", B=B, F=F, N=N, D=D, L=L)
+    eye = torch.zeros((N, D), device=DEV)
+    eye[torch.arange(N), torch.arange(N) % D] = 1.0
+    weights = [eye.clone() for _ in range(F)]
+    idx, off = syn.make_indices(w), syn.make_offsets(w)
+    dense = torch.randint(-3, 4, (B, D), device=DEV).float()
+    pooled, inter_sep, fp, fi, fi2 = _run_all_paths(ops, weights, idx, off, dense, B, L, False)
+    ref_p, ref_i, _ = oracle_stage(host_tables(weights), idx, off, dense.cpu().numpy(), B, L,
+                                   False)
+    counts = np.zeros((B, F, D))
+    for k in range(F):
+        for b in range(B):
+            for r in idx[k, b * L:(b + 1) * L]:
+                counts[b, k, r % D] += 1
+    assert np.array_equal(ref_p, counts)
+    for got, what in ((pooled, "gather"), (fp, "fused pooled")):
+        assert_bits_equal(got, ref_p, "one-hot " + what)
+    for got, what in ((inter_sep, "interact"), (fi, "fused"), (fi2, "fused, no pooled")):
+        assert_bits_equal(got, ref_i.astype(np.float32), "one-hot dots " + what)
+
+
+def test_bag_of_copies_is_exact(ops):
+    """A bag of L copies of one row r pools to exactly L * W[r] when the rows
+    hold k/256 values (|k| < 256): every partial sum is representable."""
+    B, F, N, D, L = 45, 5, 300, 64, 12
+    rng = np.random.default_rng(23)
+    weights = [torch.from_numpy((rng.integers(-255, 256, (N, D)) / 256.0).astype(np.float32))
+               .to(DEV) for _ in range(F)]
+    rows = rng.integers(0, N, (F, B))
+    idx = np.repeat(rows, L, axis=1).astype(np.int32)
+    off = syn.make_offsets(syn.Workload("copies", B=B, F=F, N=N, D=D, L=L))
+    dense = torch.zeros((B, D), device=DEV)
+    pooled, _, fp, _, _ = _run_all_paths(ops, weights, idx, off, dense, B, L, False)
+    want = np.stack([np.stack([L * weights[k][rows[k, b]].cpu().numpy().astype(np.float64)
+                               for k in range(F)]) for b in range(B)])
+    ref_p, _, _ = oracle_stage(host_tables(weights), idx, off, dense.cpu().numpy(), B, L, False)
+    assert np.array_equal(ref_p, want)
+    assert_bits_equal(pooled, want.astype(np.float32), "copies gather")
+    assert_bits_equal(fp, want.astype(np.float32), "copies fused")
+
+
 def test_repeat_runs_are_bit_identical_and_launch_once(ops):
     w = syn.C2_CONCAT.scaled(B=512)
     weights, idx, off, dense = _inputs(w)
@@ -448,37 +500,18 @@ def test_host_pipeline_overlapped_batches(ops):
 
 
 def test_path_choice(ops):
-    """Under "tma" qualifying calls run the TMA gather, under "pipe" calls with
-    16-byte row chunks in one column window run the pipelined kernels, and all
-    other calls (every call under "auto") the per-block register loads."""
-    prev = ops.set_gather_path("tma")
+    """Every call runs the per-block register-load path; the retired path
+    numbers are rejected."""
+    prev = ops.set_gather_path("auto")
     try:
-        for (B, F, N, D, L) in [(70, 5, 300, 64, 16), (33, 26, 200, 128, 20), (19, 2, 50, 16, 4),
-                                (9, 3, 40, 48, 11)]:
-            weights, idx, off, dense = _random_case(B + F, B, F, N, D, L)
-            ops.embbag_sum_multi(weights, _dev_i32(idx), _dev_i32(off), L)
-            assert ops.last_gather_path() == "tma"
-            ops.sparse_interact(weights, _dev_i32(idx), _dev_i32(off), dense, L)
-            assert ops.last_gather_path() == "tma"
-        weights, idx, off, dense = _random_case(3, 8, 2, 20, 6, 3)  # 24-byte rows
-        ops.embbag_sum_multi(weights, _dev_i32(idx), _dev_i32(off), 3)
-        assert ops.last_gather_path() == "ldg"
-        for name, want in (("pipe", "pipe"), ("auto", "ldg")):
-            ops.set_gather_path(name)
-            for D in (16, 64, 128, 256):
-                weights, idx, off, dense = _random_case(D, 5, 3, 40, D, 4)
-                ops.embbag_sum_multi(weights, _dev_i32(idx), _dev_i32(off), 4)
-                assert ops.last_gather_path() == want
-                ops.sparse_interact(weights, _dev_i32(idx), _dev_i32(off), dense, 4)
-                assert ops.last_gather_path() == want
-            for D in (6, 512):  # 24-byte rows; two column windows
-                weights, idx, off, dense = _random_case(D, 5, 3, 40, D, 4)
-                ops.embbag_sum_multi(weights, _dev_i32(idx), _dev_i32(off), 4)
-                assert ops.last_gather_path() == "ldg"
-        ops.set_gather_path("ldg")
-        weights, idx, off, dense = _random_case(4, 8, 2, 20, 64, 3)
-        ops.sparse_interact(weights, _dev_i32(idx), _dev_i32(off), dense, 3)
-        assert ops.last_gather_path() == "ldg"
+        for D in (6, 16, 64, 128, 512):
+            weights, idx, off, dense = _random_case(D, 5, 3, 40, D, 4)
+            ops.embbag_sum_multi(weights, _dev_i32(idx), _dev_i32(off), 4)
+            assert ops.last_gather_path() == "ldg"
+            ops.sparse_interact(weights, _dev_i32(idx), _dev_i32(off), dense, 4)
+            assert ops.last_gather_path() == "ldg"
+        for retired in (2, 3, 4):
+            assert ops._lib.dlrm_set_gather_path(retired) == -9
         torch.cuda.synchronize()
     finally:
         ops.set_gather_path(prev)

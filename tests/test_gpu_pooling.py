@@ -28,16 +28,6 @@ def ops():
     return _ops
 
 
-@pytest.fixture(params=["pipe", "tma", "ldg"], autouse=True)
-def gather_path(request, ops):
-    """Every test runs on the pipelined path and on the TMA gather path (each
-    where the call qualifies; the per-block register loads serve the rest) and
-    on the per-block register-load path."""
-    prev = ops.set_gather_path(request.param)
-    yield request.param
-    ops.set_gather_path(prev)
-
-
 def _host_bits(t: torch.Tensor) -> np.ndarray:
     """Host copy of a table: f32 values, or bf16 bit patterns as uint16."""
     if t.dtype == torch.bfloat16:
