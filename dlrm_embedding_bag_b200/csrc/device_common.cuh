@@ -40,13 +40,36 @@ enum PoolKind { kPoolSum = 0, kPoolWeighted = 1, kPoolMax = 2 };
 // Row loaders: one lane loads VEC consecutive table elements per request and
 // hands them out widened to f32.
 
+#ifndef DLRM_ROW_LOAD_HINT
+#define DLRM_ROW_LOAD_HINT 0
+#endif
 struct LdF32x4 {  // 128-bit loads of 4 floats
   static constexpr int VEC = 4;
   using Elem = float;
   using Raw = float4;
   __device__ __forceinline__ static Raw zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
   __device__ __forceinline__ static Raw load(const Elem* p) {
+#if DLRM_ROW_LOAD_HINT == 1
+    float4 r;
+    asm("ld.global.nc.L2::256B.v4.f32 {%0, %1, %2, %3}, [%4];"
+        : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+        : "l"(p));
+    return r;
+#elif DLRM_ROW_LOAD_HINT == 2
+    float4 r;
+    asm("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+        : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+        : "l"(p));
+    return r;
+#elif DLRM_ROW_LOAD_HINT == 3
+    float4 r;
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.f32 {%0, %1, %2, %3}, [%4];"
+        : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+        : "l"(p));
+    return r;
+#else
     return __ldg(reinterpret_cast<const float4*>(p));
+#endif
   }
   __device__ __forceinline__ static float get(const Raw& r, int e) {
     return e == 0 ? r.x : e == 1 ? r.y : e == 2 ? r.z : r.w;

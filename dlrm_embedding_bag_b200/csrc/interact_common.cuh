@@ -168,6 +168,134 @@ __device__ __forceinline__ void dots_from_smem(const float* feat, const FeatLayo
   }
 }
 
+// The 4x4 tiles (I, J), I >= J, of the lower triangle, decoded once per block
+// from their flat index with the pair decoder (tile (I, J) is pair (I+1, J) of
+// a triangle one larger): tiles[t] = I << 8 | J. Run by nthreads threads.
+__device__ __forceinline__ void decode_tiles(uint16_t* tiles, int nT, int tid, int nthreads) {
+  for (int t = tid; t < nT; t += nthreads) {
+    int I1, J;
+    pair_from_flat_small(t, I1, J);
+    tiles[t] = static_cast<uint16_t>(((I1 - 1) << 8) | J);
+  }
+}
+
+// dots_from_smem for a row length fixed at compile time: D4 float4 chunks of
+// data per feature row, RS float4 per row in shared memory, 2^LQ lanes per
+// tile, tiles from the table decode_tiles wrote. Every shared-memory read of
+// a tile is an immediate offset from one of two base addresses and the column
+// loop is fully unrolled. Same tasks, sums and stores as dots_from_smem.
+template <int D4, int RS, int LQ>
+__device__ __forceinline__ void dots_fixed(const float* feat, const FeatLayout& Lf,
+                                           const uint16_t* tiles, int S_here,
+                                           float* __restrict__ out, int64_t b0,
+                                           int64_t row_stride, int64_t col0, int tid,
+                                           int nthreads) {
+  constexpr int Q = 1 << LQ;
+  constexpr int ITER = (D4 + Q - 1) / Q;
+  const int total = (S_here * Lf.nT) << LQ;
+  const int lane = tid & 31;
+  const int per_sample = Lf.F1p * RS;
+  for (int base = tid - lane; base < total; base += nthreads) {
+    const int task = base + lane;
+    const bool active = task < total;
+    const int tt = active ? task : 0;
+    const int q = tt & (Q - 1);
+    const int rest = tt >> LQ;
+    int t = rest, s = 0;
+    if (S_here > 1) {
+      s = rest / Lf.nT;
+      t = rest - s * Lf.nT;
+    }
+    const int IJ = tiles[t];
+    const int I = IJ >> 8, J = IJ & 255;
+    const float4* fi = reinterpret_cast<const float4*>(feat) + s * per_sample + 4 * I * RS + q;
+    const float4* fj = reinterpret_cast<const float4*>(feat) + s * per_sample + 4 * J * RS + q;
+    float acc[16];
+#pragma unroll
+    for (int v = 0; v < 16; ++v) acc[v] = 0.f;
+#pragma unroll
+    for (int it = 0; it < ITER; ++it) {
+      if (it * Q + q < D4 || (D4 % Q) == 0) {
+        float4 a[4], bv[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) a[r] = fi[r * RS + it * Q];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) bv[c] = fj[c * RS + it * Q];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float x = acc[4 * r + c];
+            x = fmaf(a[r].x, bv[c].x, x);
+            x = fmaf(a[r].y, bv[c].y, x);
+            x = fmaf(a[r].z, bv[c].z, x);
+            x = fmaf(a[r].w, bv[c].w, x);
+            acc[4 * r + c] = x;
+          }
+      }
+    }
+    tile_reduce_store<LQ>(acc, q, active, I, J, Lf.F1, out + (b0 + s) * row_stride + col0);
+  }
+}
+
+// dots_fixed for the runtime lq (2, 3 or 4: the shapes the launches choose
+// for these row lengths; smaller lq goes to dots_from_smem).
+template <int D4, int RS>
+__device__ __forceinline__ void dots_fixed_lq(const float* feat, const FeatLayout& Lf,
+                                              const uint16_t* tiles, int S_here, int lq,
+                                              float* __restrict__ out, int64_t b0,
+                                              int64_t row_stride, int64_t col0, int tid,
+                                              int nthreads) {
+  switch (lq) {
+    case 2:
+      dots_fixed<D4, RS, 2>(feat, Lf, tiles, S_here, out, b0, row_stride, col0, tid, nthreads);
+      break;
+    case 3:
+      dots_fixed<D4, RS, 3>(feat, Lf, tiles, S_here, out, b0, row_stride, col0, tid, nthreads);
+      break;
+    default:
+      dots_fixed<D4, RS, 4>(feat, Lf, tiles, S_here, out, b0, row_stride, col0, tid, nthreads);
+      break;
+  }
+}
+
+
+// Bytes of the tile table decode_tiles writes (a multiple of 16).
+__host__ __device__ inline int64_t tile_table_bytes(int nT) { return (2 * nT + 15) / 16 * 16; }
+
+// The tile table sits in the last tile_table_bytes(nT) of the block's dynamic
+// shared memory.
+__device__ __forceinline__ uint16_t* tile_table(void* smem_base, int nT) {
+  uint32_t total;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(total));
+  return reinterpret_cast<uint16_t*>(static_cast<char*>(smem_base) + total -
+                                     tile_table_bytes(nT));
+}
+
+// The dot phase of the interaction kernel for any row shape: the
+// compile-time routine for the common row lengths (D = 64 and 128 with the
+// padded layout) and lq >= 2, dots_from_smem for the rest. tiles is the table
+// decode_tiles wrote (used by the fixed routine), or null when the block's
+// shared memory has no room for it. (Measured on B200: in the interaction
+// kernel the fixed routine took c3 from 24.6 to 23.0 us; in the fused kernel,
+// whose dot phase runs beside other blocks' gathers, it cost 2.5 us, so the
+// fused kernel keeps dots_from_smem.)
+template <int UNROLL = 1>
+__device__ __forceinline__ void dots_any(const float* feat, const FeatLayout& Lf,
+                                         const uint16_t* tiles, int S_here, int lq,
+                                         float* __restrict__ out, int64_t b0, int64_t row_stride,
+                                         int64_t col0, int tid, int nthreads) {
+  if (tiles != nullptr && lq >= 2 && Lf.D4 == 16 && Lf.Dp == 68) {
+    dots_fixed_lq<16, 17>(feat, Lf, tiles, S_here, lq, out, b0, row_stride, col0, tid, nthreads);
+    return;
+  }
+  if (tiles != nullptr && lq >= 2 && Lf.D4 == 32 && Lf.Dp == 132) {
+    dots_fixed_lq<32, 33>(feat, Lf, tiles, S_here, lq, out, b0, row_stride, col0, tid, nthreads);
+    return;
+  }
+  dots_from_smem<UNROLL>(feat, Lf, S_here, lq, out, b0, row_stride, col0, tid, nthreads);
+}
+
 // Ampere-style asynchronous global -> shared copies (cp.async), used to stage
 // the next group of samples while the current one is computed.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {

@@ -53,10 +53,19 @@ __device__ __forceinline__ void stage_interact_group(float* buf, const FeatLayou
   }
 }
 
+// Blocks of the interaction kernel per SM (its register budget), and the
+// unrolling of the general dot routine's column loop.
+#ifndef DLRM_INTERACT_MIN_BLOCKS
+#define DLRM_INTERACT_MIN_BLOCKS 4
+#endif
+#ifndef DLRM_INTERACT_UNROLL
+#define DLRM_INTERACT_UNROLL 2
+#endif
+
 template <int VEC, int DP>
-__global__ void __launch_bounds__(kBlockThreads, 2)
+__global__ void __launch_bounds__(kBlockThreads, DLRM_INTERACT_MIN_BLOCKS)
     interact_kernel(const float* __restrict__ dense, const float* __restrict__ emb, int B, int F,
-                    int D, int S, int lq, int nbuf, float* __restrict__ out) {
+                    int D, int S, int lq, int nbuf, int with_tiles, float* __restrict__ out) {
   extern __shared__ __align__(16) float feat[];
   const FeatLayout Lf = FeatLayout::make(F, D);
   // buffer i at feat + i * bstride
@@ -70,6 +79,8 @@ __global__ void __launch_bounds__(kBlockThreads, 2)
   // The copies never write the padding, so it is zeroed once per buffer.
   for (int i = 0; i < nbuf; ++i)
     zero_feature_padding(feat + i * bstride, Lf, D, S, threadIdx.x, blockDim.x);
+  uint16_t* tiles = with_tiles ? tile_table(feat, Lf.nT) : nullptr;
+  if (tiles) decode_tiles(tiles, Lf.nT, threadIdx.x, blockDim.x);
   int64_t g = blockIdx.x;
   if (nbuf == 1) {
     for (; g < ngroups; g += gridDim.x) {
@@ -77,8 +88,8 @@ __global__ void __launch_bounds__(kBlockThreads, 2)
       cp_async_commit();
       cp_async_wait<0>();
       __syncthreads();
-      dots_from_smem<2, DP>(feat, Lf, samples(g), lq, out, g * S, P, 0, threadIdx.x,
-                            blockDim.x);
+      dots_any<DLRM_INTERACT_UNROLL>(feat, Lf, tiles, samples(g), lq, out, g * S, P, 0,
+                                     threadIdx.x, blockDim.x);
       __syncthreads();
     }
     return;
@@ -93,8 +104,8 @@ __global__ void __launch_bounds__(kBlockThreads, 2)
     cp_async_commit();
     cp_async_wait<1>();  // group g has landed (only the copy of group gn may be pending)
     __syncthreads();
-    dots_from_smem<2, DP>(feat + (it & 1) * bstride, Lf, samples(g), lq, out, g * S, P, 0,
-                          threadIdx.x, blockDim.x);
+    dots_any<DLRM_INTERACT_UNROLL>(feat + (it & 1) * bstride, Lf, tiles, samples(g), lq, out,
+                                   g * S, P, 0, threadIdx.x, blockDim.x);
     __syncthreads();  // buffer it&1 is refilled in the next iteration
   }
   cp_async_wait<0>();
@@ -322,11 +333,13 @@ static cudaError_t run_interact(const float* dense, const float* emb, int B, int
   const int64_t per = Lf.floats_per_sample() * 4;
   if (per > smem_limit) return cudaErrorInvalidValue;
   auto* fn = &interact_kernel<VEC, DP>;
-  const int64_t budget = std::min<int64_t>(smem_limit, 100 * 1024);  // two blocks per SM
+  const int64_t budget = std::min<int64_t>(smem_limit, 200 * 1024 / DLRM_INTERACT_MIN_BLOCKS);
   int S, lq;
   choose_interact_shape(F, D, B, budget, S, lq);
   const int nbuf = (2 * S * per <= smem_limit) ? 2 : 1;
-  const int64_t smem = nbuf * S * per;
+  const int64_t tbytes = tile_table_bytes(Lf.nT);
+  const int with_tiles = nbuf * S * per + tbytes <= smem_limit ? 1 : 0;
+  const int64_t smem = nbuf * S * per + (with_tiles ? tbytes : 0);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -341,7 +354,7 @@ static cudaError_t run_interact(const float* dense, const float* emb, int B, int
   const int64_t ngroups = (static_cast<int64_t>(B) + S - 1) / S;
   const int64_t grid = std::min<int64_t>(ngroups, static_cast<int64_t>(per_sm) * sms);
   fn<<<static_cast<unsigned>(grid), kBlockThreads, smem, stream>>>(dense, emb, B, F, D, S, lq,
-                                                                  nbuf, out);
+                                                                  nbuf, with_tiles, out);
   return cudaGetLastError();
 }
 

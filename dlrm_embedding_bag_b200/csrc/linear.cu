@@ -76,6 +76,7 @@ struct alignas(64) LinMaps {
   CUtensorMap a[kLinMaxAMaps];
   CUtensorMap w[kLinMaxWMaps];
   CUtensorMap y32, y16;
+  CUtensorMap yp[3];  // the three bf16 planes of an f32-activation output
 };
 
 // The K blocks of a tile, in order, are the concatenation of segments: nkb
@@ -98,6 +99,7 @@ struct LinearArgs {
   int nseg, nkb;
   int tiles_n, tiles;
   int tma_f32, tma_bf16;  // write that output through TMA stores (see the launcher)
+  int tma_planes;         // the same for the three planes (through the bf16 staging)
   int32_t* status;
 };
 
@@ -328,12 +330,12 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     const bool planes_vec = args.y_planes != nullptr && (args.ldy_planes % 8) == 0 &&
                             (args.splane_y % 8) == 0 &&
                             (reinterpret_cast<uintptr_t>(args.y_planes) % 16) == 0;
-    const bool tma_out = args.tma_f32 || args.tma_bf16;
+    const bool tma_out = args.tma_f32 || args.tma_bf16 || args.tma_planes;
     // the outputs not written through TMA
     LinOut direct;
     direct.y_f32 = args.tma_f32 ? nullptr : args.y_f32;
     direct.y_bf16 = args.tma_bf16 ? nullptr : args.y_bf16;
-    direct.y_planes = args.y_planes;
+    direct.y_planes = args.tma_planes ? nullptr : args.y_planes;
     direct.ldy_f32 = args.ldy_f32;
     direct.ldy_bf16 = args.ldy_bf16;
     direct.ldy_planes = args.ldy_planes;
@@ -399,6 +401,40 @@ __global__ void __launch_bounds__(kLinThreads, 1)
             if (F32S && args.tma_f32) tma_store_2d(&maps.y32, st32, n0 + c0, row0);
             if (args.tma_bf16) tma_store_2d(&maps.y16, st16, n0 + c0, row0);
             bulk_commit();
+          }
+          if (args.tma_planes) {
+            // the three planes one after another through the bf16 staging tile
+            // (an f32-activation layer writes no bf16 output)
+#pragma unroll
+            for (int p = 0; p < 3; ++p) {
+              if (p > 0) {
+                if (lane == 0) bulk_wait_read_all();  // the previous plane has left
+                __syncwarp();
+              }
+              uint4* rowp = reinterpret_cast<uint4*>(st16 + lane * 64);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  uint32_t h[2];
+#pragma unroll
+                  for (int u = 0; u < 2; ++u) {
+                    uint16_t a0, a1, a2;
+                    split_bf16x3(v[8 * q + 2 * e + u], a0, a1, a2);
+                    h[u] = p == 0 ? a0 : (p == 1 ? a1 : a2);
+                  }
+                  w4[e] = h[0] | (h[1] << 16);
+                }
+                rowp[q ^ ((lane >> 1) & 3)] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&maps.yp[p], st16, n0 + c0, row0);
+                bulk_commit();
+              }
+            }
           }
         }
         if (any_direct) store_chunk32(direct, row0 + lane, n0 + c0, v, f32_vec, bf_vec, planes_vec);
@@ -597,6 +633,13 @@ int launch_layer(const APart* parts, int nparts, int a_planes, const uint16_t* w
   if (e == cudaSuccess && args.tma_bf16)
     e = encode_output(&maps.y16, y_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, ldy_bf16,
                       CU_TENSOR_MAP_SWIZZLE_64B);
+  // the planes go out through the bf16 staging tile, which a layer writing
+  // planes does not otherwise use
+  args.tma_planes = y_planes != nullptr && y_bf16 == nullptr && ldy_planes % 8 == 0 &&
+                    splane_y % 8 == 0 && is_aligned(y_planes, 16);
+  for (int p = 0; p < 3 && e == cudaSuccess && args.tma_planes; ++p)
+    e = encode_output(&maps.yp[p], y_planes + p * splane_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N,
+                      M, ldy_planes, CU_TENSOR_MAP_SWIZZLE_64B);
   if (e != cudaSuccess) return cuda_fail(e);
   switch (bn) {
     case 256: e = run_linear_bn<256>(act, maps, args, sms, stream); break;
