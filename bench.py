@@ -120,7 +120,7 @@ def measured_peaks():
 # The sources the benchmarked fused kernel and its launch are built from: a
 # recorded DRAM traffic figure stays valid while none of them changes.
 FUSED_SOURCES = [os.path.join(CSRC, n) for n in (
-    "device_common.cuh", "interact_common.cuh", "kernels.cuh", "inst_f32x4.cu", "kernels.cu",
+    "device_common.cuh", "interact_common.cuh", "kernels.cuh", "inst_f32x4s.cu", "kernels.cu",
     "launch.h", "api.cu")] + [os.path.join(ROOT, "include", "dlrm_sparse.h")]
 
 

@@ -100,11 +100,13 @@ int prepare(const void* const* weights, int dtype, const int64_t* rows, const dl
 }
 
 // The vector loader needs whole 16-byte chunks per row and 16-byte aligned
-// tables and float destinations.
+// tables and float destinations. f32 rows of at most 64 floats stream past L1
+// (measured faster there; longer rows under skew gain from L1).
 int pick_loader(int dtype, int D, bool vec_ok) {
   if (dtype == DLRM_TABLE_BF16)
     return (vec_ok && D % 8 == 0) ? dlrm::kLdBF16x8 : dlrm::kLdBF16x1;
-  return (vec_ok && D % 4 == 0) ? dlrm::kLdF32x4 : dlrm::kLdF32x1;
+  if (!vec_ok || D % 4 != 0) return dlrm::kLdF32x1;
+  return D <= 64 ? dlrm::kLdF32x4S : dlrm::kLdF32x4;  // see LdF32x4S
 }
 
 int clear_status(int32_t* status_dev, cudaStream_t stream) {

@@ -40,40 +40,36 @@ enum PoolKind { kPoolSum = 0, kPoolWeighted = 1, kPoolMax = 2 };
 // Row loaders: one lane loads VEC consecutive table elements per request and
 // hands them out widened to f32.
 
-#ifndef DLRM_ROW_LOAD_HINT
-#define DLRM_ROW_LOAD_HINT 0
-#endif
+// Row loads that do not allocate in L1 (ld.global.nc.L1::no_allocate), for
+// rows that are read once per lookup and rarely again by the same SM: L1 is
+// left to the requests in flight. Measured on B200 against plain __ldg, with
+// 256-byte f32 rows (D = 64): fused c3 52.2 -> 49.9 us, c3u 70.1 -> 66.0 us,
+// gather alone c3u 65.0 -> 58.6 us; but with 512-byte rows under a steeper
+// skew (c5: D = 128, Zipf 1.2) 1.62 -> 1.70 ms and with 128-byte bf16 rows
+// 44.6 -> 49.0 us, where L1 serves enough hot rows to pay. So the launch picks
+// the streaming loader (LdF32x4S) for f32 rows of at most 64 floats only.
+__device__ __forceinline__ float4 ldg_row_f32x4(const float* p) {
+  float4 r;
+  asm("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+      : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+      : "l"(p));
+  return r;
+}
 struct LdF32x4 {  // 128-bit loads of 4 floats
   static constexpr int VEC = 4;
   using Elem = float;
   using Raw = float4;
   __device__ __forceinline__ static Raw zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
   __device__ __forceinline__ static Raw load(const Elem* p) {
-#if DLRM_ROW_LOAD_HINT == 1
-    float4 r;
-    asm("ld.global.nc.L2::256B.v4.f32 {%0, %1, %2, %3}, [%4];"
-        : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
-        : "l"(p));
-    return r;
-#elif DLRM_ROW_LOAD_HINT == 2
-    float4 r;
-    asm("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
-        : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
-        : "l"(p));
-    return r;
-#elif DLRM_ROW_LOAD_HINT == 3
-    float4 r;
-    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.f32 {%0, %1, %2, %3}, [%4];"
-        : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
-        : "l"(p));
-    return r;
-#else
     return __ldg(reinterpret_cast<const float4*>(p));
-#endif
   }
   __device__ __forceinline__ static float get(const Raw& r, int e) {
     return e == 0 ? r.x : e == 1 ? r.y : e == 2 ? r.z : r.w;
   }
+};
+
+struct LdF32x4S : LdF32x4 {  // the same, streaming (no L1 allocation)
+  __device__ __forceinline__ static Raw load(const Elem* p) { return ldg_row_f32x4(p); }
 };
 
 struct LdF32x1 {  // scalar fallback

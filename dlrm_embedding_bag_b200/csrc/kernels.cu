@@ -159,6 +159,7 @@ static int log2_floor(int x) {
 static int loader_vec(int loader) {
   switch (loader) {
     case kLdF32x4: return 4;
+    case kLdF32x4S: return 4;
     case kLdBF16x8: return 8;
     default: return 1;
   }
@@ -272,6 +273,7 @@ cudaError_t launch_embbag(const GatherPlan& g, float* out, cudaStream_t stream) 
   GatherLaunch a{g.tp, g.bp, g.B, g.F, g.D, out, g.pool, sh, stream};
   switch (g.loader) {
     case kLdF32x4: return counted(launch_gather_f32x4(a));
+    case kLdF32x4S: return counted(launch_gather_f32x4s(a));
     case kLdF32x1: return counted(launch_gather_f32x1(a));
     case kLdBF16x8: return counted(launch_gather_bf16x8(a));
     case kLdBF16x1: return counted(launch_gather_bf16x1(a));
@@ -305,6 +307,7 @@ cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_
   if (a.smem > smem_limit) return cudaErrorInvalidValue;
   switch (g.loader) {
     case kLdF32x4: return counted(launch_fused_f32x4(a));
+    case kLdF32x4S: return counted(launch_fused_f32x4s(a));
     case kLdF32x1: return counted(launch_fused_f32x1(a));
     case kLdBF16x8: return counted(launch_fused_bf16x8(a));
     case kLdBF16x1: return counted(launch_fused_bf16x1(a));

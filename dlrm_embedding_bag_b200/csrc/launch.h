@@ -15,7 +15,7 @@ namespace dlrm {
 #endif
 
 // Which row loader a launch uses.
-enum LoaderKind { kLdF32x4 = 0, kLdF32x1 = 1, kLdBF16x8 = 2, kLdBF16x1 = 3 };
+enum LoaderKind { kLdF32x4 = 0, kLdF32x1 = 1, kLdBF16x8 = 2, kLdBF16x1 = 3, kLdF32x4S = 4 };
 
 // Template shape of the gather for a row length D: the loader, G lanes per bag,
 // CPL column chunks per lane, and the number of column windows that cover D.
@@ -58,10 +58,12 @@ int cuda_fail(cudaError_t e);
 
 // One pair of launchers per loader (inst_*.cu).
 cudaError_t launch_gather_f32x4(const GatherLaunch& a);
+cudaError_t launch_gather_f32x4s(const GatherLaunch& a);
 cudaError_t launch_gather_f32x1(const GatherLaunch& a);
 cudaError_t launch_gather_bf16x8(const GatherLaunch& a);
 cudaError_t launch_gather_bf16x1(const GatherLaunch& a);
 cudaError_t launch_fused_f32x4(const FusedLaunch& a);
+cudaError_t launch_fused_f32x4s(const FusedLaunch& a);
 cudaError_t launch_fused_f32x1(const FusedLaunch& a);
 cudaError_t launch_fused_bf16x8(const FusedLaunch& a);
 cudaError_t launch_fused_bf16x1(const FusedLaunch& a);
