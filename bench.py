@@ -552,7 +552,8 @@ def run_ours(args, w: syn.Workload):
                                    "value": w.B * w.F * w.L / (u_ms / 1e3),
                                    "unit": "lookups/s",
                                    "achieved_gbs": algorithmic_bytes(wu) / (u_ms / 1e3) / 1e9,
-                                   "algorithmic_bytes_per_launch": algorithmic_bytes(wu)}
+                                   "algorithmic_bytes_per_launch": algorithmic_bytes(wu),
+                                   "traffic": recorded_traffic(wu.name)}
             del idx_u, call_u
 
     # e2e through the host-buffer entry point: every step copies its batch's
