@@ -108,6 +108,17 @@ def algorithmic_bytes(w: syn.Workload, write_pooled: bool = True, esz: int = 4,
     return rows + idx + offs + dense + pooled + inter
 
 
+def hold_stream(steps: int, per_step_ms: float = 0.1) -> None:
+    """Keep the current stream busy (a device-side spin of about steps x
+    per_step_ms, at most 50 ms) while the host queues the steps that follow,
+    so that each step's CUDA events bracket the GPU's work and not a gap in
+    which the GPU waited for the host to launch it. The spin runs before the
+    first step, outside every step's events."""
+    import torch
+    ms = min(50.0, steps * per_step_ms)
+    torch.cuda._sleep(int(ms * 2.0e6))  # cycles at about 2 GHz
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -480,6 +491,7 @@ def run_ours(args, w: syn.Workload):
         sampler.start()
         n0 = ops.launch_count()
         w0 = time.perf_counter()
+        hold_stream(args.steps)
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
             starts[i].record()
@@ -516,6 +528,7 @@ def run_ours(args, w: syn.Workload):
         for _ in range(5):
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(21)]
             torch.cuda.synchronize()
+            hold_stream(20)
             ev[0].record()
             for i in range(20):
                 step()
@@ -541,6 +554,7 @@ def run_ours(args, w: syn.Workload):
                 call_u(stream)
             ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
             ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+            hold_stream(args.steps)
             for i in range(args.steps):
                 flush.fill_(i & 0xFF)
                 ev_s[i].record()
@@ -681,6 +695,7 @@ def run_ours(args, w: syn.Workload):
             "clocks": clocks, "remeasured": remeasured,
             "gpu_launches": launches,
             "region_wall_ms": 1e3 * wall,
+            "region_hold_ms": min(50.0, args.steps * 0.1),
             "step_ms_p50": statistics.median(per), "step_ms_min": min(per),
             "e2e": e2e,
         }
@@ -740,6 +755,7 @@ def run_sweep(args):
         torch.cuda.synchronize()
         st = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         en = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        hold_stream(args.steps)
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
             st[i].record()
@@ -784,6 +800,7 @@ def run_mlp(args, w: syn.Workload):
         torch.cuda.synchronize()
         st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
         en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        hold_stream(steps, 0.2)
         for i in range(steps):
             flush.fill_(i & 0xFF)
             st[i].record()

@@ -20,6 +20,12 @@
 //     activation and store f32 and/or bf16, then hand the accumulator back -
 //     so the epilogue of tile i runs while the MMAs of tile i+1 fill the
 //     other accumulator.
+// Large layers run the same roles on CTA pairs (clusters of two, tcgen05
+// cta_group::2): a pair owns 256 x BN tiles, each CTA loads its 128 rows of A
+// and half of the tile's W rows per stage, the even CTA issues M = 256 MMAs
+// over both CTAs' shared memory, and each CTA's epilogue drains its own 128
+// accumulator rows from its own TMEM. Per SM, a stage then brings in 16 KB of
+// W instead of 32 KB for the same tensor-core work.
 // Every wait on an mbarrier is bounded; a wait that runs out sets
 // DLRM_FLAG_TIMEOUT in the optional status word, ends that role's loop, and
 // the CTA still frees its tensor memory and exits.
@@ -40,30 +46,36 @@ namespace {
 constexpr int kLinBM = 128;    // rows of a tile (tcgen05 M)
 constexpr int kLinBK = 64;     // K per stage: 64 bf16 = one 128-byte swizzle row
 // Shared-memory ring depth: 4 stages, except with 256-column tiles (48 KB
-// stages) next to the f32 output staging, where only 3 fit.
-template <int BN, bool F32S>
-constexpr int lin_stages() { return (BN >= 256 && F32S) ? 3 : 4; }
+// stages) next to the f32 output staging, where only 3 fit; CTA pairs hold
+// half of the W rows per stage (32 KB stages at BN = 256): 6 stages, 5 next
+// to the f32 staging.
+template <int BN, bool F32S, bool PAIR>
+constexpr int lin_stages() {
+  if constexpr (PAIR) return F32S ? 5 : 6;
+  return (BN >= 256 && F32S) ? 3 : 4;
+}
 constexpr int kLinEpiWarps = 8;  // two per TMEM lane quarter, each half of the columns
 constexpr int kLinThreads = 64 + 32 * kLinEpiWarps;  // producer warp, MMA warp, epilogue
 constexpr long long kLinWaitLimit = 200000000LL;  // clock cycles, about 0.1 s
 
-template <int BN, bool F32S>
+template <int BN, bool F32S, bool PAIR>
 struct LinSmem {
-  static constexpr int kStages = lin_stages<BN, F32S>();
+  static constexpr int kStages = lin_stages<BN, F32S, PAIR>();
   static constexpr int kA = kLinBM * kLinBK * 2;
-  static constexpr int kB = BN * kLinBK * 2;
+  static constexpr int kB = (PAIR ? BN / 2 : BN) * kLinBK * 2;
   static constexpr int kStage = kA + kB;
   // After the ring: each epilogue warp's output staging (a 32 x 32 f32 tile in
   // the 128-byte swizzled layout when F32S -- the f32 output goes out through
   // TMA --, then a 32 x 32 bf16 tile in the 64-byte swizzled layout), its slice
   // of the tile's bias, then the barriers full[S], empty[S], acc_full[2],
-  // acc_empty[2] and the TMEM slot.
+  // acc_empty[2], mma_done and the TMEM slot.
   static constexpr int kStage32 = F32S ? 32 * 32 * 4 : 0;
   static constexpr int kStage16 = 32 * 32 * 2;
   static constexpr int kStaging = kStages * kStage;
   static constexpr int kBias = kStaging + kLinEpiWarps * (kStage32 + kStage16);
   static constexpr int kBars = kBias + kLinEpiWarps * (BN / 2) * 4;
-  static constexpr int kTotal = kBars + (2 * kStages + 4) * 8 + 8 + 1024;  // + alignment
+  static constexpr int kTotal = kBars + (2 * kStages + 5) * 8 + 8 + 1024;  // + alignment
+  static_assert(kTotal <= 227 * 1024, "shared memory of one CTA");
 };
 
 // Tensor maps of one launch: the A operand's parts (up to two, lo and hi)
@@ -97,7 +109,7 @@ struct LinearArgs {
   int M, N;
   LinSeg seg[kLinMaxSegs];
   int nseg, nkb;
-  int tiles_n, tiles;
+  int tiles_n, tiles;  // column tiles; tiles (CTA pairs: 256-row tile pairs)
   int tma_f32, tma_bf16;  // write that output through TMA stores (see the launcher)
   int tma_planes;         // the same for the three planes (through the bf16 staging)
   int32_t* status;
@@ -206,10 +218,12 @@ __device__ __forceinline__ void store_chunk32(const LinOut& o, int row, int nb,
   }
 }
 
-template <int BN, int ACT, bool F32S>
+template <int BN, int ACT, bool F32S, bool PAIR>
 __global__ void __launch_bounds__(kLinThreads, 1)
     linear_bf16_kernel(const __grid_constant__ LinMaps maps, const __grid_constant__ LinearArgs args) {
-  using L = LinSmem<BN, F32S>;
+  using L = LinSmem<BN, F32S, PAIR>;
+  constexpr int CG = PAIR ? 2 : 1;
+  constexpr int kUnitM = CG * kLinBM;  // rows of the tile a CTA (pair) owns
   constexpr uint32_t kCols = 2 * BN;  // two f32 accumulators (a power of two >= 128)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -218,12 +232,17 @@ __global__ void __launch_bounds__(kLinThreads, 1)
   uint64_t* empty = full + L::kStages;
   uint64_t* acc_full = empty + L::kStages;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* mma_done = acc_empty + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(mma_done + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // CTA pairs: rank in the pair (0 = the MMA issuer), pair index and count
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int unit0 = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int unit_step = PAIR ? static_cast<int>(cluster_count_x()) : static_cast<int>(gridDim.x);
 
   if (warp == 1) {
-    tmem_alloc(tslot, kCols);
-    tmem_relinquish();
+    tmem_alloc<CG>(tslot, kCols);
+    tmem_relinquish<CG>();
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
@@ -232,12 +251,18 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kLinEpiWarps);  // one arrival per epilogue warp
+      // one arrival per epilogue warp (of both CTAs of a pair: the issuer's
+      // barrier gathers them)
+      mbar_init(&acc_empty[b], CG * kLinEpiWarps);
     }
+    mbar_init(mma_done, 1);
     mbar_init_fence();
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (PAIR)
+    cluster_sync();  // both CTAs' barriers exist before either signals the other's
+  else
+    __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tslot;
   const int nkb = args.nkb;
@@ -255,8 +280,9 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       // (a no-op without such a dependency).
       asm volatile("griddepcontrol.wait;" ::: "memory");
       int g = 0;
-      for (int t = blockIdx.x; t < args.tiles && !timed_out; t += gridDim.x) {
-        const int m0 = (t / args.tiles_n) * kLinBM, n0 = (t % args.tiles_n) * BN;
+      for (int t = unit0; t < args.tiles && !timed_out; t += unit_step) {
+        const int m0 = (t / args.tiles_n) * kUnitM + static_cast<int>(rank) * kLinBM;
+        const int n0 = (t % args.tiles_n) * BN;
         int si = 0, sb0 = 0;  // current segment and its first K block
         for (int kb = 0; kb < nkb; ++kb, ++g) {
           const int s = g % L::kStages;
@@ -270,22 +296,37 @@ __global__ void __launch_bounds__(kLinThreads, 1)
           const int kk = (kb - sb0) * kLinBK;
           uint8_t* sa = smem + s * L::kStage;
           uint8_t* sb = sa + L::kA;
-          mbar_arrive_expect_tx(&full[s], L::kStage);
-          tma_load_2d(sa, &maps.a[sg.a], &full[s], sg.a_k0 + kk, m0);
-          tma_load_2d(sb, &maps.w[sg.w], &full[s], sg.w_k0 + kk, n0);
+          if constexpr (PAIR) {
+            // every stage's bytes (both CTAs') are counted on the issuer's full
+            // barrier, which only the issuer's producer arms
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * L::kStage);
+            const uint32_t fb = map_to_cta(smem_u32(&full[s]), 0);
+            tma_load_2d_pair(sa, &maps.a[sg.a], fb, sg.a_k0 + kk, m0);
+            tma_load_2d_pair(sb, &maps.w[sg.w], fb, sg.w_k0 + kk,
+                             n0 + static_cast<int>(rank) * (BN / 2));
+          } else {
+            mbar_arrive_expect_tx(&full[s], L::kStage);
+            tma_load_2d(sa, &maps.a[sg.a], &full[s], sg.a_k0 + kk, m0);
+            tma_load_2d(sb, &maps.w[sg.w], &full[s], sg.w_k0 + kk, n0);
+          }
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // MMA issuer.
-      constexpr uint32_t idesc = idesc_bf16_f32(kLinBM, BN);
+    if (lane == 0 && rank == 0) {
+      // MMA issuer (of a pair: the even CTA).
+      constexpr uint32_t idesc = idesc_bf16_f32(kUnitM, BN);
       int g = 0, j = 0;
-      for (int t = blockIdx.x; t < args.tiles && !timed_out; t += gridDim.x, ++j) {
+      for (int t = unit0; t < args.tiles && !timed_out; t += unit_step, ++j) {
         const int b = j & 1;
-        if (j >= 2 && !mbar_wait_bounded(&acc_empty[b], ((j >> 1) - 1) & 1, kLinWaitLimit)) {
-          timed_out = true;
-          break;
+        if (j >= 2) {
+          const uint32_t par = ((j >> 1) - 1) & 1;
+          const bool ok = PAIR ? mbar_wait_cluster_bounded(&acc_empty[b], par, kLinWaitLimit)
+                               : mbar_wait_bounded(&acc_empty[b], par, kLinWaitLimit);
+          if (!ok) {
+            timed_out = true;
+            break;
+          }
         }
         tc_fence_after_sync();
         const uint32_t acc = tmem + static_cast<uint32_t>(b * BN);
@@ -300,12 +341,24 @@ __global__ void __launch_bounds__(kLinThreads, 1)
           const uint32_t sb = sa + L::kA;
 #pragma unroll
           for (int kk = 0; kk < kLinBK / 16; ++kk)
-            tc_mma_bf16(acc, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32), idesc,
-                        (kb | kk) != 0 ? 1u : 0u);
-          tc_commit(&empty[s]);  // the stage is free once these MMAs have read it
+            tc_mma_bf16<CG>(acc, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32), idesc,
+                            (kb | kk) != 0 ? 1u : 0u);
+          // the stage (both CTAs' halves) is free once these MMAs have read it
+          if constexpr (PAIR)
+            tc_commit_pair_both(&empty[s]);
+          else
+            tc_commit<CG>(&empty[s]);
         }
-        tc_commit(&acc_full[b]);  // the accumulator is final once all of them are done
+        // the accumulator (both CTAs' rows) is final once all of them are done
+        if constexpr (PAIR)
+          tc_commit_pair_both(&acc_full[b]);
+        else
+          tc_commit<CG>(&acc_full[b]);
       }
+      // every MMA issued has completed (and read the peer's shared memory)
+      // before this CTA or its peer can leave
+      tc_commit<CG>(mma_done);
+      if (!mbar_wait_bounded(mma_done, 0, kLinWaitLimit)) timed_out = true;
     }
   } else {
     // Epilogue warps 2..9: warp w reads TMEM lane quarter w % 4 (rows 32*(w%4) ..
@@ -345,9 +398,10 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     const bool any_direct =
         direct.y_f32 != nullptr || direct.y_bf16 != nullptr || direct.y_planes != nullptr;
     int j = 0;
-    for (int t = blockIdx.x; t < args.tiles; t += gridDim.x, ++j) {
+    for (int t = unit0; t < args.tiles; t += unit_step, ++j) {
       const int b = j & 1;
-      const int m0 = (t / args.tiles_n) * kLinBM, n0 = (t % args.tiles_n) * BN;
+      const int m0 = (t / args.tiles_n) * kUnitM + static_cast<int>(rank) * kLinBM;
+      const int n0 = (t % args.tiles_n) * BN;
       for (int c = lane; c < kColsPerWarp; c += 32) {
         const int n = n0 + c_begin + c;
         bias_s[c] = (args.bias != nullptr && n < args.N) ? __ldg(args.bias + n) : 0.f;
@@ -441,14 +495,23 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       }
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[b]);  // this warp has drained its share
+      if (lane == 0) {  // this warp has drained its share
+        if constexpr (PAIR)  // on the issuer's barrier, for both CTAs' warps
+          mbar_arrive_cluster(map_to_cta(smem_u32(&acc_empty[b]), 0));
+        else
+          mbar_arrive(&acc_empty[b]);
+      }
     }
     if (lane == 0) bulk_wait_all();  // every TMA store of this warp has completed
   }
   if (timed_out && args.status != nullptr) atomicOr(args.status, DLRM_FLAG_TIMEOUT);
   tc_fence_before_sync();
-  __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, kCols);
+  if constexpr (PAIR)
+    cluster_sync();  // neither CTA leaves while the other may still use its memory
+  else
+    __syncthreads();
+  tc_fence_after_sync();
+  if (warp == 1) tmem_dealloc<CG>(tmem, kCols);
 }
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ x, int64_t ldx, int64_t rows,
@@ -478,51 +541,70 @@ cudaError_t encode_bf16_operand(CUtensorMap* map, const void* base, int64_t cols
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int BN, int ACT, bool F32S>
+template <int BN, int ACT, bool F32S, bool PAIR>
 cudaError_t run_linear(const LinMaps& maps, LinearArgs args, int sms, cudaStream_t stream) {
-  auto* fn = &linear_bf16_kernel<BN, ACT, F32S>;
-  constexpr int smem = LinSmem<BN, F32S>::kTotal;
+  auto* fn = &linear_bf16_kernel<BN, ACT, F32S, PAIR>;
+  constexpr int smem = LinSmem<BN, F32S, PAIR>::kTotal;
+  constexpr int kUnitM = (PAIR ? 2 : 1) * kLinBM;
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   args.tiles_n = (args.N + BN - 1) / BN;
-  const int64_t tiles = static_cast<int64_t>((args.M + kLinBM - 1) / kLinBM) * args.tiles_n;
+  const int64_t tiles = static_cast<int64_t>((args.M + kUnitM - 1) / kUnitM) * args.tiles_n;
   if (tiles > INT32_MAX) return cudaErrorInvalidValue;
   args.tiles = static_cast<int>(tiles);
-  // one CTA per SM: the shared-memory ring and the 2 x BN TMEM columns size it
-  const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
   // programmatic dependent launch: the prologue (TMEM allocation, barriers)
   // overlaps the tail of the kernel before it on the stream
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kLinThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // one CTA per SM: the shared-memory ring and the 2 x BN TMEM columns size it
+  int64_t grid = std::min<int64_t>(tiles, sms);
+  if constexpr (PAIR) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+    // as many pairs as can be resident at once (a GPC with an odd number of
+    // free SMs leaves one idle)
+    int pairs = sms / 2;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    int fit = 0;
+    if (cudaOccupancyMaxActiveClusters(&fit, fn, &cfg) == cudaSuccess && fit > 0)
+      pairs = std::min(pairs, fit);
+    else
+      (void)cudaGetLastError();
+    grid = 2 * std::min<int64_t>(tiles, pairs);
+  }
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
   return cudaLaunchKernelEx(&cfg, fn, maps, args);
 }
 
-template <int BN, bool F32S>
+template <int BN, bool F32S, bool PAIR>
 cudaError_t run_linear_act(int act, const LinMaps& maps, const LinearArgs& args, int sms,
                            cudaStream_t stream) {
   switch (act) {
-    case DLRM_ACT_RELU: return run_linear<BN, DLRM_ACT_RELU, F32S>(maps, args, sms, stream);
-    case DLRM_ACT_SIGMOID: return run_linear<BN, DLRM_ACT_SIGMOID, F32S>(maps, args, sms, stream);
-    default: return run_linear<BN, DLRM_ACT_NONE, F32S>(maps, args, sms, stream);
+    case DLRM_ACT_RELU: return run_linear<BN, DLRM_ACT_RELU, F32S, PAIR>(maps, args, sms, stream);
+    case DLRM_ACT_SIGMOID:
+      return run_linear<BN, DLRM_ACT_SIGMOID, F32S, PAIR>(maps, args, sms, stream);
+    default: return run_linear<BN, DLRM_ACT_NONE, F32S, PAIR>(maps, args, sms, stream);
   }
 }
 
-// The instance with f32 output staging (and, at 256 columns, a 3-stage ring)
-// only when the f32 output goes out through TMA.
-template <int BN>
+// The instance with f32 output staging (and, at 256 columns on one CTA, a
+// 3-stage ring) only when the f32 output goes out through TMA.
+template <int BN, bool PAIR = false>
 cudaError_t run_linear_bn(int act, const LinMaps& maps, const LinearArgs& args, int sms,
                           cudaStream_t stream) {
-  return args.tma_f32 ? run_linear_act<BN, true>(act, maps, args, sms, stream)
-                      : run_linear_act<BN, false>(act, maps, args, sms, stream);
+  return args.tma_f32 ? run_linear_act<BN, true, PAIR>(act, maps, args, sms, stream)
+                      : run_linear_act<BN, false, PAIR>(act, maps, args, sms, stream);
 }
 
 // 2-D output map {N, M} with row pitch ld elements, box {32, 32}, written from a
@@ -560,6 +642,22 @@ int choose_bn(int64_t M, int64_t N, int sms) {
   return 64;
 }
 
+// 256-column tiles run on CTA pairs (256 x 256 per pair) when a tile has at
+// least 16 K blocks and the pairs' tile count still covers every SM. Measured
+// on B200 at B=65536: pairs win where the MMAs dominate a tile (f32
+// activations, 24 and 30 K blocks: 67.6 -> 63.5 us and 124.4 -> 108.6 us) and
+// lose where a tile's epilogue is as long as its MMAs (bf16 activations, 8
+// and 10 K blocks: 30.8 -> 32.9 us and 49.2 -> 53.3 us; 1 and 3 K blocks:
+// 34.9 -> 40.9 us, 59.4 -> 61.3 us): the issuer waits for both CTAs' loads and
+// both epilogues, the slower of two each time.
+bool choose_pair(int64_t M, int64_t N, int bn, int nkb, int sms) {
+#ifdef DLRM_LIN_NO_PAIR
+  return false;
+#endif
+  return bn == 256 && nkb >= 16 &&
+         ((M + 2 * kLinBM - 1) / (2 * kLinBM)) * ((N + 255) / 256) >= sms / 2;
+}
+
 bool is_aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 
@@ -580,6 +678,13 @@ int launch_layer(const APart* parts, int nparts, int a_planes, const uint16_t* w
   const int64_t K = parts[0].k + (nparts > 1 ? parts[1].k : 0);
   const int sms = sm_count_current();
   const int bn = choose_bn(M, N, sms);
+  // K blocks per tile: every (A plane, W plane) product sums all of K
+  int nkb_tile = 0;
+  for (int p = 0; p < nparts; ++p)
+    for (int i = 0; i < a_planes; ++i)
+      for (int j = 0; j < w_planes; ++j)
+        if (i + j < 3) nkb_tile += static_cast<int>((parts[p].k + kLinBK - 1) / kLinBK);
+  const bool pair = choose_pair(M, N, bn, nkb_tile, sms);
   LinMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   cudaError_t e = cudaSuccess;
@@ -588,7 +693,7 @@ int launch_layer(const APart* parts, int nparts, int a_planes, const uint16_t* w
       e = encode_bf16_operand(&maps.a[p * 3 + i], parts[p].base + i * parts[p].splane,
                               parts[p].k, M, parts[p].ld, kLinBM);
   for (int j = 0; j < w_planes && e == cudaSuccess; ++j)
-    e = encode_bf16_operand(&maps.w[j], w + j * splane_w, K, N, ldw, bn);
+    e = encode_bf16_operand(&maps.w[j], w + j * splane_w, K, N, ldw, pair ? bn / 2 : bn);
   if (e != cudaSuccess) return cuda_fail(e);
 
   LinearArgs args;
@@ -642,7 +747,10 @@ int launch_layer(const APart* parts, int nparts, int a_planes, const uint16_t* w
                       M, ldy_planes, CU_TENSOR_MAP_SWIZZLE_64B);
   if (e != cudaSuccess) return cuda_fail(e);
   switch (bn) {
-    case 256: e = run_linear_bn<256>(act, maps, args, sms, stream); break;
+    case 256:
+      e = pair ? run_linear_bn<256, true>(act, maps, args, sms, stream)
+               : run_linear_bn<256>(act, maps, args, sms, stream);
+      break;
     case 128: e = run_linear_bn<128>(act, maps, args, sms, stream); break;
     default: e = run_linear_bn<64>(act, maps, args, sms, stream); break;
   }

@@ -4,6 +4,12 @@
 // an mbarrier, tcgen05.ld of the f32 accumulator, and the 2-D TMA tile load
 // that stages the operands.
 //
+// CG is the CTA group of the tcgen05 operations: 1 (one CTA, M = 128 per
+// MMA) or 2 (a CTA pair of a cluster, M = 256 per MMA: the pair's even CTA
+// issues the MMA, each CTA holds half of A's rows and half of B's rows in its
+// shared memory at the same offsets, and each CTA's TMEM receives its own 128
+// rows of D). A kernel uses one CTA group for all of its tcgen05 operations.
+//
 // No multicast form of any TMA load is used.
 #pragma once
 
@@ -16,23 +22,40 @@ namespace dlrm {
 // ---- TMEM ---------------------------------------------------------------
 
 // Allocate `ncols` TMEM columns (a power of two >= 32) for this CTA; the base
-// address lands in *dst. Executed by one whole warp.
+// address lands in *dst. Executed by one whole warp (with CG = 2 by one warp
+// in each CTA of the pair, which get the same address).
+template <int CG = 1>
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                   smem_u32(dst)),
-               "r"(ncols)
-               : "memory");
+  if constexpr (CG == 2)
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+  else
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
 }
 
 // Give up the right to allocate more (lets other CTAs on the SM allocate).
+template <int CG = 1>
 __device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  if constexpr (CG == 2)
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  else
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
 }
 
-// Free what tmem_alloc returned. Executed by one whole warp.
+// Free what tmem_alloc returned. Executed by one whole warp (per CTA).
+template <int CG = 1>
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
+  if constexpr (CG == 2)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+  else
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
 }
 
 // Order tcgen05 operations across a thread synchronisation.
@@ -76,23 +99,52 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 // ---- MMA --------------------------------------------------------------
 
 // D[tmem] (+)= A[smem] * B[smem]^T for one K=16 step; accumulate = 0 starts
-// the accumulator from zero. Issued by a single thread.
+// the accumulator from zero. Issued by a single thread (with CG = 2, of the
+// pair's even CTA; the descriptors' addresses select the same tiles in both).
+template <int CG = 1>
 __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
+  if constexpr (CG == 2)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
-// One arrival on `bar` once every tcgen05 operation this thread issued so far
-// has completed.
+// One arrival on `bar` (this CTA's) once every tcgen05 operation this thread
+// issued so far has completed.
+template <int CG = 1>
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
+  if constexpr (CG == 2)
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+  else
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// CTA pair: one arrival on the mbarrier at `bar`'s offset in each CTA of the
+// pair (mask 0b11) once every tcgen05 operation this thread issued so far has
+// completed. This is the completion signal of the tensor cores, not a copy.
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(static_cast<uint16_t>(0x3))
+      : "memory");
 }
 
 // ---- TMEM -> registers ------------------------------------------------------
@@ -142,6 +194,19 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// CTA pair: the box of a 2-D tensor map at (x, y) lands at dst in this CTA's
+// shared memory; completion is counted in bytes on the mbarrier at the
+// shared::cluster address `bar_cluster`, which may be the peer CTA's (the even
+// CTA's barrier counts both CTAs' tiles of a stage). Not a multicast load.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
       : "memory");
 }
 

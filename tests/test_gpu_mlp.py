@@ -420,3 +420,53 @@ def test_dlrm_forward_f32_chain():
     wl, bl, actl = top.layers[-1]
     a_last32 = torch.from_numpy(f32_of(a_last).astype(np.float32)).to(DEV)
     _check_f32a(ctr, a_last32, wl, bl, actl, what="f32 CTR head")
+
+
+def _pair_rows(M, n, seed):
+    """Sampled rows of a layer run on CTA pairs: random ones plus each half of
+    the first and the last 256-row pair (the even and the odd CTA's rows)."""
+    rng = np.random.default_rng(seed)
+    last = (M - 1) // 256 * 256
+    edge = {0, 127, 128, 255, last, min(M - 1, last + 127), min(M - 1, last + 128), M - 1}
+    rows = np.unique(np.concatenate([rng.choice(M, n, replace=False),
+                                     np.array(sorted(edge))]))
+    return torch.from_numpy(rows).to(DEV)
+
+
+@pytest.mark.parametrize("M,N,k_lo,k_hi", [(65536, 512, 64, 528), (19999, 512, 1024, 0),
+                                           (20100, 200, 64, 960), (40000, 256, 512, 0)])
+@pytest.mark.parametrize("mode", ["bf16", "f32"])
+def test_linear_cta_pair_tiles(M, N, k_lo, k_hi, mode):
+    """Layers large enough for 256 x 256 tiles on CTA pairs (cta_group::2,
+    chosen for tiles of at least 16 K blocks: every case with f32
+    activations, the K = 1024 ones with bf16 activations; the others run the
+    one-CTA tiles at the same size): the DLRMv1 top layer 0 at B=65536 (split
+    A), a row count whose last pair has rows only in its even CTA, N below one
+    tile with split A, and a 256-wide layer; checked against the oracle on
+    sampled rows."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(M + N + k_lo + k_hi)
+    K = k_lo + k_hi
+    b = torch.empty(N, device=DEV).normal_(0, 0.5, generator=g)
+    w = _rand_bf16(g, N, K, K ** -0.5)
+    rows = _pair_rows(M, 64, M)
+    if mode == "bf16":
+        a_lo = _rand_bf16(g, M, k_lo)
+        a_hi = _rand_bf16(g, M, k_hi) if k_hi else None
+        y32, y16 = mlp.linear_bf16(a_lo, w, b, "relu", a_hi=a_hi, bf16=True)
+        torch.cuda.synchronize()
+        _check_layer(y32, None, a_lo, w, b, "relu", a_hi=a_hi, rows=rows,
+                     what=f"pair M={M} N={N} K={k_lo}+{k_hi}")
+        assert np.array_equal(_bits(y16), _bits(y32.to(torch.bfloat16)))
+    else:
+        a_lo = _rand_f32(g, M, k_lo)
+        a_hi = _rand_f32(g, M, k_hi) if k_hi else None
+        y32, planes = mlp.linear_f32a(mlp.split_bf16x3(a_lo), w, b, "relu",
+                                      a_hi=None if a_hi is None else mlp.split_bf16x3(a_hi),
+                                      planes=True)
+        torch.cuda.synchronize()
+        _check_f32a(y32, a_lo, w, b, "relu", a_hi=a_hi, rows=rows,
+                    what=f"f32a pair M={M} N={N} K={k_lo}+{k_hi}")
+        p = [(_bits(planes[i][rows]).astype(np.uint32) << 16).view(np.float32)
+             .astype(np.float64) for i in range(3)]
+        assert np.array_equal(p[0] + p[1] + p[2], y32[rows].double().cpu().numpy())
