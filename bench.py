@@ -119,6 +119,37 @@ def hold_stream(steps: int, per_step_ms: float = 0.1) -> None:
     torch.cuda._sleep(int(ms * 2.0e6))  # cycles at about 2 GHz
 
 
+def pcie_copy_rates(h2d_bytes: int, d2h_bytes: int, dev, reps: int = 20) -> dict:
+    """Plain copies of one step's sizes between page-locked host memory and
+    the device: host-to-device alone, device-to-host alone, and both at once
+    on two streams (GB/s over the bytes moved, device synchronised on both
+    sides of `reps` copies, after a warm-up). The last is the ceiling of a
+    pipeline that overlaps a step's inputs with another step's outputs."""
+    import torch
+    hin = torch.ones(h2d_bytes, dtype=torch.uint8).pin_memory()
+    hout = torch.ones(d2h_bytes, dtype=torch.uint8).pin_memory()
+    din = torch.empty(h2d_bytes, dtype=torch.uint8, device=dev)
+    dout = torch.empty(d2h_bytes, dtype=torch.uint8, device=dev)
+    s1, s2 = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+    def rate(h2d, d2h):
+        for n in (3, reps):
+            torch.cuda.synchronize(dev)
+            t0 = time.perf_counter()
+            for _ in range(n):
+                if h2d:
+                    with torch.cuda.stream(s1):
+                        din.copy_(hin, non_blocking=True)
+                if d2h:
+                    with torch.cuda.stream(s2):
+                        hout.copy_(dout, non_blocking=True)
+            torch.cuda.synchronize(dev)
+            dt = time.perf_counter() - t0
+        return reps * ((h2d_bytes if h2d else 0) + (d2h_bytes if d2h else 0)) / dt / 1e9
+
+    return {"h2d_gbs": rate(True, False), "d2h_gbs": rate(False, True),
+            "duplex_gbs": rate(True, True)}
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -647,13 +678,30 @@ def run_ours(args, w: syn.Workload):
             bo.copy_(off_t)
             bd.copy_(dense_t)
         pack_ms = (time.perf_counter() - p0) / 5 * 1e3
+        # host cost of one submit when none waits (the ring drained first)
+        sub_s, nsub = 0.0, 0
+        for r in range(10):
+            pipe.drain()
+            h0 = time.perf_counter()
+            for i in range(args.e2e_depth):
+                pipe.submit(*batches[(r + i) % E2E_BATCHES], outs[i])
+            sub_s += time.perf_counter() - h0
+            nsub += args.e2e_depth
+        pipe.drain()
+        submit_ms = sub_s / nsub * 1e3
+        link = pcie_copy_rates(pipe.h2d_bytes(), pipe.d2h_bytes(), dev)
+        step_bytes = pipe.h2d_bytes() + pipe.d2h_bytes()
+        link["e2e_gbs"] = step_bytes / (e2e_ms / args.steps / 1e3) / 1e9
+        link["frac_of_duplex"] = link["e2e_gbs"] / link["duplex_gbs"]
         e2e = {"value": lookups / (e2e_ms / 1e3), "unit": "lookups/s",
                "h2d_bytes_per_step": pipe.h2d_bytes(), "d2h_bytes_per_step": pipe.d2h_bytes(),
                "ms_per_step": e2e_ms / args.steps,
+               "host_submit_ms_per_batch": submit_ms,
                "unpacked": {"value": lookups / (loose_ms / 1e3), "ms_per_step": loose_ms / args.steps,
                             "note": "indices, offsets and dense in three separate pinned "
                                     "buffers: three host-to-device copies per step"},
                "host_pack_ms_per_batch": pack_ms,
+               "link": link,
                "path": f"dlrm_sparse_interact_host via ops.HostPipeline ({args.e2e_depth} streams): one "
                        f"pinned [indices|offsets|dense] block in, interaction rows out, {E2E_BATCHES} distinct "
                        f"batches in rotation; pooled written to device staging"}

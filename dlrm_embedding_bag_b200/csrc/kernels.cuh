@@ -207,18 +207,20 @@ __global__ void __launch_bounds__(kBlockThreads, kFusedMinBlocks)
   const int S_here = (B - b0 < S) ? static_cast<int>(B - b0) : S;
   const int64_t sample_floats = Lf.floats_per_sample();
 
-  // dense rows -> feature row 0 (16-byte loads when the pointer allows)
+  // dense rows -> feature row 0 with asynchronous copies (16-byte ones when the
+  // pointer allows), waited for before the dot phase: the copying warp starts
+  // its bags at once instead of a memory round trip later
   const bool dense_vec = ((D & 3) == 0) && ((reinterpret_cast<uintptr_t>(dense) & 15) == 0);
   for (int s = 0; s < S_here; ++s) {
     const float* src = dense + (b0 + s) * D;
     float* dst = feat + s * sample_floats;
     if (dense_vec) {
-      for (int c = threadIdx.x; c < (D >> 2); c += blockDim.x)
-        reinterpret_cast<float4*>(dst)[c] = __ldg(reinterpret_cast<const float4*>(src) + c);
+      for (int c = threadIdx.x; c < (D >> 2); c += blockDim.x) cp_async16(dst + 4 * c, src + 4 * c);
     } else {
-      for (int c = threadIdx.x; c < D; c += blockDim.x) dst[c] = __ldg(src + c);
+      for (int c = threadIdx.x; c < D; c += blockDim.x) cp_async4(dst + c, src + c);
     }
   }
+  cp_async_commit();
   zero_feature_padding(feat, Lf, D, S_here, threadIdx.x, blockDim.x);
 
   // bags (s, k) -> feature row k + 1; every group runs the same number of rounds
@@ -231,6 +233,7 @@ __global__ void __launch_bounds__(kBlockThreads, kFusedMinBlocks)
     const int flags = (oob ? DLRM_FLAG_INDEX_OOB : 0) | (bad_any ? DLRM_FLAG_OFFSETS : 0);
     if (flags) atomicOr(bp.status, flags);
   }
+  cp_async_wait<0>();  // this thread's dense copies have landed
   __syncthreads();
 
   const int64_t P = static_cast<int64_t>(Lf.F1) * (Lf.F1 - 1) / 2;
