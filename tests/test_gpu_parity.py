@@ -12,8 +12,8 @@ import torch
 
 import oracle
 from dlrm_embedding_bag_b200 import synthetic as syn
-from gpu_cases import (assert_bits_equal, check_inter, host_tables, oracle_stage,
-                       sampled_oracle)
+from gpu_cases import (assert_bits_equal, assert_dots_close, check_inter, host_tables,
+                       oracle_stage, sampled_oracle)
 
 pytestmark = pytest.mark.gpu
 
@@ -109,11 +109,39 @@ def test_full_size_sampled(ops, cfg):
     assert_bits_equal(fp[sel], ref_p, w.name + " fused pooled (sampled)")
     assert_bits_equal(pooled[sel], ref_p, w.name + " embbag_sum_multi (sampled)")
     check_inter(fi[sel], ref_i, bound, w.D, w.concat_dense, w.name + " fused (sampled)")
+    # the interaction alone on the full-size pooled vectors, same samples
+    inter_sep = ops.interact_lower_tri(dense, pooled)
+    torch.cuda.synchronize()
+    ref_plain = ref_i[:, w.D:] if w.concat_dense else ref_i
+    check_inter(inter_sep[sel], ref_plain, bound, w.D, False,
+                w.name + " interact_lower_tri (sampled)")
     # properties over every sample: finite, and both paths pool identically
-    assert torch.isfinite(fi).all()
+    assert torch.isfinite(fi).all() and torch.isfinite(inter_sep).all()
     assert torch.equal(fp.view(torch.int32), pooled.view(torch.int32))
-    del weights, fp, fi, pooled
+    del weights, fp, fi, pooled, inter_sep
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("B,F,D", [(20000, 8, 64), (12000, 8, 128), (70001, 26, 128),
+                                   (1500, 32, 64), (37, 59, 64), (3, 25, 128)])
+def test_interact_batches_and_table_counts(ops, B, F, D):
+    """The interaction alone on batches of many samples per block (a partial
+    last group), about one sample per block, F = 59 and a batch smaller than
+    one block; checked against the oracle on sampled rows, with the first and
+    the last sample always among them."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(B + F + D)
+    dense = torch.empty((B, D), device=DEV).normal_(0, 1, generator=g)
+    emb = torch.empty((B, F, D), device=DEV).normal_(0, 1, generator=g)
+    out = ops.interact_lower_tri(dense, emb)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(B)
+    samples = np.unique(np.concatenate([[0, B - 1], rng.integers(0, B, min(B, 96))]))
+    sel = torch.from_numpy(samples).to(DEV)
+    ref, _, bound = oracle.interact_lower_tri(dense[sel].cpu().numpy(), emb[sel].cpu().numpy(),
+                                              with_f64=True)
+    assert_dots_close(out[sel], ref, bound, f"interact B={B} F={F} D={D}")
+    assert torch.isfinite(out).all()
 
 
 # ------------------------------------------------------------------ shapes and edge cases
