@@ -587,6 +587,34 @@ def run_ours(args, w: syn.Workload):
         return sum(a.elapsed_time(b) for a, b in zip(ev_s, ev_e)) / args.steps
 
     extras = {}
+    if world == 1 and args.kernel != "interact":
+        # the device's random-row read rate for the stage's row size, without
+        # index loads: dlrm_probe_row_gather over a 4 GiB buffer (32 x L2), 8 M
+        # rows per call, cold and clean L2 before each call, best of 3
+        probe = torch.empty(4 << 30, dtype=torch.uint8, device=dev)
+        sink = torch.zeros(1, dtype=torch.int32, device=dev)
+        row_bytes = w.D * (2 if args.tables == "bf16" else 4)
+        ceiling = {}
+        for rb in sorted({128, 256, row_bytes} & {16, 32, 64, 128, 256, 512}):
+            best = None
+            for t in range(3):
+                flush.fill_(t)
+                sweep_sum.copy_(sweep.sum())
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                ops.probe_row_gather(probe, rb, 8 << 20, sink, seed=t)
+                e1.record()
+                torch.cuda.synchronize()
+                ms = e0.elapsed_time(e1)
+                best = ms if best is None else min(best, ms)
+            ceiling[str(rb)] = {"rows_per_s": (8 << 20) / (best / 1e3),
+                                "gbs": (8 << 20) * rb / (best / 1e3) / 1e9}
+        del probe
+        extras["row_read_ceiling"] = {
+            "row_bytes": ceiling, "stage_row_bytes": row_bytes,
+            "method": "dlrm_probe_row_gather: 8 M random rows of a 4 GiB buffer per call, row ids "
+                      "hashed in registers (no index loads), 128-bit loads without L1 allocation, "
+                      "cold clean L2, best of 3"}
     if world == 1:
         cc_ms = cold_clean(step)
         extras["cold_clean_l2"] = {
@@ -798,6 +826,18 @@ def run_ours(args, w: syn.Workload):
             line["hbm_check"]["frac"] = line["hbm_check"]["achieved_gbs"] / peak
             cc = line["hbm_check"]["cold_clean_l2"]
             cc["frac"] = cc["achieved_gbs"] / peak
+        if "row_read_ceiling" in line:
+            rc_ = line["row_read_ceiling"]
+            lim = rc_["row_bytes"].get(str(rc_["stage_row_bytes"]))
+            if lim is not None:
+                # lookups/s of the stage against rows/s of the probe at the same row size
+                rc_["stage_frac"] = line["value"] / lim["rows_per_s"]
+                if "hbm_check" in line:
+                    hc = line["hbm_check"]
+                    hc["row_ceiling_frac"] = hc["value"] / lim["rows_per_s"]
+                    hc["cold_clean_l2"]["row_ceiling_frac"] = (
+                        w.B * w.F * w.L / (hc["cold_clean_l2"]["ms_per_step"] / 1e3) /
+                        lim["rows_per_s"])
         if "cold_clean_l2" in line:
             cc = line["cold_clean_l2"]
             cc["achieved_gbs"] = per_launch / (cc["ms_per_step"] / 1e3) / 1e9

@@ -387,4 +387,17 @@ int dlrm_probe_bounded_wait(int64_t limit_cycles, int32_t* status_dev, dlrm_stre
   return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
 }
 
+int dlrm_probe_row_gather(const void* table, int64_t rows, int row_bytes, int64_t count,
+                          uint64_t seed, uint32_t* sink_dev, dlrm_stream_t stream) {
+  if (table == nullptr || sink_dev == nullptr) return DLRM_ERR_NULL;
+  if (row_bytes != 16 && row_bytes != 32 && row_bytes != 64 && row_bytes != 128 &&
+      row_bytes != 256 && row_bytes != 512)
+    return DLRM_ERR_SHAPE;
+  if (rows < 1 || count < 0) return DLRM_ERR_SHAPE;
+  if (!aligned(table, 16) || !aligned(sink_dev, 4)) return DLRM_ERR_ALIGN;
+  const cudaError_t e = dlrm::launch_probe_row_gather(
+      table, rows, row_bytes / 16, count, seed, sink_dev, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DLRM_OK : cuda_fail(e);
+}
+
 }  // extern "C"

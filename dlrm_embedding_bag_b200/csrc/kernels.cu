@@ -123,6 +123,52 @@ __global__ void probe_wait_kernel(long long limit, int32_t* status) {
   if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, limit)) atomicOr(status, DLRM_FLAG_TIMEOUT);
 }
 
+// The random-row read probe (dlrm_probe_row_gather). Row n of the request
+// stream is row splitmix64(seed + n) mod rows (Steele, Lea and Flood's
+// SplitMix64 finaliser; the high half of a 64 x 64-bit product maps it onto
+// [0, rows) without a division). A row of `chunks` 16-byte chunks is read by
+// `chunks` consecutive lanes, 32 / chunks rows per warp at a time, eight such
+// slots in flight before any value is used.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  x += 0x9E3779B97F4A7C15ull;
+  x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
+  x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
+  return x ^ (x >> 31);
+}
+
+__global__ void __launch_bounds__(kBlockThreads, 4)
+    row_gather_probe_kernel(const uint4* __restrict__ table, int64_t rows, int lchunks,
+                            int64_t count, uint64_t seed, uint32_t* __restrict__ sink) {
+  constexpr int U = 8;
+  const int chunks = 1 << lchunks;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane >> lchunks, c = lane & (chunks - 1);
+  const int per_warp = 32 >> lchunks;  // rows per warp slot
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t span = static_cast<int64_t>(per_warp) * U;
+  uint32_t acc = 0;
+  for (int64_t base = warp * span; base < count; base += nwarps * span) {
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t n = base + static_cast<int64_t>(u) * per_warp + sub;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (n < count) {
+        const uint64_t row = __umul64hi(splitmix64(seed + static_cast<uint64_t>(n)),
+                                        static_cast<uint64_t>(rows));
+        const float4 f = ldg_row_f32x4(reinterpret_cast<const float*>(
+            table + static_cast<int64_t>(row) * chunks + c));
+        v[u] = make_uint4(__float_as_uint(f.x), __float_as_uint(f.y), __float_as_uint(f.z),
+                          __float_as_uint(f.w));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) acc ^= v[u].x ^ v[u].y ^ v[u].z ^ v[u].w;
+  }
+  if (acc == 0x2545F491u) atomicXor(sink, acc);
+}
+
 // Below 2^24 it runs pair_from_flat_small, the decoder dots_from_smem runs on
 // the tile index in the interaction and fused kernels; from 2^24 on, the
 // 64-bit pair_from_flat.
@@ -382,6 +428,15 @@ cudaError_t launch_interact(const float* dense, const float* emb, int B, int F, 
 
 cudaError_t launch_probe_wait(int64_t limit, int32_t* status, cudaStream_t stream) {
   probe_wait_kernel<<<1, 32, 0, stream>>>(static_cast<long long>(limit), status);
+  return counted(cudaGetLastError());
+}
+
+cudaError_t launch_probe_row_gather(const void* table, int64_t rows, int chunks, int64_t count,
+                                    uint64_t seed, uint32_t* sink, cudaStream_t stream) {
+  if (count == 0) return cudaSuccess;
+  const int lchunks = log2_floor(chunks);
+  row_gather_probe_kernel<<<static_cast<unsigned>(4 * sm_count()), kBlockThreads, 0, stream>>>(
+      static_cast<const uint4*>(table), rows, lchunks, count, seed, sink);
   return counted(cudaGetLastError());
 }
 

@@ -103,6 +103,8 @@ cudaError_t launch_pair_decode(int64_t p0, int64_t count, int32_t* i_out, int32_
 int64_t launch_count();
 
 cudaError_t launch_probe_wait(int64_t limit, int32_t* status, cudaStream_t stream);
+cudaError_t launch_probe_row_gather(const void* table, int64_t rows, int chunks, int64_t count,
+                                    uint64_t seed, uint32_t* sink, cudaStream_t stream);
 // Counts one kernel launch of this library (dlrm_launch_count).
 void note_launch();
 

@@ -62,6 +62,7 @@ SIGNATURES = {
     "dlrm_last_cuda_error": (_I, []),
     "dlrm_launch_count": (_I64, []),
     "dlrm_probe_bounded_wait": (_I, [_I64, _P, _P]),
+    "dlrm_probe_row_gather": (_I, [_P, _I64, _I, _I64, ctypes.c_uint64, _P, _P]),
     # include/dlrm_mlp.h
     "dlrm_linear_bf16": (_I, [_P, _I64, _I64, _P, _I64, _I64, _P, _I64, _P, _I64, _I64, _I, _P,
                               _I64, _P, _I64, _P, _P]),
@@ -600,6 +601,21 @@ def status_from_flags(flags: int) -> int:
 def launch_count() -> int:
     """Kernels the library has launched in this process."""
     return int(_lib.dlrm_launch_count())
+
+
+def probe_row_gather(table: torch.Tensor, row_bytes: int, count: int, sink: torch.Tensor,
+                     seed: int = 0) -> None:
+    """Read ``count`` random rows of ``row_bytes`` bytes from ``table`` (any
+    contiguous device tensor, taken as ``numel * itemsize // row_bytes`` rows),
+    the device's random-row read ceiling without index loads (see the header);
+    ``sink`` is one int32 on the device. Time it with events on the current
+    stream."""
+    if not table.is_cuda or not table.is_contiguous():
+        raise ValueError("table must be a contiguous device tensor")
+    rows = table.numel() * table.element_size() // row_bytes
+    _check(_lib.dlrm_probe_row_gather(table.data_ptr(), rows, row_bytes, count, seed,
+                                      _dev(sink, "sink", torch.int32), _stream()),
+           "dlrm_probe_row_gather")
 
 
 def probe_bounded_wait(status: torch.Tensor, limit_cycles: int = 1_000_000) -> None:

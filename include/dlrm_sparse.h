@@ -356,6 +356,28 @@ DLRM_API int64_t dlrm_launch_count(void);
 DLRM_API int dlrm_probe_bounded_wait(int64_t limit_cycles, int32_t* status_dev,
                                      dlrm_stream_t stream);
 
+/*
+ * dlrm_probe_row_gather -- measurement aid: the device's rate of random row
+ * reads for rows of `row_bytes` bytes, without the stage's offset and index
+ * loads (the roofline that the gather's row reads meet). No counterpart on the
+ * pages. `count` rows of `table` are read, row n (0 <= n < count) at row id
+ * splitmix64(seed + n) mod rows, each row by row_bytes/16 lanes with one
+ * 128-bit load per lane that does not allocate in L1, eight rows in flight per
+ * lane. The XOR of every word read is folded into one value per thread, which
+ * is written to *sink_dev only if it equals a fixed constant (so the reads
+ * cannot be left out; the sink's content is otherwise unspecified). Time the
+ * call with events on `stream` to get rows/s.
+ *   table    : dev, `rows` rows of `row_bytes` bytes, 16-byte aligned; read only.
+ *   rows     : >= 1.
+ *   row_bytes: 16, 32, 64, 128, 256 or 512 (DLRM_ERR_SHAPE otherwise).
+ *   count    : >= 0 rows to read.
+ *   sink_dev : dev uint32, 4-byte aligned, required.
+ * Asynchronous on `stream`.
+ */
+DLRM_API int dlrm_probe_row_gather(const void* table, int64_t rows, int row_bytes,
+                                   int64_t count, uint64_t seed, uint32_t* sink_dev,
+                                   dlrm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -36,7 +36,7 @@ def test_header_declares_the_stage_entry_points():
     names = _declared()
     assert {"embbag_sum_multi", "interact_lower_tri", "dlrm_sparse_interact"} <= names
     assert {"dlrm_linear_bf16", "dlrm_f32_to_bf16"} <= names
-    assert len(names) == 21
+    assert len(names) == 22
 
 
 def test_library_exports_every_declared_symbol(ops):
@@ -66,7 +66,8 @@ def _declarations():
 def _ctype_of(decl):
     if "*" in decl or decl == "dlrm_stream_t":
         return ctypes.c_void_p
-    return {"int": ctypes.c_int, "int64_t": ctypes.c_int64, "int32_t": ctypes.c_int32}[decl]
+    return {"int": ctypes.c_int, "int64_t": ctypes.c_int64, "int32_t": ctypes.c_int32,
+            "uint64_t": ctypes.c_uint64}[decl]
 
 
 def test_binding_signatures_match_the_headers(ops):
@@ -242,6 +243,15 @@ def test_probe_host_checks(ops):
     lib = ops._lib
     assert lib.dlrm_probe_bounded_wait(1000, None, None) == -1
     assert lib.dlrm_probe_bounded_wait(1000, 0x10002, None) == -3
+    T, S = 0x10000, 0x20000  # never dereferenced: every call fails its host checks
+    assert lib.dlrm_probe_row_gather(None, 10, 256, 5, 0, S, None) == -1
+    assert lib.dlrm_probe_row_gather(T, 10, 256, 5, 0, None, None) == -1
+    for rb in (0, 8, 48, 100, 1024):
+        assert lib.dlrm_probe_row_gather(T, 10, rb, 5, 0, S, None) == -2, rb
+    assert lib.dlrm_probe_row_gather(T, 0, 256, 5, 0, S, None) == -2
+    assert lib.dlrm_probe_row_gather(T, 10, 256, -1, 0, S, None) == -2
+    assert lib.dlrm_probe_row_gather(T + 8, 10, 256, 5, 0, S, None) == -3
+    assert lib.dlrm_probe_row_gather(T, 10, 256, 5, 0, S + 2, None) == -3
 
 
 def test_header_compiles_as_c_and_matches_the_binding(ops, tmp_path):

@@ -555,3 +555,16 @@ def test_prepared_call_matches_plain_call(ops):
     torch.cuda.synchronize()
     assert torch.equal(p1.view(torch.int32), p2.view(torch.int32))
     assert torch.equal(i1.view(torch.int32), i2.view(torch.int32))
+
+
+@pytest.mark.parametrize("row_bytes", [16, 128, 256, 512])
+def test_probe_row_gather_runs(ops, row_bytes):
+    """The random-row read probe: one launch, no error, and on a table of
+    zeros the folded value is zero, so the sink keeps its content."""
+    table = torch.zeros(1 << 20, dtype=torch.float32, device=DEV)  # 4 MB
+    sink = torch.full((1,), 12345, dtype=torch.int32, device=DEV)
+    n0 = ops.launch_count()
+    ops.probe_row_gather(table, row_bytes, 100_000, sink, seed=7)
+    torch.cuda.synchronize()
+    assert ops.launch_count() == n0 + 1
+    assert int(sink.item()) == 12345
