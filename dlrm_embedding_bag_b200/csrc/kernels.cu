@@ -53,8 +53,9 @@ __device__ __forceinline__ void stage_interact_group(float* buf, const FeatLayou
   }
 }
 
-// Blocks of the interaction kernel per SM (its register budget), and the
-// unrolling of the general dot routine's column loop.
+// Blocks of the interaction kernel per SM (its register budget: 128 registers
+// at 128-thread blocks; eight blocks would spill), and the unrolling of the
+// general dot routine's column loop.
 #ifndef DLRM_INTERACT_MIN_BLOCKS
 #define DLRM_INTERACT_MIN_BLOCKS 4
 #endif
@@ -136,7 +137,9 @@ __device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
   return x ^ (x >> 31);
 }
 
-__global__ void __launch_bounds__(kBlockThreads, 4)
+constexpr int kProbeThreads = 256;
+
+__global__ void __launch_bounds__(kProbeThreads, 4)
     row_gather_probe_kernel(const uint4* __restrict__ table, int64_t rows, int lchunks,
                             int64_t count, uint64_t seed, uint32_t* __restrict__ sink) {
   constexpr int U = 8;
@@ -364,7 +367,8 @@ cudaError_t launch_fused(const GatherPlan& g, const float* dense, float* pooled_
 // Samples per group S and lanes per tile 2^lq for the interaction kernel.
 // Measured on B200 (B=2048, F=32, D=64 and B=65536, F=26, D=128), four lanes
 // per tile beat one or two (shorter serial chains per thread), and the best
-// group is the largest that still gives one task per thread: S*nT*4 <= 256.
+// group is the largest that still gives one task per thread: S*nT*4 <= the
+// block's threads (at least one sample).
 // S is further capped by the shared-memory budget of two buffers.
 static void choose_interact_shape(int F, int D, int B, int64_t smem_budget, int& S, int& lq) {
   const FeatLayout Lf = FeatLayout::make(F, D);
@@ -395,9 +399,9 @@ static cudaError_t run_interact(const float* dense, const float* emb, int B, int
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  // threads: the group's tasks rounded up to whole warps, at most 256 (B=65536,
-  // F=26, D=128: 224 threads for 2 x 112 tasks, 447 -> 398 us on B200; at
-  // B=2048, F=32, D=64, 192 threads for 180 tasks time the same as 256)
+  // threads: the group's tasks rounded up to whole warps, at most a full block
+  // (with 256-thread blocks this took B=65536, F=26, D=128 from 447 to 398 us
+  // on B200: 224 threads for 2 x 112 tasks)
   const int threads = std::min<int>(kBlockThreads, (S * (Lf.nT << lq) + 31) / 32 * 32);
   int per_sm = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
@@ -435,7 +439,7 @@ cudaError_t launch_probe_row_gather(const void* table, int64_t rows, int chunks,
                                     uint64_t seed, uint32_t* sink, cudaStream_t stream) {
   if (count == 0) return cudaSuccess;
   const int lchunks = log2_floor(chunks);
-  row_gather_probe_kernel<<<static_cast<unsigned>(4 * sm_count()), kBlockThreads, 0, stream>>>(
+  row_gather_probe_kernel<<<static_cast<unsigned>(4 * sm_count()), kProbeThreads, 0, stream>>>(
       static_cast<const uint4*>(table), rows, lchunks, count, seed, sink);
   return counted(cudaGetLastError());
 }

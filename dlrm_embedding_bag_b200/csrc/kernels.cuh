@@ -13,7 +13,7 @@ namespace dlrm {
 #define DLRM_ROWS_IN_FLIGHT 8
 #endif
 #ifndef DLRM_GATHER_MIN_BLOCKS
-#define DLRM_GATHER_MIN_BLOCKS 4
+#define DLRM_GATHER_MIN_BLOCKS 8
 #endif
 constexpr int kRowsInFlight = DLRM_ROWS_IN_FLIGHT;
 constexpr int kGatherMinBlocks = DLRM_GATHER_MIN_BLOCKS;

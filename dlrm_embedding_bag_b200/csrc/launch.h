@@ -11,7 +11,7 @@ namespace dlrm {
 
 // Blocks of the fused kernel that the register allocation keeps resident per SM.
 #ifndef DLRM_FUSED_MIN_BLOCKS
-#define DLRM_FUSED_MIN_BLOCKS 4
+#define DLRM_FUSED_MIN_BLOCKS 8
 #endif
 
 // Which row loader a launch uses.
