@@ -763,6 +763,12 @@ def run_ours(args, w: syn.Workload):
         pipe.drain()
         submit_ms = sub_s / nsub * 1e3
         assert link is not None
+        # again now that the process has moved a few GB through the link: its
+        # first copies can run at under half the rate (seen on one B200 machine at
+        # 22 GB/s host-to-device at the start); the best of both is the ceiling
+        later = pcie_copy_rates(pipe.h2d_bytes(), pipe.d2h_bytes(), dev)
+        link = {k: (max(link[k], later[k]) if k.endswith("_gbs") else link[k]) for k in link}
+        link["method"] += "; taken at the start of the run and after the e2e loops, best of both"
         step_bytes = pipe.h2d_bytes() + pipe.d2h_bytes()
         link["e2e_gbs"] = step_bytes / (e2e_ms / args.steps / 1e3) / 1e9
         link["frac_of_duplex"] = link["e2e_gbs"] / link["duplex_gbs"]
