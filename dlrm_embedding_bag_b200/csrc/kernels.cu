@@ -232,12 +232,14 @@ int64_t interact_smem_per_sample(int F, int D) {
 
 // Samples per block of the fused kernel. A block's S*F bags go to its lane
 // groups in rounds; measured on B200, blocks do best with at least two bags per
-// lane group and little idle time in the last round (B=2048, F=32, D=64: S=1;
-// F=8: S=4; B=65536, F=26, D=128: S=2, 12 % faster than S=1), while blocks too
-// large for four to share an SM lose more than they gain. So: the smallest S
-// up to 4 with >= 2 bags per group, >= 90 % of the rounds' slots used and four
-// blocks' shared memory fitting an SM; else the S with the best product of slot
-// use and resident blocks.
+// lane group and little idle time in the last round, while blocks too large for
+// DLRM_FUSED_MIN_BLOCKS of them to share an SM lose more than they gain (with
+// 256-thread blocks, four per SM: B=65536, F=26, D=128 ran 12 % faster at S=2
+// than at S=1). So: the smallest S up to 4 with >= 2 bags per group, >= 90 % of
+// the rounds' slots used and DLRM_FUSED_MIN_BLOCKS blocks' shared memory
+// fitting an SM; else the S with the best product of slot use and resident
+// blocks. With 128-thread blocks: S = 1 at B=2048, F=32, D=64 and at B=65536,
+// F=26, D=128; S = 2 at F=8, D=64.
 #ifndef DLRM_FUSED_MAX_S
 #define DLRM_FUSED_MAX_S 4
 #endif
