@@ -149,23 +149,8 @@ __device__ __forceinline__ void tc_commit_pair_both(uint64_t* bar) {
 
 // ---- TMEM -> registers ------------------------------------------------------
 
-// 16 consecutive 32-bit columns of the warp's 32 TMEM lanes (lane i of the
+// 32 consecutive 32-bit columns of the warp's 32 TMEM lanes (lane i of the
 // warp gets row i of its quarter): taddr = base + (32*(warp%4) << 16) + col.
-__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// 32 consecutive 32-bit columns of the warp's 32 TMEM lanes (as above).
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
   asm volatile(
