@@ -238,28 +238,6 @@ __device__ __forceinline__ void dots_fixed(const float* feat, const FeatLayout& 
   }
 }
 
-// dots_fixed for the runtime lq (2, 3 or 4: the shapes the launches choose
-// for these row lengths; smaller lq goes to dots_from_smem).
-template <int D4, int RS>
-__device__ __forceinline__ void dots_fixed_lq(const float* feat, const FeatLayout& Lf,
-                                              const uint16_t* tiles, int S_here, int lq,
-                                              float* __restrict__ out, int64_t b0,
-                                              int64_t row_stride, int64_t col0, int tid,
-                                              int nthreads) {
-  switch (lq) {
-    case 2:
-      dots_fixed<D4, RS, 2>(feat, Lf, tiles, S_here, out, b0, row_stride, col0, tid, nthreads);
-      break;
-    case 3:
-      dots_fixed<D4, RS, 3>(feat, Lf, tiles, S_here, out, b0, row_stride, col0, tid, nthreads);
-      break;
-    default:
-      dots_fixed<D4, RS, 4>(feat, Lf, tiles, S_here, out, b0, row_stride, col0, tid, nthreads);
-      break;
-  }
-}
-
-
 // Bytes of the tile table decode_tiles writes (a multiple of 16).
 __host__ __device__ inline int64_t tile_table_bytes(int nT) { return (2 * nT + 15) / 16 * 16; }
 
@@ -272,26 +250,31 @@ __device__ __forceinline__ uint16_t* tile_table(void* smem_base, int nT) {
                                      tile_table_bytes(nT));
 }
 
-// The dot phase of the interaction kernel for any row shape: the
-// compile-time routine for the common row lengths (D = 64 and 128 with the
-// padded layout) and lq >= 2, dots_from_smem for the rest. tiles is the table
-// decode_tiles wrote (used by the fixed routine), or null when the block's
-// shared memory has no room for it. (Measured on B200: in the interaction
-// kernel the fixed routine took c3 from 24.6 to 23.0 us; in the fused kernel,
-// whose dot phase runs beside other blocks' gathers, it cost 2.5 us, so the
-// fused kernel keeps dots_from_smem.)
-template <int UNROLL = 1>
+// The dot phase of the interaction kernel: for the padded row length DP of
+// the kernel instance (68 floats: D = 64; 132: D = 128) and four lanes per
+// tile (the interaction launch's choice for those rows), the compile-time
+// routine; dots_from_smem for the rest. Each instance holds only its own
+// routine: with every fixed routine in every instance, instruction fetch was
+// the kernel's largest stall. tiles is the table decode_tiles wrote (used by
+// the fixed routine), or null when the block's shared memory has no room for
+// it. (Measured on B200: in the interaction kernel the fixed routine took c3
+// from 24.6 to 23.0 us; in the fused kernel, whose dot phase runs beside other
+// blocks' gathers, it cost 2.5 us, so the fused kernel keeps dots_from_smem.)
+template <int UNROLL, int DP>
 __device__ __forceinline__ void dots_any(const float* feat, const FeatLayout& Lf,
                                          const uint16_t* tiles, int S_here, int lq,
                                          float* __restrict__ out, int64_t b0, int64_t row_stride,
                                          int64_t col0, int tid, int nthreads) {
-  if (tiles != nullptr && lq >= 2 && Lf.D4 == 16 && Lf.Dp == 68) {
-    dots_fixed_lq<16, 17>(feat, Lf, tiles, S_here, lq, out, b0, row_stride, col0, tid, nthreads);
-    return;
-  }
-  if (tiles != nullptr && lq >= 2 && Lf.D4 == 32 && Lf.Dp == 132) {
-    dots_fixed_lq<32, 33>(feat, Lf, tiles, S_here, lq, out, b0, row_stride, col0, tid, nthreads);
-    return;
+  if constexpr (DP == 68) {
+    if (tiles != nullptr && lq == 2 && Lf.D4 == 16 && Lf.Dp == 68) {
+      dots_fixed<16, 17, 2>(feat, Lf, tiles, S_here, out, b0, row_stride, col0, tid, nthreads);
+      return;
+    }
+  } else if constexpr (DP == 132) {
+    if (tiles != nullptr && lq == 2 && Lf.D4 == 32 && Lf.Dp == 132) {
+      dots_fixed<32, 33, 2>(feat, Lf, tiles, S_here, out, b0, row_stride, col0, tid, nthreads);
+      return;
+    }
   }
   dots_from_smem<UNROLL>(feat, Lf, S_here, lq, out, b0, row_stride, col0, tid, nthreads);
 }

@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kBlockThreads, DLRM_INTERACT_MIN_BLOCKS)
       cp_async_commit();
       cp_async_wait<0>();
       __syncthreads();
-      dots_any<DLRM_INTERACT_UNROLL>(feat, Lf, tiles, samples(g), lq, out, g * S, P, 0,
+      dots_any<DLRM_INTERACT_UNROLL, DP>(feat, Lf, tiles, samples(g), lq, out, g * S, P, 0,
                                      threadIdx.x, blockDim.x);
       __syncthreads();
     }
@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(kBlockThreads, DLRM_INTERACT_MIN_BLOCKS)
       // bounded (about a second): the copies cannot stall, this only guards
       // the GPU against a broken barrier sequence
       mbar_wait_bounded(&bars[it & 1], (it >> 1) & 1, 2000000000LL);
-      dots_any<DLRM_INTERACT_UNROLL>(feat + (it & 1) * bstride, Lf, tiles, samples(g), lq, out,
+      dots_any<DLRM_INTERACT_UNROLL, DP>(feat + (it & 1) * bstride, Lf, tiles, samples(g), lq, out,
                                      g * S, P, 0, threadIdx.x, blockDim.x);
       __syncthreads();  // buffer it & 1 is refilled in the next iteration
     }
@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kBlockThreads, DLRM_INTERACT_MIN_BLOCKS)
     cp_async_commit();
     cp_async_wait<1>();  // group g has landed (only the copy of group gn may be pending)
     __syncthreads();
-    dots_any<DLRM_INTERACT_UNROLL>(feat + (it & 1) * bstride, Lf, tiles, samples(g), lq, out,
+    dots_any<DLRM_INTERACT_UNROLL, DP>(feat + (it & 1) * bstride, Lf, tiles, samples(g), lq, out,
                                    g * S, P, 0, threadIdx.x, blockDim.x);
     __syncthreads();  // buffer it&1 is refilled in the next iteration
   }
