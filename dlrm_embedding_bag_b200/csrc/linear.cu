@@ -321,8 +321,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         const int b = j & 1;
         if (j >= 2) {
           const uint32_t par = ((j >> 1) - 1) & 1;
-          const bool ok = PAIR ? mbar_wait_cluster_bounded(&acc_empty[b], par, kLinWaitLimit)
-                               : mbar_wait_bounded(&acc_empty[b], par, kLinWaitLimit);
+          const bool ok = mbar_wait_bounded(&acc_empty[b], par, kLinWaitLimit);
           if (!ok) {
             timed_out = true;
             break;
@@ -497,7 +496,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       __syncwarp();
       if (lane == 0) {  // this warp has drained its share
         if constexpr (PAIR)  // on the issuer's barrier, for both CTAs' warps
-          mbar_arrive_cluster(map_to_cta(smem_u32(&acc_empty[b]), 0));
+          mbar_arrive_remote(map_to_cta(smem_u32(&acc_empty[b]), 0));
         else
           mbar_arrive(&acc_empty[b]);
       }
@@ -642,19 +641,16 @@ int choose_bn(int64_t M, int64_t N, int sms) {
   return 64;
 }
 
-// 256-column tiles run on CTA pairs (256 x 256 per pair) when a tile has at
-// least 16 K blocks and the pairs' tile count still covers every SM. Measured
-// on B200 at B=65536: pairs win where the MMAs dominate a tile (f32
-// activations, 24 and 30 K blocks: 67.6 -> 63.5 us and 124.4 -> 108.6 us) and
-// lose where a tile's epilogue is as long as its MMAs (bf16 activations, 8
-// and 10 K blocks: 30.8 -> 32.9 us and 49.2 -> 53.3 us; 1 and 3 K blocks:
-// 34.9 -> 40.9 us, 59.4 -> 61.3 us): the issuer waits for both CTAs' loads and
-// both epilogues, the slower of two each time.
-bool choose_pair(int64_t M, int64_t N, int bn, int nkb, int sms) {
+// 256-column tiles run on CTA pairs (256 x 256 per pair) when the pairs' tile
+// count still covers every SM. Measured on B200 at B=65536 against one CTA per
+// tile: f32 activations, 3, 24 and 30 K blocks per tile, 58.4 -> 54.3 us,
+// 67.6 -> 63.0 us and 124.4 -> 106.6 us; bf16 activations, 1, 8 and 10 K
+// blocks, 35.7 -> 33.8 us, 31.7 -> 29.7 us and 50.1 -> 45.0 us.
+bool choose_pair(int64_t M, int64_t N, int bn, int sms) {
 #ifdef DLRM_LIN_NO_PAIR
   return false;
 #endif
-  return bn == 256 && nkb >= 16 &&
+  return bn == 256 &&
          ((M + 2 * kLinBM - 1) / (2 * kLinBM)) * ((N + 255) / 256) >= sms / 2;
 }
 
@@ -678,13 +674,7 @@ int launch_layer(const APart* parts, int nparts, int a_planes, const uint16_t* w
   const int64_t K = parts[0].k + (nparts > 1 ? parts[1].k : 0);
   const int sms = sm_count_current();
   const int bn = choose_bn(M, N, sms);
-  // K blocks per tile: every (A plane, W plane) product sums all of K
-  int nkb_tile = 0;
-  for (int p = 0; p < nparts; ++p)
-    for (int i = 0; i < a_planes; ++i)
-      for (int j = 0; j < w_planes; ++j)
-        if (i + j < 3) nkb_tile += static_cast<int>((parts[p].k + kLinBK - 1) / kLinBK);
-  const bool pair = choose_pair(M, N, bn, nkb_tile, sms);
+  const bool pair = choose_pair(M, N, bn, sms);
   LinMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   cudaError_t e = cudaSuccess;

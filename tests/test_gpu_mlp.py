@@ -438,12 +438,10 @@ def _pair_rows(M, n, seed):
 @pytest.mark.parametrize("mode", ["bf16", "f32"])
 def test_linear_cta_pair_tiles(M, N, k_lo, k_hi, mode):
     """Layers large enough for 256 x 256 tiles on CTA pairs (cta_group::2,
-    chosen for tiles of at least 16 K blocks: every case with f32
-    activations, the K = 1024 ones with bf16 activations; the others run the
-    one-CTA tiles at the same size): the DLRMv1 top layer 0 at B=65536 (split
-    A), a row count whose last pair has rows only in its even CTA, N below one
-    tile with split A, and a 256-wide layer; checked against the oracle on
-    sampled rows."""
+    every case here, in both activation modes): the DLRMv1 top layer 0 at
+    B=65536 (split A), a row count whose last pair has rows only in its even
+    CTA, N below one tile with split A, and a 256-wide layer; checked against
+    the oracle on sampled rows."""
     g = torch.Generator(device=DEV)
     g.manual_seed(M + N + k_lo + k_hi)
     K = k_lo + k_hi
