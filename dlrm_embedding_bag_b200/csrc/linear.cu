@@ -66,8 +66,9 @@ struct LinSmem {
   static constexpr int kStage = kA + kB;
   // After the ring: each epilogue warp's output staging (a 32 x 32 f32 tile in
   // the 128-byte swizzled layout when F32S -- the f32 output goes out through
-  // TMA --, then a 32 x 32 bf16 tile in the 64-byte swizzled layout), its slice
-  // of the tile's bias, then the barriers full[S], empty[S], acc_full[2],
+  // TMA --, then a 32 x 32 bf16 tile in the 64-byte swizzled layout), the
+  // bias region (4 BN floats: the whole bias vector, or each warp's slice of
+  // the tile's), then the barriers full[S], empty[S], acc_full[2],
   // acc_empty[2], mma_done and the TMEM slot.
   static constexpr int kStage32 = F32S ? 32 * 32 * 4 : 0;
   static constexpr int kStage16 = 32 * 32 * 2;
@@ -362,7 +363,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
   } else {
     // Epilogue warps 2..9: warp w reads TMEM lane quarter w % 4 (rows 32*(w%4) ..
     // +31 of a tile) and column half (w - 2) / 4 of the accumulator, 32 columns
-    // per tcgen05.ld; its slice of the bias is staged in shared memory per tile.
+    // per tcgen05.ld; the bias is read from shared memory (staged below).
     // A 32 x 32 result block goes out either through the warp's staging tiles
     // and one TMA store per output (lane r writes row r; 16-byte chunk q of a row
     // sits at chunk q ^ (r & 7) of a 128-byte f32 row and q ^ ((r >> 1) & 3) of a
@@ -396,16 +397,33 @@ __global__ void __launch_bounds__(kLinThreads, 1)
     direct.N = args.N;
     const bool any_direct =
         direct.y_f32 != nullptr || direct.y_bf16 != nullptr || direct.y_planes != nullptr;
+    // A bias vector that fits the bias region whole (N <= 4 BN, every layer of
+    // the DLRMv1 MLPs) is staged once, by all epilogue warps, zero-filled to a
+    // multiple of 32 columns; a longer one is staged per tile, each warp its
+    // own slice. (Restaging per tile cost every warp an L2 round trip per tile:
+    // with the ring taking the shared memory, L1 keeps no lines across tiles.)
+    constexpr int kBiasCols = kLinEpiWarps * kColsPerWarp;
+    const bool bias_whole = args.N <= kBiasCols;
+    float* bias_all = reinterpret_cast<float*>(smem + L::kBias);
+    if (bias_whole) {
+      const int n_end = (args.N + 31) & ~31;
+      for (int n = ew * 32 + lane; n < n_end; n += kLinEpiWarps * 32)
+        bias_all[n] = (args.bias != nullptr && n < args.N) ? __ldg(args.bias + n) : 0.f;
+      asm volatile("bar.sync 1, %0;" ::"r"(kLinEpiWarps * 32) : "memory");  // epilogue warps only
+    }
     int j = 0;
     for (int t = unit0; t < args.tiles; t += unit_step, ++j) {
       const int b = j & 1;
       const int m0 = (t / args.tiles_n) * kUnitM + static_cast<int>(rank) * kLinBM;
       const int n0 = (t % args.tiles_n) * BN;
-      for (int c = lane; c < kColsPerWarp; c += 32) {
-        const int n = n0 + c_begin + c;
-        bias_s[c] = (args.bias != nullptr && n < args.N) ? __ldg(args.bias + n) : 0.f;
+      const float* bias_w = bias_whole ? bias_all + n0 + c_begin : bias_s;  // column c_begin
+      if (!bias_whole) {
+        for (int c = lane; c < kColsPerWarp; c += 32) {
+          const int n = n0 + c_begin + c;
+          bias_s[c] = (args.bias != nullptr && n < args.N) ? __ldg(args.bias + n) : 0.f;
+        }
+        __syncwarp();
       }
-      __syncwarp();
       const bool ok =
           __all_sync(0xffffffffu, mbar_wait_bounded(&acc_full[b], (j >> 1) & 1, kLinWaitLimit));
       if (!ok) {
@@ -420,7 +438,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       for (int c0 = c_begin; c0 < c_begin + kColsPerWarp && n0 + c0 < args.N; c0 += 32) {
         float v[32];
         tmem_ld_32x32b_x32(trow + c0, v);
-        const float4* bq = reinterpret_cast<const float4*>(bias_s + (c0 - c_begin));
+        const float4* bq = reinterpret_cast<const float4*>(bias_w + (c0 - c_begin));
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const float4 bb = bq[q];
