@@ -30,6 +30,7 @@
 // DLRM_FLAG_TIMEOUT in the optional status word, ends that role's loop, and
 // the CTA still frees its tensor memory and exits.
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cstdint>
 #include <cstring>
@@ -57,6 +58,7 @@ constexpr int lin_stages() {
 constexpr int kLinEpiWarps = 8;  // two per TMEM lane quarter, each half of the columns
 constexpr int kLinThreads = 64 + 32 * kLinEpiWarps;  // producer warp, MMA warp, epilogue
 constexpr long long kLinWaitLimit = 200000000LL;  // clock cycles, about 0.1 s
+constexpr int kLinMaxDevices = 64;  // devices whose launch set-up is cached
 
 template <int BN, bool F32S, bool PAIR>
 struct LinSmem {
@@ -563,9 +565,24 @@ cudaError_t run_linear(const LinMaps& maps, LinearArgs args, int sms, cudaStream
   auto* fn = &linear_bf16_kernel<BN, ACT, F32S, PAIR>;
   constexpr int smem = LinSmem<BN, F32S, PAIR>::kTotal;
   constexpr int kUnitM = (PAIR ? 2 : 1) * kLinBM;
-  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
+  // Per device, the instance's shared-memory size is set and (pairs) the
+  // resident cluster count queried once: 0 = not yet, else that count + 1.
+  // (Both calls on every launch made a layer cost about 20 us of host time.)
+  static std::atomic<int> prepared[kLinMaxDevices];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    dev = -1;
+  }
+  const bool cacheable = dev >= 0 && dev < kLinMaxDevices;
+  const int cached = cacheable ? prepared[dev].load(std::memory_order_acquire) : 0;
+  cudaError_t e = cudaSuccess;
+  if (cached == 0) {
+    e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
+  int fit = cached > 0 ? cached - 1 : 0;
   args.tiles_n = (args.N + BN - 1) / BN;
   const int64_t tiles = static_cast<int64_t>((args.M + kUnitM - 1) / kUnitM) * args.tiles_n;
   if (tiles > INT32_MAX) return cudaErrorInvalidValue;
@@ -593,13 +610,14 @@ cudaError_t run_linear(const LinMaps& maps, LinearArgs args, int sms, cudaStream
     // free SMs leaves one idle)
     int pairs = sms / 2;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-    int fit = 0;
-    if (cudaOccupancyMaxActiveClusters(&fit, fn, &cfg) == cudaSuccess && fit > 0)
-      pairs = std::min(pairs, fit);
-    else
+    if (cached == 0 && cudaOccupancyMaxActiveClusters(&fit, fn, &cfg) != cudaSuccess) {
       (void)cudaGetLastError();
+      fit = 0;
+    }
+    if (fit > 0) pairs = std::min(pairs, fit);
     grid = 2 * std::min<int64_t>(tiles, pairs);
   }
+  if (cacheable && cached == 0) prepared[dev].store(fit + 1, std::memory_order_release);
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   return cudaLaunchKernelEx(&cfg, fn, maps, args);
 }
