@@ -183,7 +183,25 @@ __device__ __forceinline__ void decode_tiles(uint16_t* tiles, int nT, int tid, i
 // data per feature row, RS float4 per row in shared memory, 2^LQ lanes per
 // tile, tiles from the table decode_tiles wrote. Every shared-memory read of
 // a tile is an immediate offset from one of two base addresses and the column
-// loop is fully unrolled. Same tasks, sums and stores as dots_from_smem.
+// loop is fully unrolled. Same tasks and stores as dots_from_smem; each dot
+// keeps two partial sums (its even and its odd columns) updated by packed
+// two-lane FMAs, added once at the end (measured on B200: the interaction at
+// B=65536, F=26, D=128 332.5 -> 317.4 us; unchanged at B=2048, F=32, D=64).
+
+// Two round-to-nearest f32 fused multiply-adds in one packed instruction
+// (sm_100 fma.rn.f32x2): (d0, d1) = (a0 * b0 + d0, a1 * b1 + d1).
+__device__ __forceinline__ void fma2_rn(float& d0, float& d1, float a0, float a1, float b0,
+                                        float b1) {
+  asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\t"
+      "mov.b64 pb, {%4, %5};\n\t"
+      "mov.b64 pd, {%0, %1};\n\t"
+      "fma.rn.f32x2 pd, pa, pb, pd;\n\t"
+      "mov.b64 {%0, %1}, pd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 template <int D4, int RS, int LQ>
 __device__ __forceinline__ void dots_fixed(const float* feat, const FeatLayout& Lf,
                                            const uint16_t* tiles, int S_here,
@@ -210,9 +228,9 @@ __device__ __forceinline__ void dots_fixed(const float* feat, const FeatLayout& 
     const int I = IJ >> 8, J = IJ & 255;
     const float4* fi = reinterpret_cast<const float4*>(feat) + s * per_sample + 4 * I * RS + q;
     const float4* fj = reinterpret_cast<const float4*>(feat) + s * per_sample + 4 * J * RS + q;
-    float acc[16];
+    float acc2[32];  // per dot, the partial sums of its even and of its odd columns
 #pragma unroll
-    for (int v = 0; v < 16; ++v) acc[v] = 0.f;
+    for (int v = 0; v < 32; ++v) acc2[v] = 0.f;
 #pragma unroll
     for (int it = 0; it < ITER; ++it) {
       if (it * Q + q < D4 || (D4 % Q) == 0) {
@@ -225,15 +243,16 @@ __device__ __forceinline__ void dots_fixed(const float* feat, const FeatLayout& 
         for (int r = 0; r < 4; ++r)
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            float x = acc[4 * r + c];
-            x = fmaf(a[r].x, bv[c].x, x);
-            x = fmaf(a[r].y, bv[c].y, x);
-            x = fmaf(a[r].z, bv[c].z, x);
-            x = fmaf(a[r].w, bv[c].w, x);
-            acc[4 * r + c] = x;
+            float& e = acc2[2 * (4 * r + c)];
+            float& o = acc2[2 * (4 * r + c) + 1];
+            fma2_rn(e, o, a[r].x, a[r].y, bv[c].x, bv[c].y);
+            fma2_rn(e, o, a[r].z, a[r].w, bv[c].z, bv[c].w);
           }
       }
     }
+    float acc[16];
+#pragma unroll
+    for (int v = 0; v < 16; ++v) acc[v] = acc2[2 * v] + acc2[2 * v + 1];
     tile_reduce_store<LQ>(acc, q, active, I, J, Lf.F1, out + (b0 + s) * row_stride + col0);
   }
 }
