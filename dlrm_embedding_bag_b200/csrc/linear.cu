@@ -441,13 +441,23 @@ __global__ void __launch_bounds__(kLinThreads, 1)
         float v[32];
         tmem_ld_32x32b_x32(trow + c0, v);
         const float4* bq = reinterpret_cast<const float4*>(bias_w + (c0 - c_begin));
+        if (ACT != DLRM_ACT_SIGMOID || n0 + c0 + 32 <= args.N) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 bb = bq[q];
-          v[4 * q] = activate<ACT>(__fadd_rn(v[4 * q], bb.x));
-          v[4 * q + 1] = activate<ACT>(__fadd_rn(v[4 * q + 1], bb.y));
-          v[4 * q + 2] = activate<ACT>(__fadd_rn(v[4 * q + 2], bb.z));
-          v[4 * q + 3] = activate<ACT>(__fadd_rn(v[4 * q + 3], bb.w));
+          for (int q = 0; q < 8; ++q) {
+            const float4 bb = bq[q];
+            v[4 * q] = activate<ACT>(__fadd_rn(v[4 * q], bb.x));
+            v[4 * q + 1] = activate<ACT>(__fadd_rn(v[4 * q + 1], bb.y));
+            v[4 * q + 2] = activate<ACT>(__fadd_rn(v[4 * q + 2], bb.z));
+            v[4 * q + 3] = activate<ACT>(__fadd_rn(v[4 * q + 3], bb.w));
+          }
+        } else {
+          // the sigmoid of the columns past N (never stored) is skipped: the
+          // 256 -> 1 output layer would evaluate 32 of them for one
+          const float* bs = reinterpret_cast<const float*>(bq);
+          const int valid = args.N - (n0 + c0);  // 1 .. 31, the same in every lane
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < valid) v[i] = activate<ACT>(__fadd_rn(v[i], bs[i]));
         }
         if (tma_out) {
           if (lane == 0) bulk_wait_read_all();  // the previous block has left the staging
