@@ -468,3 +468,49 @@ def test_linear_cta_pair_tiles(M, N, k_lo, k_hi, mode):
         p = [(_bits(planes[i][rows]).astype(np.uint32) << 16).view(np.float32)
              .astype(np.float64) for i in range(3)]
         assert np.array_equal(p[0] + p[1] + p[2], y32[rows].double().cpu().numpy())
+
+
+# Layers with K <= 16 (the DLRMv1 bottom MLP reads 13 dense features): one
+# zero-filled K block per tile, every output form, the same oracle bounds.
+@pytest.mark.parametrize("M,N,K", [(20000, 512, 13), (777, 1000, 16), (513, 9, 5), (3, 1, 1),
+                                   (100, 2048, 13), (4099, 64, 7)])
+def test_linear_small_k(M, N, K):
+    _run(M, N, K, act="relu", seed=M + N + K)
+
+
+@pytest.mark.parametrize("act", ["none", "relu", "sigmoid"])
+def test_linear_small_k_outputs(act):
+    # bf16 output alone, pitched outputs, no bias, a column count off the 8-wide groups
+    _run(1003, 100, 13, act=act, seed=11, pitch_a=16, pitch_y=104)
+    _run(1003, 100, 13, act=act, bias=False, seed=12)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(13)
+    a = _rand_bf16(g, 515, 13, pitch=16)
+    w = _rand_bf16(g, 77, 13)
+    y32, _ = mlp.linear_bf16(a, w, None, act)
+    _, y16 = mlp.linear_bf16(a, w, None, act, f32=False, bf16=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bits(y16), _bits(y32.to(torch.bfloat16)))
+
+
+@pytest.mark.parametrize("M,N,K", [(20000, 512, 13), (300, 1000, 16), (65, 9, 3)])
+@pytest.mark.parametrize("wdt", ["bf16", "f32"])
+@pytest.mark.parametrize("act", ["relu", "sigmoid"])
+def test_linear_f32a_small_k(M, N, K, wdt, act):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(M + N + K + (wdt == "f32"))
+    a = _rand_f32(g, M, K)
+    b = torch.empty(N, device=DEV).normal_(0, 0.5, generator=g)
+    if wdt == "bf16":
+        w = _rand_bf16(g, N, K, K ** -0.5)
+        wk = w
+    else:
+        w = _rand_f32(g, N, K, K ** -0.5)
+        wk = mlp.split_bf16x3(w)
+    y32, planes = mlp.linear_f32a(mlp.split_bf16x3(a), wk, b, act, planes=True)
+    torch.cuda.synchronize()
+    _check_f32a(y32, a, w, b, act, w_planes=1 if wdt == "bf16" else 3,
+                what=f"M={M} N={N} K={K} {wdt} weights {act}")
+    p = [(_bits(planes[i]).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+         for i in range(3)]
+    assert np.array_equal(p[0] + p[1] + p[2], y32.double().cpu().numpy())
