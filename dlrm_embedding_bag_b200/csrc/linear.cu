@@ -7,14 +7,16 @@
 // t = c, c + gridDim.x, ... (N tiles fastest, so CTAs running side by side
 // share A rows in L2). Ten warps:
 //   - warp 0 (one thread) streams 64-wide K blocks of A (128 x 64 bf16) and W
-//     (BN x 64) into a 3- or 4-stage shared-memory ring with 2-D TMA loads (128-byte
-//     swizzle), running ahead across tiles; K blocks 0..nkb_lo-1 read A_lo,
-//     the rest read A_hi, and W's column offset follows, so the
-//     concatenation is never built;
+//     (BN x 64) into a shared-memory ring (3 to 6 stages, by stage size) with 2-D
+//     TMA loads (128-byte swizzle), running ahead across tiles; K blocks
+//     0..nkb_lo-1 read A_lo, the rest read A_hi, and W's column offset follows,
+//     so the concatenation is never built. An f32-activation operand is three
+//     bf16 planes: on CTA pairs a stage holds a K block's three plane boxes next
+//     to the W box they share;
 //   - warp 1 allocates tensor memory for two f32 accumulators (2 x BN
-//     columns) and one thread issues four tcgen05.mma (K = 16 each) per
-//     stage into the tile's accumulator, committing each stage back to the
-//     producer and each finished accumulator to the epilogue;
+//     columns) and one thread issues four tcgen05.mma (K = 16 each) per A box
+//     of a stage into the tile's accumulator, committing each stage back to
+//     the producer and each finished accumulator to the epilogue;
 //   - warps 2-9 read the finished accumulator (warp w owns TMEM lanes
 //     32*(w%4)..+31 and half of the columns), add the bias, apply the
 //     activation and store f32 and/or bf16, then hand the accumulator back -
