@@ -514,3 +514,23 @@ def test_linear_f32a_small_k(M, N, K, wdt, act):
     p = [(_bits(planes[i]).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
          for i in range(3)]
     assert np.array_equal(p[0] + p[1] + p[2], y32.double().cpu().numpy())
+
+
+@pytest.mark.parametrize("M,N,k_lo,k_hi", [(40000, 256, 512, 0), (20100, 200, 64, 960)])
+def test_linear_f32a_cta_pairs_f32_weights(M, N, k_lo, k_hi):
+    """f32 activations against f32 weights (three weight planes, six plane
+    products) on CTA pairs, where each stage holds one A plane: the path the
+    bf16-weight layers leave for stages with all three A planes."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(M + N + 3)
+    K = k_lo + k_hi
+    b = torch.empty(N, device=DEV).normal_(0, 0.5, generator=g)
+    w = _rand_f32(g, N, K, K ** -0.5)
+    a_lo = _rand_f32(g, M, k_lo)
+    a_hi = _rand_f32(g, M, k_hi) if k_hi else None
+    rows = _pair_rows(M, 64, M + 1)
+    y32, _ = mlp.linear_f32a(mlp.split_bf16x3(a_lo), mlp.split_bf16x3(w), b, "relu",
+                             a_hi=None if a_hi is None else mlp.split_bf16x3(a_hi))
+    torch.cuda.synchronize()
+    _check_f32a(y32, a_lo, w, b, "relu", a_hi=a_hi, rows=rows, w_planes=3,
+                what=f"f32a pair, f32 weights, M={M} N={N} K={k_lo}+{k_hi}")
