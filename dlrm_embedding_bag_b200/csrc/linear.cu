@@ -11,8 +11,8 @@
 //     TMA loads (128-byte swizzle), running ahead across tiles; K blocks
 //     0..nkb_lo-1 read A_lo, the rest read A_hi, and W's column offset follows,
 //     so the concatenation is never built. An f32-activation operand is three
-//     bf16 planes: on CTA pairs a stage holds a K block's three plane boxes next
-//     to the W box they share;
+//     bf16 planes: a stage holds a K block's three plane boxes next to the W
+//     box they share;
 //   - warp 1 allocates tensor memory for two f32 accumulators (2 x BN
 //     columns) and one thread issues four tcgen05.mma (K = 16 each) per A box
 //     of a stage into the tile's accumulator, committing each stage back to
@@ -52,10 +52,12 @@ constexpr int kLinBK = 64;     // K per stage: 64 bf16 = one 128-byte swizzle ro
 // stages) next to the f32 output staging, where only 3 fit; CTA pairs hold
 // half of the W rows per stage (32 KB stages at BN = 256): 6 stages, 5 next
 // to the f32 staging. With the three planes of an f32-activation operand in
-// one stage (AG = 3: 64 KB stages on pairs), 3 stages, 2 next to the staging.
+// one stage (AG = 3: 64 KB stages on pairs, 56 or 64 KB on one CTA at 64 or
+// 128 columns), 3 stages, 2 next to the f32 staging at 128 columns or more.
 template <int BN, bool F32S, bool PAIR, int AG>
 constexpr int lin_stages() {
   if constexpr (PAIR && AG == 3) return F32S ? 2 : 3;
+  if constexpr (AG == 3) return (BN >= 128 && F32S) ? 2 : 3;
   if constexpr (PAIR) return F32S ? 5 : 6;
   return (BN >= 256 && F32S) ? 3 : 4;
 }
@@ -316,7 +318,9 @@ __global__ void __launch_bounds__(kLinThreads, 1)
                              n0 + static_cast<int>(rank) * (BN / 2));
           } else {
             mbar_arrive_expect_tx(&full[s], L::kStage);
-            tma_load_2d(sa, &maps.a[sg.a], &full[s], sg.a_k0 + kk, m0);
+#pragma unroll
+            for (int i = 0; i < AG; ++i)
+              tma_load_2d(sa + i * L::kA, &maps.a[sg.a + i], &full[s], sg.a_k0 + kk, m0);
             tma_load_2d(sb, &maps.w[sg.w], &full[s], sg.w_k0 + kk, n0);
           }
         }
@@ -759,12 +763,14 @@ int launch_layer(const APart* parts, int nparts, int a_planes, const uint16_t* w
   // Products summed: A plane i times W plane j for i + j < 3 (all three A
   // planes against a single weight plane; against three weight planes the six
   // products whose planes' leading bits lie within 2^-16 of the value's).
-  // Three A planes against one weight plane on CTA pairs load the planes into
-  // one stage next to the W block they share (AG = 3): a third of the W
-  // bytes per tile. Measured on B200 at B=65536 (f32 activations, bf16
-  // weights): top layer 0 (30 K blocks per tile) 106.5 -> 98.3 us, the
-  // 13 -> 512 layer 53.3 -> 49.1 us, the 512 -> 256 layers unchanged.
-  const bool group_planes = a_planes == 3 && w_planes == 1 && pair;
+  // Three A planes against one weight plane load the planes into one stage
+  // next to the W block they share (AG = 3): a third of the W bytes per tile.
+  // Not at 256 columns on one CTA (an 80 KB stage leaves too shallow a ring).
+  // Measured on B200 (f32 activations, bf16 weights): at B=65536 top layer 0
+  // (pairs, 30 K blocks per tile) 106.5 -> 98.3 us, the 13 -> 512 layer 53.3 ->
+  // 49.1 us, the 64-column layers 34.8 -> 30.7 us; at B=2048 (one CTA per
+  // tile) every layer 1.5-3 us faster, the f32 forward graph 112.6 -> 101.6 us.
+  const bool group_planes = a_planes == 3 && w_planes == 1 && (pair || bn <= 128);
   int w_off = 0;
   for (int p = 0; p < nparts && group_planes; ++p) {
     const int nkb = static_cast<int>((parts[p].k + kLinBK - 1) / kLinBK);
@@ -816,8 +822,14 @@ int launch_layer(const APart* parts, int nparts, int a_planes, const uint16_t* w
           : group_planes ? run_linear_bn<256, true, 3>(act, maps, args, sms, stream)
                          : run_linear_bn<256, true>(act, maps, args, sms, stream);
       break;
-    case 128: e = run_linear_bn<128>(act, maps, args, sms, stream); break;
-    default: e = run_linear_bn<64>(act, maps, args, sms, stream); break;
+    case 128:
+      e = group_planes ? run_linear_bn<128, false, 3>(act, maps, args, sms, stream)
+                       : run_linear_bn<128>(act, maps, args, sms, stream);
+      break;
+    default:
+      e = group_planes ? run_linear_bn<64, false, 3>(act, maps, args, sms, stream)
+                       : run_linear_bn<64>(act, maps, args, sms, stream);
+      break;
   }
   if (e != cudaSuccess) return cuda_fail(e);
   note_launch();
